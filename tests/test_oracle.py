@@ -1,0 +1,394 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these re-types an oracle formula: each pins a function against a
+closed form worked by hand (tests/golden), an invariant the pages state, a
+textbook value, or a brute-force loop over tiny inputs written independently of
+numpy.  Chosen so that a dropped term, a wrong sign or index, or a transposed
+operand fails at least one test.
+"""
+import math
+import os
+import random
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# ------------------------------------------------------------------ partition
+
+def test_partition_gqa_closed_form():
+    p = O.partition_subparams([4096, 1024, 1024], 8, 128)
+    for row in _golden_rows("partition_gqa_tp8.txt"):
+        r, *v = [int(t) for t in row]
+        assert p.width[r] == v[0:3]
+        assert p.src_off[r] == v[3:6]
+        assert p.dst_off[r] == v[6:9]
+        assert p.shard_width[r] == v[9]
+        assert p.shard_base[r] == v[10]
+
+
+def test_partition_single_subparam_configs():
+    # nanotron MLP Module: the column output per rank is intermediate // tp.
+    for inter, tp in [(1024, 4), (14336, 8), (28672, 8)]:
+        p = O.partition_subparams([inter], tp, 1)
+        assert p.shard_width == [inter // tp] * tp
+        assert p.src_off == [[r * inter // tp] for r in range(tp)]
+
+
+def _brute_partition(sub_sizes, tp, align):
+    """Independent enumeration: deal units round-robin, then lay blocks out in rank order."""
+    owners = []  # per sub-param: owner rank of every row
+    for s in sub_sizes:
+        units = s // align
+        count = [0] * tp
+        for u in range(units):
+            count[u % tp] += 1
+        row_owner = []
+        for r in range(tp):
+            row_owner += [r] * (count[r] * align)
+        owners.append(row_owner)
+    return owners
+
+
+@pytest.mark.parametrize("align", [1, 2, 4])
+def test_partition_brute_force(align):
+    rng = random.Random(1)
+    cases = 0
+    for tp in range(1, 9):
+        for n_sub in range(1, 4):
+            for _ in range(25):
+                subs = [align * rng.randint(1, 32 // align) for _ in range(n_sub)]
+                if any(s // align < tp for s in subs):
+                    with pytest.raises(O.OracleError) as e:
+                        O.partition_subparams(subs, tp, align)
+                    assert e.value.kind == "INDIVISIBLE"
+                    continue
+                p = O.partition_subparams(subs, tp, align)
+                owners = _brute_partition(subs, tp, align)
+                start = 0
+                seen = []
+                for j, s in enumerate(subs):
+                    for r in range(tp):
+                        rows = [start + i for i, o in enumerate(owners[j]) if o == r]
+                        assert p.width[r][j] == len(rows)
+                        assert p.src_off[r][j] == rows[0]
+                        assert rows == list(range(rows[0], rows[0] + len(rows)))
+                    start += s
+                # concatenating every shard's rows covers the fused weight exactly once
+                for r in range(tp):
+                    col = 0
+                    for j in range(n_sub):
+                        assert p.dst_off[r][j] == col
+                        seen += list(range(p.src_off[r][j], p.src_off[r][j] + p.width[r][j]))
+                        col += p.width[r][j]
+                    assert p.shard_width[r] == col
+                assert sorted(seen) == list(range(sum(subs)))
+                assert sum(p.shard_width) == sum(subs)
+                assert p.shard_base == [sum(p.shard_width[:r]) for r in range(tp)]
+                cases += 1
+    assert cases > 100
+
+
+def test_partition_errors():
+    for args, kind in [(([4096], 0, 1), "SHAPE"), (([4096], 65, 1), "SHAPE"),
+                       (([], 2, 1), "SHAPE"), (([1] * 9, 1, 1), "SHAPE"),
+                       (([0], 1, 1), "SHAPE"), (([100], 2, 0), "SHAPE"),
+                       (([100], 2, 3), "INDIVISIBLE"), (([128], 2, 128), "INDIVISIBLE"),
+                       (([3], 4, 1), "INDIVISIBLE")]:
+        with pytest.raises(O.OracleError) as e:
+            O.partition_subparams(*args)
+        assert e.value.kind == kind, args
+
+
+def test_bias_size_rule():
+    p = O.partition_subparams([8, 4, 4], 2, 1)
+    O.check_bias_size(p, 16)
+    with pytest.raises(O.OracleError):
+        O.check_bias_size(p, 15)
+
+
+# ----------------------------------------------------------------------- GELU
+
+def test_gelu_erf_textbook_phi():
+    for y, phi in (_golden_rows("normal_cdf.txt")):
+        y, phi = float(y), float(phi)
+        assert O.gelu_erf(np.array([y]))[0] == pytest.approx(y * phi, rel=1e-14, abs=1e-16)
+
+
+def test_gelu_identities():
+    y = np.linspace(-7.0, 7.0, 2801)
+    for f in (O.gelu_erf, O.gelu_tanh):
+        assert f(np.array([0.0]))[0] == 0.0
+        # Phi(y) + Phi(-y) = 1 and tanh odd  =>  gelu(y) - gelu(-y) = y
+        np.testing.assert_allclose(f(y) - f(-y), y, rtol=0, atol=1e-13)
+        big = np.array([12.0, 30.0])
+        np.testing.assert_allclose(f(big), big, rtol=1e-15)
+        np.testing.assert_allclose(f(-big), 0.0, atol=1e-12)
+    # the tanh form approximates the erf form closely but is a different function
+    d = np.abs(O.gelu_tanh(y) - O.gelu_erf(y))
+    assert 1e-4 < d.max() < 5e-4
+
+
+# --------------------------------------------------------------------- column
+
+def _brute_column(x, w, b, part, act):
+    """Triple loop over python floats, written from the definition."""
+    M, K = len(x), len(x[0])
+    act_f = {"none": lambda v: v,
+             "gelu_erf": lambda v: 0.5 * v * (1 + math.erf(v / math.sqrt(2))),
+             "gelu_tanh": lambda v: 0.5 * v * (1 + math.tanh(math.sqrt(2 / math.pi)
+                                                             * (v + 0.044715 * v ** 3)))}[act]
+    out = []
+    for r in range(part.tp):
+        y = [[None] * part.shard_width[r] for _ in range(M)]
+        for j in range(len(part.sub_sizes)):
+            for c in range(part.width[r][j]):
+                n = part.src_off[r][j] + c
+                for m in range(M):
+                    s = 0.0
+                    for k in range(K):
+                        s += x[m][k] * w[n][k]
+                    if b is not None:
+                        s += b[n]
+                    y[m][part.dst_off[r][j] + c] = act_f(s)
+        out.append(np.array(y))
+    return out
+
+
+@pytest.mark.parametrize("act", ["none", "gelu_erf", "gelu_tanh"])
+def test_column_brute_force(act):
+    rng = np.random.default_rng(3)
+    for subs, tp, align, M, K in [([12, 6, 6], 3, 2, 5, 7), ([10], 4, 1, 3, 9), ([8, 4], 1, 1, 2, 3)]:
+        p = O.partition_subparams(subs, tp, align)
+        x = rng.standard_normal((M, K))
+        w = rng.standard_normal((sum(subs), K))
+        b = rng.standard_normal(sum(subs))
+        got = O.column_linear(x, w, b, p, act)
+        ref = _brute_column(x.tolist(), w.tolist(), b.tolist(), p, act)
+        for g, r in zip(got, ref):
+            np.testing.assert_allclose(g, r, rtol=1e-12, atol=1e-12)
+
+
+def test_column_concat_of_shards_is_unsharded_matmul():
+    # SubParamLinearLayer.gather_params / nanotron: shards put back together give
+    # the unsharded linear.  Scatter each piece back to its fused rows.
+    rng = np.random.default_rng(4)
+    subs, tp = [4096 // 16, 1024 // 16, 1024 // 16], 8
+    p = O.partition_subparams(subs, tp, 8)
+    x = rng.standard_normal((6, 40))
+    w = rng.standard_normal((sum(subs), 40))
+    b = rng.standard_normal(sum(subs))
+    shards = O.column_linear(x, w, b, p)
+    full = np.zeros((6, sum(subs)))
+    for r in range(tp):
+        for j in range(3):
+            s, d, n = p.src_off[r][j], p.dst_off[r][j], p.width[r][j]
+            full[:, s:s + n] = shards[r][:, d:d + n]
+    np.testing.assert_allclose(full, x @ w.T + b, rtol=1e-13, atol=1e-13)
+
+
+def test_column_tp1_is_plain_linear_and_identity_weight_copies():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, 6))
+    p = O.partition_subparams([6], 1, 1)
+    y = O.column_linear(x, np.eye(6), None, p)[0]
+    np.testing.assert_array_equal(y, x)
+    w = rng.standard_normal((3, 6))
+    p = O.partition_subparams([3], 1, 1)
+    y = O.column_linear(x, w, None, p)[0]
+    assert y[1, 2] == pytest.approx(sum(x[1, k] * w[2, k] for k in range(6)), rel=1e-14)
+
+
+def test_column_rejects_bias_size():
+    p = O.partition_subparams([4, 4], 2, 1)
+    with pytest.raises(O.OracleError):
+        O.column_linear(np.ones((1, 2)), np.ones((8, 2)), np.ones(7), p)
+
+
+# ------------------------------------------------------------------------ row
+
+def test_row_brute_force_and_partials_sum_to_full_product():
+    rng = np.random.default_rng(6)
+    M, N, kw = 3, 5, [4, 3, 3, 2]
+    K = sum(kw)
+    hfull = rng.standard_normal((M, K))
+    w2 = rng.standard_normal((N, K))
+    b = rng.standard_normal(N)
+    res = rng.standard_normal((M, N))
+    h, off = [], 0
+    for k in kw:
+        h.append(hfull[:, off:off + k])
+        off += k
+    w2s = O.row_weight_slices(w2, kw)
+    y = O.row_linear_reduce(h, w2s, b, res)
+    # brute force: one loop over the whole contraction dim
+    for m in range(M):
+        for n in range(N):
+            s = sum(hfull[m][k] * w2[n][k] for k in range(K))
+            assert y[m, n] == pytest.approx(s + b[n] + res[m, n], rel=1e-12, abs=1e-12)
+    # o_wo: the per-shard partials are {unreduced}; their sum is the full product
+    parts = O.row_partials(h, w2s)
+    np.testing.assert_allclose(sum(parts), hfull @ w2.T, rtol=1e-13, atol=1e-13)
+    # each partial only sees its own slice: zeroing rank 1's slice drops exactly P_1
+    h0 = [a.copy() for a in h]
+    h0[1][:] = 0
+    np.testing.assert_allclose(O.row_linear_reduce(h0, w2s), sum(parts) - parts[1], atol=1e-12)
+    # tp = 1 is the plain linear
+    np.testing.assert_allclose(O.row_linear_reduce([hfull], [w2]), hfull @ w2.T, rtol=1e-14)
+
+
+# -------------------------------------------------------------------- RMSNorm
+
+def test_rmsnorm_constant_row_closed_form():
+    for c in [1e-4, 0.5, 3.0, -2.0]:
+        y = O.rmsnorm(np.full((1, 16), c), eps=1e-6)
+        np.testing.assert_allclose(y, c / math.sqrt(c * c + 1e-6), rtol=1e-14)
+    # epsilon sits inside the square root: c=1e-3 gives 1/sqrt(2), not 1e-3/(1e-3+1e-6)
+    assert O.rmsnorm(np.full((1, 4), 1e-3))[0, 0] == pytest.approx(1 / math.sqrt(2), rel=1e-12)
+
+
+def test_rmsnorm_invariants_and_brute_force():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((5, 33)) * 3
+    y = O.rmsnorm(x)
+    ms = (x * x).mean(axis=1)
+    np.testing.assert_allclose((y * y).mean(axis=1), ms / (ms + 1e-6), rtol=1e-12)
+    np.testing.assert_allclose(O.rmsnorm(7.0 * x, eps=0.0), O.rmsnorm(x, eps=0.0), rtol=1e-13)
+    s = rng.standard_normal(33) * 0.1
+    np.testing.assert_allclose(O.rmsnorm(x, s, centered=True), O.rmsnorm(x, 1.0 + s), rtol=1e-14)
+    np.testing.assert_allclose(O.rmsnorm(x, s, centered=False), y * s, rtol=1e-14)
+    for m in range(5):
+        acc = 0.0
+        for v in x[m]:
+            acc += v * v
+        inv = 1.0 / math.sqrt(acc / 33 + 1e-6)
+        for h in range(33):
+            assert O.rmsnorm(x, s, True)[m, h] == pytest.approx(x[m, h] * inv * (1 + s[h]),
+                                                                 rel=1e-12)
+
+
+# -------------------------------------------------------------------- LM head
+
+def test_vocab_layout_closed_forms():
+    for row in _golden_rows("vocab_layout.txt"):
+        V, tp, n = int(row[0]), int(row[1]), int(row[2])
+        if row[3] == "error":
+            with pytest.raises(O.OracleError):
+                O.vocab_layout(V, tp, n)
+            continue
+        lay = O.vocab_layout(V, tp, n)
+        assert lay.shard == int(row[3])
+        assert lay.split_sizes == [int(t) for t in row[4].split(",")]
+        assert lay.global_id(int(row[5]), int(row[6]), int(row[7])) == int(row[8])
+
+
+def _brute_argmax(x, w, tp, shard):
+    B, V = len(x), len(w)
+    best = []
+    for b in range(B):
+        per = []
+        for r in range(tp):
+            bi, bv = -1, -math.inf
+            for v in range(r * shard, min((r + 1) * shard, V)):
+                s = sum(x[b][k] * w[v][k] for k in range(len(x[b])))
+                if s > bv:
+                    bi, bv = v, s
+            per.append((bv, bi))
+        g = max(range(tp), key=lambda r: (per[r][0], -per[r][1]))
+        best.append((per, per[g][1]))
+    return best
+
+
+def test_lmhead_brute_force():
+    rng = np.random.default_rng(8)
+    for B, K, V, tp, n in [(3, 5, 37, 4, 2), (2, 4, 9, 8, 1), (1, 3, 16, 2, 4)]:
+        x = rng.standard_normal((B, K))
+        w = rng.standard_normal((V, K))
+        res = O.lmhead_argmax(x, w, tp, n)
+        lay = O.vocab_layout(V, tp, n)
+        ref = _brute_argmax(x.tolist(), w.tolist(), tp, lay.shard)
+        for b in range(B):
+            per, gid = ref[b]
+            assert res.ids[b] == gid
+            for r in range(tp):
+                assert res.shard_idx[r, b] == per[r][1]
+                if per[r][1] < 0:
+                    assert res.shard_max[r, b] == -math.inf
+                else:
+                    assert res.shard_max[r, b] == pytest.approx(per[r][0], rel=1e-12)
+
+
+def test_lmhead_planted_maximum_and_ties():
+    rng = np.random.default_rng(9)
+    B, K, V, tp, n = 4, 16, 203, 8, 3
+    lay = O.vocab_layout(V, tp, n)
+    x = rng.standard_normal((B, K))
+    w = rng.standard_normal((V, K)) * 0.01
+    planted = [lay.shard - 1, lay.shard, V - 1, 2 * lay.shard + lay.split_sizes[0]]
+    for b, v in enumerate(planted):
+        w[v] = 2.0 * x[b] / np.linalg.norm(x[b])
+    res = O.lmhead_argmax(x, w, tp, n)
+    assert list(res.ids) == planted
+    # an exact tie goes to the lowest id, also across shards
+    w2 = w.copy()
+    w2[5] = w2[planted[0]]
+    res = O.lmhead_argmax(x, w2, tp, n)
+    assert res.ids[0] == 5
+    assert res.shard_idx[0, 0] == 5
+    # equal maxima on shards 1 and 3: the lower global id (shard 1) is reported
+    w3 = w.copy()
+    w3[3 * lay.shard + 2] = w3[planted[1]]
+    res = O.lmhead_argmax(x, w3, tp, n)
+    assert res.ids[1] == planted[1]
+    assert res.shard_idx[3, 1] == 3 * lay.shard + 2
+
+
+def test_lmhead_empty_shard():
+    x = np.ones((1, 2))
+    w = np.arange(18.0).reshape(9, 2)
+    res = O.lmhead_argmax(x, w, 8, 1)          # shard 2: ids 0..7 on shards 0..3, id 8 on 4
+    assert list(res.shard_idx[:, 0]) == [1, 3, 5, 7, 8, -1, -1, -1]
+    assert res.shard_max[5, 0] == -math.inf
+    assert res.ids[0] == 8
+
+
+# ---------------------------------------------------------------- stack / MLP
+
+def test_mlp_tp_invariance_and_stack_composition():
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((4, 16))
+    w1 = rng.standard_normal((32, 16)) * 0.2
+    w2 = rng.standard_normal((16, 32)) * 0.2
+    s = rng.standard_normal(16) * 0.1
+    ref = None
+    for tp in (1, 2, 4, 8):
+        y = O.tp_mlp(x, w1, w2, tp, "gelu_erf", scale=s, centered=True, norm=True)
+        if ref is None:
+            # tp = 1 written out: gelu(norm(x) W1^T) W2^T
+            xn = x / np.sqrt((x * x).mean(1, keepdims=True) + 1e-6) * (1 + s)
+            ref = O.gelu_erf(xn @ w1.T) @ w2.T
+        np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+    layers = [(w1, w2, None), (w1 * 0.5, w2 * 2.0, None)]
+    z = O.tp_stack(x, layers, 4, "gelu_erf")
+    z1 = x + O.tp_mlp(x, w1, w2, 1, "gelu_erf", norm=True)
+    z2 = z1 + O.tp_mlp(z1, w1 * 0.5, w2 * 2.0, 1, "gelu_erf", norm=True)
+    np.testing.assert_allclose(z, z2, rtol=1e-12, atol=1e-12)
+
+
+def test_rel_frobenius():
+    o = np.array([3.0, 4.0])
+    assert O.rel_frobenius(o + np.array([0.0, 0.5]), o) == pytest.approx(0.1)
