@@ -1,0 +1,227 @@
+/*
+ * tpl.h -- C ABI of the tensor-parallel sharded-linear library for B200 (sm_100a).
+ *
+ * One GPU computes every tensor-parallel (TP) shard of a transformer block's
+ * linear layers locally.  The calls follow the shapes of the pages they come
+ * from:
+ *
+ *   - nanotron rules, "Tensor-Parallel Component Patterns" (sections
+ *     "Attention Module" and "MLP Module"): TP linears take the full logical
+ *     dimensions plus the TP size and shard internally; c_fc is column-parallel
+ *     with intermediate/tp columns per rank, then GELU, then the row-parallel
+ *     c_proj.  Hidden states arrive as [batch, seq, hidden]; this ABI takes the
+ *     flattened row count M = batch * seq.
+ *   - DeepSpeed "Class SubParamLinearLayer": a fused weight made of several
+ *     logical sub-parameters (fused QKV, unequal GQA widths) partitioned one
+ *     by one along the output dim; forward is matmul(input, W^T) + bias; the
+ *     bias must match the output size.
+ *   - google-research two_d_parallel_xmap.py: allgather_layernorm (RMSNorm,
+ *     epsilon inside the rsqrt, optional centred scale), the o_wo section
+ *     (per-shard partial products summed over the sharded contraction) and
+ *     the residual section; unembed_manual (fp32 logits).
+ *   - Tenstorrent lm_head_1d.py: vocab-sharded, chunked LM head
+ *     (LMHead1D.from_model_args split sizes); the argmax over shards, left to
+ *     the caller there, is fused on the device here.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *     the library never frees or keeps them.  Pointers marked "host" are read
+ *     during the call only.
+ *   - Matrices are dense and row-major; weights use the nn.Linear layout
+ *     [out][in], so both GEMM operands are K-contiguous.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Device
+ *     work is enqueued on it and the call returns without waiting.  Argument
+ *     checks happen on the host before anything is enqueued; a rejected call
+ *     enqueues nothing.
+ *   - bf16 in -> bf16 out with fp32 accumulation and fp32 epilogue maths;
+ *     fp32 in -> fp32 out.
+ *   - A kernel that gives up waiting on its own pipeline records
+ *     TPL_ERR_TIMEOUT in a per-device status word; tpl_get_device_status reads
+ *     and clears it.
+ *   - The library allocates no device memory.  The calls are thread-safe.
+ */
+#ifndef TPL_H
+#define TPL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TPL_OK = 0,
+  TPL_ERR_NULL = 1,         /* a required pointer is NULL                          */
+  TPL_ERR_SHAPE = 2,        /* a size is out of range or sizes disagree            */
+  TPL_ERR_INDIVISIBLE = 3,  /* a partition leaves a rank without rows, or a size
+                               is not a multiple of the alignment unit             */
+  TPL_ERR_DTYPE = 4,        /* unknown dtype or activation                         */
+  TPL_ERR_ALIGN = 5,        /* a pointer or row stride breaks the 16-byte rule     */
+  TPL_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed                   */
+  TPL_ERR_TIMEOUT = 7,      /* a kernel gave up waiting on its pipeline            */
+  TPL_ERR_UNSUPPORTED = 8   /* valid request outside what this build implements    */
+} tpl_status;
+
+typedef enum { TPL_FP32 = 0, TPL_BF16 = 1 } tpl_dtype;
+
+typedef enum {
+  TPL_ACT_NONE = 0,
+  TPL_ACT_GELU_ERF = 1,   /* 0.5 y (1 + erf(y / sqrt 2))                           */
+  TPL_ACT_GELU_TANH = 2   /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3)))       */
+} tpl_act;
+
+#define TPL_MAX_TP 64
+#define TPL_MAX_SUB 8
+
+/*
+ * Per-rank layout of a column-parallel fused weight (caller-owned POD).
+ * For rank r and sub-parameter j: rows src_off[r][j] .. + width[r][j] of the
+ * fused weight (and the same entries of the fused bias) produce columns
+ * dst_off[r][j] .. of rank r's shard.  shard_base[r] is the sum of the shard
+ * widths of the lower ranks.
+ */
+typedef struct {
+  int32_t tp_size;
+  int32_t n_sub;
+  int64_t logical_out;
+  int64_t width[TPL_MAX_TP][TPL_MAX_SUB];
+  int64_t src_off[TPL_MAX_TP][TPL_MAX_SUB];
+  int64_t dst_off[TPL_MAX_TP][TPL_MAX_SUB];
+  int64_t shard_width[TPL_MAX_TP];
+  int64_t shard_base[TPL_MAX_TP];
+} tpl_partition;
+
+/*
+ * Sub-parameter partition (DeepSpeed "Class SubParamLinearLayer": the shape
+ * spec (n, -1) / ((q, k, v), -1) with partition_dim 0; nanotron "MLP Module":
+ * intermediate // tp columns per rank).  Host only, no device work.
+ *
+ *   sub_sizes  host, [n_sub] logical output sizes in the fused order (q, k, v).
+ *   n_sub      1 .. TPL_MAX_SUB.     tp_size  1 .. TPL_MAX_TP.
+ *   align      rows per indivisible unit (head_dim for attention, 1 for MLP).
+ *   out        host, filled on success; untouched on error.
+ *
+ * Each sub-parameter is cut into sub_sizes[j] / align units; rank r gets
+ * units / tp + (r < units % tp) of them.  Errors: TPL_ERR_NULL,
+ * TPL_ERR_SHAPE (counts or sizes out of range), TPL_ERR_INDIVISIBLE (size not
+ * a multiple of align, or a rank left with zero rows of some sub-parameter).
+ */
+tpl_status tpl_partition_subparams(const int64_t* sub_sizes, int32_t n_sub, int32_t tp_size,
+                                   int64_t align, tpl_partition* out);
+
+/*
+ * Column-parallel linear with sub-parameter partitioning, bias and activation
+ * fused in the epilogue (SubParamLinearLayer.forward; nanotron c_fc + F.gelu).
+ *
+ *   p      host, a partition from tpl_partition_subparams.
+ *   x      device, [M][K] activations (dtype dt).
+ *   w      device, [p->logical_out][K] fused weight, nn.Linear layout.
+ *   bias   device, [p->logical_out] in the fused order, or NULL.
+ *   y      device; rank r's shard is the row-major [M][shard_width[r]] block
+ *          starting at element M * shard_base[r].
+ *   Y_r = act(X W_r^T + b_r).  M == 0 is a no-op (x, w, y may then be NULL).
+ *
+ * bf16 runs on the tcgen05 tensor cores and needs K % 8 == 0 and 16-byte
+ * aligned x and w (else TPL_ERR_ALIGN); fp32 runs on the CUDA cores.
+ */
+tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                             const void* w, const void* bias, tpl_dtype dt, tpl_act act,
+                             void* y, void* stream);
+
+/*
+ * Row-parallel linear whose per-shard partial products are reduced on the
+ * device inside the GEMM (google-research o_wo section; nanotron c_proj):
+ *   Y = sum_{r=0}^{tp-1} H_r W2_r^T (+ bias) (+ residual)
+ * The shards are consecutive stretches of one fp32 accumulator, so the sum is
+ * taken in rank order with no extra pass.
+ *
+ *   h         device; rank r's block [M][k_w[r]] starts at element
+ *             M * sum_{q<r} k_w[q] (the layout tpl_column_linear writes).
+ *   k_w       host, [tp] contraction width of each rank.
+ *   w         device; rank r's block [N][k_w[r]] starts at element
+ *             N * sum_{q<r} k_w[q] (columns of the unsharded [N][K] weight).
+ *   bias      device [N] or NULL, added once after the sum.
+ *   residual  device [M][N] or NULL; may alias y (x <- x + f(x)).
+ *   y         device [M][N].
+ *   partials  device [tp][M][N] fp32 or NULL.  When given, each rank's
+ *             partial product is also written out unreduced (a check of the
+ *             reduction; slower: one extra pass per rank).
+ *   M == 0 is a no-op (h, w, y may then be NULL).
+ *
+ * bf16 needs every k_w[r] % 8 == 0 and 16-byte aligned h and w.
+ */
+tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
+                                 int64_t N, const void* w, const void* bias,
+                                 const void* residual, tpl_dtype dt, void* y, float* partials,
+                                 void* stream);
+
+/*
+ * RMSNorm (google-research allgather_layernorm; weight-gathered layernorm):
+ *   y = x / sqrt(mean(x^2) + eps) * g,  g = 1 + scale (centered != 0),
+ *   g = scale (centered == 0), or g = 1 (scale == NULL).
+ * fp32 maths, one rounding on store.
+ *
+ *   x      device [M][H];  y  device [M][H], may alias x.
+ *   scale  device fp32 [H] or NULL.
+ *   M == 0 is a no-op (x, y may then be NULL).
+ */
+tpl_status tpl_rmsnorm(const void* x, int64_t M, int64_t H, const float* scale, int32_t centered,
+                       float eps, tpl_dtype dt, void* y, void* stream);
+
+/*
+ * Bytes of device workspace tpl_lmhead_argmax needs for B rows and tp shards.
+ * Errors as for tpl_lmhead_argmax's shape checks.
+ */
+tpl_status tpl_lmhead_workspace_size(int64_t B, int64_t V, int32_t tp, int32_t n_chunks,
+                                     size_t* bytes);
+
+/*
+ * Decode LM head over a vocab split into tp shards of n_chunks chunks
+ * (Tenstorrent LMHead1D; google-research unembed_manual), with the per-shard
+ * and the global argmax fused in.
+ *
+ * Layout (LMHead1D.from_model_args with tile 1): shard = ceil(V / tp);
+ * chunk_cols = ceil(shard / n_chunks); split sizes [chunk_cols] * (n - 1) +
+ * [shard - sum]; the call is rejected (TPL_ERR_SHAPE) unless that gives exactly
+ * n_chunks splits with a positive last one.  Column j of chunk c on shard r
+ * is global id r * shard + sum(split[:c]) + j; ids >= V are padding and never
+ * reported.
+ *
+ *   x          device bf16 [B][K], 1 <= B <= 256, K % 8 == 0.
+ *   w          device bf16 [V][K].
+ *   logits     device fp32 [B][V] or NULL (logits[b][v] = x[b] . w[v]).
+ *   shard_max  device fp32 [tp][B]; -inf for a shard with no real id.
+ *   shard_idx  device int32 [tp][B] global ids; -1 for an empty shard.
+ *   ids        device int32 [B] global argmax.
+ *   workspace  device, ws_bytes >= tpl_lmhead_workspace_size(...), 16-byte
+ *              aligned.  It must be zero-filled before its first use; every
+ *              call that completes leaves it zero-filled again, so it can be
+ *              reused without clearing.  After TPL_ERR_TIMEOUT, clear it again.
+ * Ties go to the lowest global id.  Calls sharing a workspace must not overlap.
+ */
+tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
+                             int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
+                             int32_t* shard_idx, int32_t* ids, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/*
+ * Synchronises `stream`, then returns TPL_ERR_TIMEOUT if any kernel of this
+ * library on the current device recorded a pipeline timeout since the last
+ * call (and clears it), TPL_ERR_CUDA if the stream reports an error, else
+ * TPL_OK.
+ */
+tpl_status tpl_get_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* tpl_status_string(tpl_status s);
+
+/* Number of tensor-core/CUDA kernels this library enqueued in the calling
+ * process since load (host-side count, for launch accounting). */
+uint64_t tpl_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TPL_H */

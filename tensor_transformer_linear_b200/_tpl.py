@@ -1,0 +1,252 @@
+"""ctypes binding of libtpl.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does
+nothing but check that torch tensors are CUDA tensors of the right dtype and
+shape, pass their data pointers and the current stream, and turn a non-zero
+status into :class:`TplError`.  Output tensors the caller does not pass are
+allocated with torch (device memory is torch's job).  There is no CPU path: a
+CPU tensor, or a missing ``libtpl.so``, raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtpl.so")
+
+TPL_MAX_TP = 64
+TPL_MAX_SUB = 8
+
+STATUS = {0: "TPL_OK", 1: "TPL_ERR_NULL", 2: "TPL_ERR_SHAPE", 3: "TPL_ERR_INDIVISIBLE",
+          4: "TPL_ERR_DTYPE", 5: "TPL_ERR_ALIGN", 6: "TPL_ERR_CUDA", 7: "TPL_ERR_TIMEOUT",
+          8: "TPL_ERR_UNSUPPORTED"}
+ACT = {"none": 0, None: 0, "gelu_erf": 1, "gelu_tanh": 2}
+DTYPE = {torch.float32: 0, torch.bfloat16: 1}
+
+EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_reduce",
+            "tpl_rmsnorm", "tpl_lmhead_workspace_size", "tpl_lmhead_argmax",
+            "tpl_get_device_status", "tpl_status_string", "tpl_launch_count")
+
+
+class TplError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        self.name = STATUS.get(code, str(code))
+        super().__init__(f"{where}: {self.name}")
+
+
+class Partition(ctypes.Structure):
+    _fields_ = [("tp_size", ctypes.c_int32), ("n_sub", ctypes.c_int32),
+                ("logical_out", ctypes.c_int64),
+                ("width", (ctypes.c_int64 * TPL_MAX_SUB) * TPL_MAX_TP),
+                ("src_off", (ctypes.c_int64 * TPL_MAX_SUB) * TPL_MAX_TP),
+                ("dst_off", (ctypes.c_int64 * TPL_MAX_SUB) * TPL_MAX_TP),
+                ("shard_width", ctypes.c_int64 * TPL_MAX_TP),
+                ("shard_base", ctypes.c_int64 * TPL_MAX_TP)]
+
+    def as_lists(self):
+        tp, ns = self.tp_size, self.n_sub
+        return dict(width=[[self.width[r][j] for j in range(ns)] for r in range(tp)],
+                    src_off=[[self.src_off[r][j] for j in range(ns)] for r in range(tp)],
+                    dst_off=[[self.dst_off[r][j] for j in range(ns)] for r in range(tp)],
+                    shard_width=[self.shard_width[r] for r in range(tp)],
+                    shard_base=[self.shard_base[r] for r in range(tp)])
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m tensor_transformer_linear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.tpl_partition_subparams.argtypes = [ctypes.POINTER(i64), i32, i32, i64,
+                                              ctypes.POINTER(Partition)]
+        L.tpl_column_linear.argtypes = [ctypes.POINTER(Partition), vp, i64, i64, vp, vp, i32, i32,
+                                        vp, vp]
+        L.tpl_row_linear_reduce.argtypes = [vp, ctypes.POINTER(i64), i32, i64, i64, vp, vp, vp,
+                                            i32, vp, vp, vp]
+        L.tpl_rmsnorm.argtypes = [vp, i64, i64, vp, i32, ctypes.c_float, i32, vp, vp]
+        L.tpl_lmhead_workspace_size.argtypes = [i64, i64, i32, i32, ctypes.POINTER(sz)]
+        L.tpl_lmhead_argmax.argtypes = [vp, i64, i64, vp, i64, i32, i32, vp, vp, vp, vp, vp, sz,
+                                        vp]
+        L.tpl_get_device_status.argtypes = [vp]
+        L.tpl_status_string.argtypes = [i32]
+        L.tpl_status_string.restype = ctypes.c_char_p
+        L.tpl_launch_count.restype = ctypes.c_uint64
+        for name in EXPORTED:
+            if name not in ("tpl_status_string", "tpl_launch_count"):
+                getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise TplError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+# ---------------------------------------------------------------- entry points
+
+def tpl_partition_subparams(sub_sizes: Sequence[int], tp: int, align: int = 1) -> Partition:
+    arr = (ctypes.c_int64 * max(1, len(sub_sizes)))(*[int(s) for s in sub_sizes])
+    p = Partition()
+    _check(lib().tpl_partition_subparams(arr, len(sub_sizes), int(tp), int(align),
+                                         ctypes.byref(p)), "tpl_partition_subparams")
+    return p
+
+
+def tpl_column_linear(p: Partition, x: torch.Tensor, w: torch.Tensor,
+                      bias: Optional[torch.Tensor] = None, act: str = "none",
+                      y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Returns y holding every rank's shard (rank r: ``[M, shard_width[r]]`` at M*shard_base[r])."""
+    _cuda(x, "x")
+    dt = x.dtype
+    _cuda(w, "w", dt)
+    if bias is not None:
+        _cuda(bias, "bias", dt)
+    M, K = x.shape[0] if x.dim() == 2 else x.numel() // x.shape[-1], x.shape[-1]
+    if y is None:
+        y = torch.empty(M * p.logical_out, dtype=dt, device=x.device)
+    _cuda(y, "y", dt)
+    if y.numel() < M * p.logical_out or w.numel() != p.logical_out * K:
+        raise ValueError("y or w has the wrong size")
+    if bias is not None and bias.numel() != p.logical_out:
+        raise ValueError("bias size does not match the partition's output size")
+    _check(lib().tpl_column_linear(ctypes.byref(p), _ptr(x), M, K, _ptr(w), _ptr(bias),
+                                   DTYPE[dt], ACT[act], _ptr(y), _stream(stream)),
+           "tpl_column_linear")
+    return y
+
+
+def tpl_row_linear_reduce(h: torch.Tensor, k_w: Sequence[int], M: int, w: torch.Tensor,
+                          bias: Optional[torch.Tensor] = None,
+                          residual: Optional[torch.Tensor] = None,
+                          y: Optional[torch.Tensor] = None,
+                          partials: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``Y = sum_r H_r W2_r^T (+ bias) (+ residual)``; h and w are rank-major packed blocks."""
+    _cuda(h, "h")
+    dt = h.dtype
+    _cuda(w, "w", dt)
+    tp = len(k_w)
+    ktot = sum(int(k) for k in k_w)
+    if h.numel() != M * ktot or w.numel() % ktot != 0:
+        raise ValueError("h or w has the wrong size")
+    N = w.numel() // ktot
+    if y is None:
+        y = torch.empty((M, N), dtype=dt, device=h.device)
+    _cuda(y, "y", dt)
+    if residual is not None:
+        _cuda(residual, "residual", dt)
+    if bias is not None:
+        _cuda(bias, "bias", dt)
+    if partials is not None:
+        _cuda(partials, "partials", torch.float32)
+        if partials.numel() != tp * M * N:
+            raise ValueError("partials must hold tp * M * N floats")
+    kw = (ctypes.c_int64 * tp)(*[int(k) for k in k_w])
+    _check(lib().tpl_row_linear_reduce(_ptr(h), kw, tp, int(M), int(N), _ptr(w), _ptr(bias),
+                                       _ptr(residual), DTYPE[dt], _ptr(y), _ptr(partials),
+                                       _stream(stream)), "tpl_row_linear_reduce")
+    return y
+
+
+def tpl_rmsnorm(x: torch.Tensor, scale: Optional[torch.Tensor] = None, centered: bool = False,
+                eps: float = 1e-6, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _cuda(x, "x")
+    H = x.shape[-1]
+    M = x.numel() // H
+    if y is None:
+        y = torch.empty_like(x)
+    _cuda(y, "y", x.dtype)
+    if scale is not None:
+        _cuda(scale, "scale", torch.float32)
+        if scale.numel() != H:
+            raise ValueError("scale must have H elements")
+    _check(lib().tpl_rmsnorm(_ptr(x), M, H, _ptr(scale), 1 if centered else 0,
+                             ctypes.c_float(eps), DTYPE[x.dtype], _ptr(y), _stream(stream)),
+           "tpl_rmsnorm")
+    return y
+
+
+def tpl_lmhead_workspace_size(B: int, V: int, tp: int, n_chunks: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tpl_lmhead_workspace_size(int(B), int(V), int(tp), int(n_chunks),
+                                           ctypes.byref(n)), "tpl_lmhead_workspace_size")
+    return n.value
+
+
+def lmhead_workspace(B: int, V: int, tp: int, n_chunks: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for tpl_lmhead_argmax (reusable across calls)."""
+    n = tpl_lmhead_workspace_size(B, V, tp, n_chunks)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def tpl_lmhead_argmax(x: torch.Tensor, w: torch.Tensor, tp: int, n_chunks: int,
+                      workspace: torch.Tensor, logits: Optional[torch.Tensor] = None,
+                      ids: Optional[torch.Tensor] = None,
+                      shard_max: Optional[torch.Tensor] = None,
+                      shard_idx: Optional[torch.Tensor] = None, stream=None):
+    """Returns ``(ids [B], shard_max [tp, B], shard_idx [tp, B])``; fills ``logits`` if given."""
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(w, "w", torch.bfloat16)
+    _cuda(workspace, "workspace")
+    B, K = x.shape
+    V = w.shape[0]
+    dev = x.device
+    if ids is None:
+        ids = torch.empty(B, dtype=torch.int32, device=dev)
+    if shard_max is None:
+        shard_max = torch.empty((tp, B), dtype=torch.float32, device=dev)
+    if shard_idx is None:
+        shard_idx = torch.empty((tp, B), dtype=torch.int32, device=dev)
+    if logits is not None:
+        _cuda(logits, "logits", torch.float32)
+        if logits.numel() != B * V:
+            raise ValueError("logits must hold B * V floats")
+    _check(lib().tpl_lmhead_argmax(_ptr(x), B, K, _ptr(w), V, int(tp), int(n_chunks),
+                                   _ptr(logits), _ptr(shard_max), _ptr(shard_idx), _ptr(ids),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream)), "tpl_lmhead_argmax")
+    return ids, shard_max, shard_idx
+
+
+def tpl_get_device_status(stream=None) -> int:
+    return lib().tpl_get_device_status(_stream(stream))
+
+
+def tpl_status_string(code: int) -> str:
+    return lib().tpl_status_string(int(code)).decode()
+
+
+def tpl_launch_count() -> int:
+    return int(lib().tpl_launch_count())

@@ -1,0 +1,389 @@
+// gemm_bf16.cuh -- persistent, warp-specialised tcgen05 GEMM for the column-
+// and row-parallel linears (bf16 in, fp32 accumulate in TMEM, fused epilogue).
+//
+// Column mode (DeepSpeed SubParamLinearLayer.forward, nanotron c_fc): the
+// output columns of every rank's shard are a list of pieces, each a run of
+// consecutive fused-weight rows.  Pieces are cut into 128-column half blocks;
+// a 128x256 tile pairs two consecutive half blocks, whose weight rows are
+// fetched by two TMA boxes with independent row coordinates.  So the fused
+// QKV weight is read in place, in its own order, with no gather pass, and a
+// tile may hold the k piece of a rank in one half and its v piece in the other.
+// The epilogue adds the bias (indexed by weight row), applies GELU and stores
+// bf16 straight into the rank's shard.
+//
+// Row mode (google-research o_wo section, nanotron c_proj): the K loop runs
+// over ranks r0..r1-1 and, inside each, over that rank's contraction slice,
+// all into the same TMEM accumulator.  The cross-shard partial-sum reduction
+// is therefore the accumulation itself, in rank order, in fp32.  The epilogue
+// adds bias and residual and stores bf16 (or, for the unreduced check, stores
+// one rank's fp32 partial).
+//
+// Roles (192 threads, one CTA per SM): warp 0 issues TMA loads into a
+// kStages-deep shared-memory ring; warp 1 issues tcgen05.mma (one elected
+// lane) into one of two TMEM accumulators; warps 2..5 drain the other
+// accumulator through tcgen05.ld, so the epilogue of tile i overlaps the MMAs
+// of tile i+1.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace tpl {
+
+constexpr int kBM = 128;
+constexpr int kHalfN = 128;
+constexpr int kBK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;
+constexpr int kBHalfBytes = kHalfN * kBK * 2;
+constexpr int kStageBytes = kABytes + 2 * kBHalfBytes;
+constexpr int kMaxPieces = 64;
+constexpr int kGemmThreads = 192;
+constexpr int kAccCols = 256;  // fp32 columns of one accumulator
+constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 + 256;
+
+enum GemmMode : int { kModeColumn = 0, kModeRow = 1 };
+
+struct ColPiece {
+  int64_t out_off;   // element offset in y of (row 0, first column of the piece)
+  int32_t src_row;   // first fused-weight row; also the fused-bias index
+  int32_t width;     // columns in the piece
+  int32_t ld;        // row stride (elements) of the rank's shard
+  int32_t hb_begin;  // index of the piece's first 128-column half block
+};
+
+struct GemmArgs {
+  CUtensorMap tmA;  // column: X {K, M};      row: H  {Kr, M, tp}
+  CUtensorMap tmB;  // column: W {K, rows};   row: W2 {Kr, N, tp}
+  int32_t mode;
+  int32_t act;
+  int32_t M;
+  int32_t k_iters;  // 64-wide K blocks per rank (column mode: of K)
+  int32_t r0, r1;   // row mode: ranks accumulated
+  int32_t m_blocks, n_tiles, num_tiles, group_m;
+  int32_t n_halves;
+  int32_t vec_store;  // every output row start is 16-byte aligned
+  int32_t n_pieces;
+  ColPiece pieces[kMaxPieces];
+  const __nv_bfloat16* bias;
+  __nv_bfloat16* y;
+  int32_t N;  // row mode output width
+  const __nv_bfloat16* residual;
+  float* partials;  // row mode: store this launch's fp32 sum here instead of y
+};
+
+struct HalfInfo {
+  int32_t brow;     // weight row (column mode) or output column (row mode) of column 0
+  int32_t valid;    // columns of the half block that exist
+  int64_t out_off;  // element offset in the output of (row 0, column 0)
+  int32_t ld;       // output row stride
+  int32_t bias_off;
+};
+
+__device__ __forceinline__ HalfInfo decode_half(const GemmArgs& a, int hb) {
+  HalfInfo h;
+  if (a.mode == kModeColumn) {
+    int p = 0;
+    while (p + 1 < a.n_pieces && a.pieces[p + 1].hb_begin <= hb) ++p;
+    const ColPiece& pc = a.pieces[p];
+    const int local = (hb - pc.hb_begin) * kHalfN;
+    h.brow = pc.src_row + local;
+    h.valid = min(kHalfN, pc.width - local);
+    h.out_off = pc.out_off + local;
+    h.ld = pc.ld;
+    h.bias_off = pc.src_row + local;
+  } else {
+    const int col = hb * kHalfN;
+    h.brow = col;
+    h.valid = min(kHalfN, a.N - col);
+    h.out_off = col;
+    h.ld = a.N;
+    h.bias_off = col;
+  }
+  return h;
+}
+
+__device__ __forceinline__ void tile_coords(const GemmArgs& a, int t, int& mb, int& nt) {
+  const int per_group = a.group_m * a.n_tiles;
+  const int g = t / per_group;
+  const int first_m = g * a.group_m;
+  const int gsize = min(a.m_blocks - first_m, a.group_m);
+  const int tin = t - g * per_group;
+  mb = first_m + tin % gsize;
+  nt = tin / gsize;
+}
+
+// Epilogue of 32 accumulator columns of one row.
+__device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h, int m, int col0,
+                                            const uint32_t (&r)[32]) {
+  const int nvalid = min(32, h.valid - col0);
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+
+  if (a.mode == kModeRow && a.partials != nullptr) {
+    float* dst = a.partials + static_cast<int64_t>(m) * h.ld + h.out_off + col0;
+    if (nvalid == 32 && a.vec_store) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nvalid) dst[j] = v[j];
+    }
+    return;
+  }
+
+  if (a.bias != nullptr) {
+    const __nv_bfloat16* b = a.bias + h.bias_off + col0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) v[j] += bf16_to_f(b[j]);
+  }
+  if (a.act != TPL_ACT_NONE) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = apply_act(v[j], a.act);
+  }
+  const int64_t off = static_cast<int64_t>(m) * h.ld + h.out_off + col0;
+  if (a.residual != nullptr) {
+    const __nv_bfloat16* res = a.residual + off;
+    if (nvalid == 32 && a.vec_store) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        const uint4 q = *reinterpret_cast<const uint4*>(res + j);
+        v[j + 0] += bf16_lo(q.x); v[j + 1] += bf16_hi(q.x);
+        v[j + 2] += bf16_lo(q.y); v[j + 3] += bf16_hi(q.y);
+        v[j + 4] += bf16_lo(q.z); v[j + 5] += bf16_hi(q.z);
+        v[j + 6] += bf16_lo(q.w); v[j + 7] += bf16_hi(q.w);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nvalid) v[j] += bf16_to_f(res[j]);
+    }
+  }
+  __nv_bfloat16* dst = a.y + off;
+  if (nvalid == 32 && a.vec_store) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint4 q;
+      q.x = pack_bf16x2(v[j + 0], v[j + 1]);
+      q.y = pack_bf16x2(v[j + 2], v[j + 3]);
+      q.z = pack_bf16x2(v[j + 4], v[j + 5]);
+      q.w = pack_bf16x2(v[j + 6], v[j + 7]);
+      *reinterpret_cast<uint4*>(dst + j) = q;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) dst[j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_tcgen05(const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&tfull[i], 1);
+      ptx::mbar_init(&tempty[i], 4);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&a.tmA);
+    ptx::prefetch_tmap(&a.tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 2 * kAccCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int nr = (a.mode == kModeRow) ? (a.r1 - a.r0) : 1;
+  const int k_total = nr * a.k_iters;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < a.num_tiles; t += gridDim.x) {
+        int mb, nt;
+        tile_coords(a, t, mb, nt);
+        const bool has1 = 2 * nt + 1 < a.n_halves;
+        const HalfInfo h0 = decode_half(a, 2 * nt);
+        const HalfInfo h1 = has1 ? decode_half(a, 2 * nt + 1) : h0;
+        const uint32_t bytes = kABytes + (has1 ? 2 : 1) * kBHalfBytes;
+        for (int ki = 0; ki < k_total; ++ki) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * kStageBytes;
+          uint8_t* sB = sA + kABytes;
+          ptx::mbar_arrive_expect_tx(&full[stage], bytes);
+          const int kc = (ki % a.k_iters) * kBK;
+          if (a.mode == kModeColumn) {
+            ptx::tma_load_2d_nohint(sA, &a.tmA, &full[stage], kc, mb * kBM);
+            ptx::tma_load_2d_nohint(sB, &a.tmB, &full[stage], kc, h0.brow);
+            if (has1) ptx::tma_load_2d_nohint(sB + kBHalfBytes, &a.tmB, &full[stage], kc, h1.brow);
+          } else {
+            const int r = a.r0 + ki / a.k_iters;
+            ptx::tma_load_3d_nohint(sA, &a.tmA, &full[stage], kc, mb * kBM, r);
+            ptx::tma_load_3d_nohint(sB, &a.tmB, &full[stage], kc, h0.brow, r);
+            if (has1)
+              ptx::tma_load_3d_nohint(sB + kBHalfBytes, &a.tmB, &full[stage], kc, h1.brow, r);
+          }
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_timeout();
+        // Let the copies already in flight land before the CTA exits.
+        const int back = issued < kStages ? issued : kStages;
+        int s = stage;
+        uint32_t ph = phase;
+        volatile int no_abort = 0;
+        for (int i = 0; i < back; ++i) {
+          if (--s < 0) {
+            s = kStages - 1;
+            ph ^= 1u;
+          }
+          ptx::mbar_wait(&full[s], ph, &no_abort, 200000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    bool any_mma = false;
+    int it = 0;
+    for (int t = blockIdx.x; ok && t < a.num_tiles; t += gridDim.x, ++it) {
+      int mb, nt;
+      tile_coords(a, t, mb, nt);
+      const bool has1 = 2 * nt + 1 < a.n_halves;
+      const uint32_t idesc = has1 ? ptx::idesc_bf16(kBM, 2 * kHalfN) : ptx::idesc_bf16(kBM, kHalfN);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      int w_ok = 1;
+      if (lane == 0) w_ok = ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag);
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kAccCols;
+      for (int ki = 0; ki < k_total; ++ki) {
+        if (lane == 0) w_ok = ptx::mbar_wait(&full[stage], phase, abort_flag);
+        if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sA = ptx::smem_u32(smem + stage * kStageBytes);
+          const uint64_t adesc = ptx::sdesc_kmajor_sw128(sA);
+          const uint64_t bdesc = ptx::sdesc_kmajor_sw128(sA + kABytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            ptx::umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ki | kk) != 0);
+          ptx::umma_commit(&empty[stage]);
+          any_mma = true;
+        }
+        __syncwarp();
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) ptx::umma_commit(&tfull[acc]);
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      record_timeout();
+      if (any_mma) {
+        volatile int no_abort = 0;
+        ptx::umma_commit(drain);
+        ptx::mbar_wait(drain, 0, &no_abort, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < a.num_tiles; t += gridDim.x, ++it) {
+      int mb, nt;
+      tile_coords(a, t, mb, nt);
+      const bool has1 = 2 * nt + 1 < a.n_halves;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      int w_ok = 1;
+      if (lane == 0) w_ok = ptx::mbar_wait(&tfull[acc], acc_phase, abort_flag);
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          record_timeout();
+        }
+        break;
+      }
+      ptx::tc_fence_after();
+      const int m = mb * kBM + row;
+      for (int hh = 0; hh < (has1 ? 2 : 1); ++hh) {
+        const HalfInfo h = decode_half(a, 2 * nt + hh);
+        for (int c = 0; c < kHalfN / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
+          ptx::tmem_ld_wait();
+          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, c * 32, r);
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 2 * kAccCols);
+  }
+}
+
+}  // namespace tpl

@@ -1,0 +1,614 @@
+// tpl_api.cu -- the extern "C" entry points declared in include/tpl.h:
+// argument validation, the sub-parameter partition, TMA descriptor encoding and
+// kernel launches on the caller's stream.  Every computational step runs in
+// the kernels included below; there is no host or library fallback.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/tpl.h"
+#include "common.cuh"
+#include "gemm_bf16.cuh"
+#include "gemm_fp32.cuh"
+#include "lmhead.cuh"
+#include "rmsnorm.cuh"
+
+namespace {
+
+using tpl::ColPiece;
+using tpl::F32Piece;
+
+std::atomic<uint64_t> g_launch_count{0};
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int sm_count = 0;
+  bool gemm_attr = false;
+  bool lm_attr = false;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+tpl_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TPL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sm_count == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return TPL_ERR_CUDA;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return TPL_ERR_UNSUPPORTED;  // built for sm_100a only
+    d.sm_count = n;
+  }
+  if (!d.gemm_attr) {
+    if (cudaFuncSetAttribute(tpl::gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tpl::kGemmSmemBytes) != cudaSuccess)
+      return TPL_ERR_CUDA;
+    d.gemm_attr = true;
+  }
+  if (!d.lm_attr) {
+    if (cudaFuncSetAttribute(tpl::lmhead_argmax_tcgen05,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+      return TPL_ERR_CUDA;
+    d.lm_attr = true;
+  }
+  *out = &d;
+  return TPL_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, box {64, rows[, 1]}.
+tpl_status encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return TPL_ERR_CUDA;
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                  const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                  reinterpret_cast<const cuuint64_t*>(strides), box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TPL_OK : TPL_ERR_CUDA;
+}
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+tpl_status launched() {
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? TPL_OK : TPL_ERR_CUDA;
+}
+
+tpl_status check_partition(const tpl_partition* p) {
+  if (p->tp_size < 1 || p->tp_size > TPL_MAX_TP || p->n_sub < 1 || p->n_sub > TPL_MAX_SUB)
+    return TPL_ERR_SHAPE;
+  if (p->logical_out < 1 || p->logical_out > INT32_MAX) return TPL_ERR_SHAPE;
+  for (int r = 0; r < p->tp_size; ++r) {
+    if (p->shard_width[r] < 1 || p->shard_width[r] > INT32_MAX || p->shard_base[r] < 0)
+      return TPL_ERR_SHAPE;
+    for (int j = 0; j < p->n_sub; ++j) {
+      const int64_t w = p->width[r][j], s = p->src_off[r][j], d = p->dst_off[r][j];
+      if (w < 1 || s < 0 || d < 0 || s + w > p->logical_out || d + w > p->shard_width[r])
+        return TPL_ERR_SHAPE;
+    }
+  }
+  return TPL_OK;
+}
+
+int act_ok(int act) {
+  return act == TPL_ACT_NONE || act == TPL_ACT_GELU_ERF || act == TPL_ACT_GELU_TANH;
+}
+
+// ------------------------------------------------------------------ column
+
+tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
+                       const void* bias, int act, void* y, cudaStream_t st) {
+  if ((K % 8) != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 2) ||
+      (bias != nullptr && !aligned(bias, 2)))
+    return TPL_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  tpl_status s = device_info(&dev);
+  if (s != TPL_OK) return s;
+
+  tpl::GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    if ((s = encode_bf16(&a.tmA, x, 2, dims, str, tpl::kBM)) != TPL_OK) return s;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(p->logical_out)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    if ((s = encode_bf16(&a.tmB, w, 2, dims, str, tpl::kHalfN)) != TPL_OK) return s;
+  }
+  a.mode = tpl::kModeColumn;
+  a.act = act;
+  a.M = static_cast<int32_t>(M);
+  a.k_iters = static_cast<int32_t>((K + tpl::kBK - 1) / tpl::kBK);
+  a.m_blocks = static_cast<int32_t>((M + tpl::kBM - 1) / tpl::kBM);
+  a.group_m = 8;
+  a.bias = static_cast<const __nv_bfloat16*>(bias);
+  a.y = static_cast<__nv_bfloat16*>(y);
+
+  std::vector<ColPiece> pieces;
+  for (int r = 0; r < p->tp_size; ++r)
+    for (int j = 0; j < p->n_sub; ++j) {
+      ColPiece c;
+      c.out_off = M * p->shard_base[r] + p->dst_off[r][j];
+      c.src_row = static_cast<int32_t>(p->src_off[r][j]);
+      c.width = static_cast<int32_t>(p->width[r][j]);
+      c.ld = static_cast<int32_t>(p->shard_width[r]);
+      c.hb_begin = 0;
+      pieces.push_back(c);
+    }
+  for (size_t b = 0; b < pieces.size(); b += tpl::kMaxPieces) {
+    const size_t e = std::min(pieces.size(), b + tpl::kMaxPieces);
+    int hb = 0;
+    bool vec = aligned(y, 16);
+    a.n_pieces = static_cast<int32_t>(e - b);
+    for (size_t i = b; i < e; ++i) {
+      ColPiece c = pieces[i];
+      c.hb_begin = hb;
+      hb += (c.width + tpl::kHalfN - 1) / tpl::kHalfN;
+      vec = vec && (c.out_off % 8 == 0) && (c.ld % 8 == 0);
+      a.pieces[i - b] = c;
+    }
+    a.n_halves = hb;
+    a.vec_store = vec ? 1 : 0;
+    a.n_tiles = (hb + 1) / 2;
+    const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
+    if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
+    a.num_tiles = static_cast<int32_t>(tiles);
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
+    tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
+    if ((s = launched()) != TPL_OK) return s;
+  }
+  return TPL_OK;
+}
+
+tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
+                       const void* bias, int act, void* y, cudaStream_t st) {
+  if (!aligned(x, 4) || !aligned(w, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4)))
+    return TPL_ERR_ALIGN;
+  tpl::F32Args a;
+  std::memset(&a, 0, sizeof(a));
+  a.mode = 0;
+  a.act = act;
+  a.M = M;
+  a.K = static_cast<int32_t>(K);
+  a.x = static_cast<const float*>(x);
+  a.w = static_cast<const float*>(w);
+  a.bias = static_cast<const float*>(bias);
+  a.y = static_cast<float*>(y);
+  std::vector<F32Piece> pieces;
+  for (int r = 0; r < p->tp_size; ++r)
+    for (int j = 0; j < p->n_sub; ++j) {
+      F32Piece c;
+      c.out_off = M * p->shard_base[r] + p->dst_off[r][j];
+      c.src_row = static_cast<int32_t>(p->src_off[r][j]);
+      c.width = static_cast<int32_t>(p->width[r][j]);
+      c.ld = static_cast<int32_t>(p->shard_width[r]);
+      c.nt_begin = 0;
+      pieces.push_back(c);
+    }
+  const int64_t mb = (M + tpl::kF32BM - 1) / tpl::kF32BM;
+  if (mb > 65535) return TPL_ERR_SHAPE;
+  for (size_t b = 0; b < pieces.size(); b += tpl::kF32MaxPieces) {
+    const size_t e = std::min(pieces.size(), b + tpl::kF32MaxPieces);
+    int nt = 0;
+    a.n_pieces = static_cast<int32_t>(e - b);
+    for (size_t i = b; i < e; ++i) {
+      F32Piece c = pieces[i];
+      c.nt_begin = nt;
+      nt += (c.width + tpl::kF32BN - 1) / tpl::kF32BN;
+      a.pieces[i - b] = c;
+    }
+    a.n_tiles = nt;
+    dim3 grid(nt, static_cast<unsigned>(mb));
+    tpl::gemm_fp32_simt<<<grid, tpl::kF32Threads, 0, st>>>(a);
+    tpl_status s = launched();
+    if (s != TPL_OK) return s;
+  }
+  return TPL_OK;
+}
+
+// --------------------------------------------------------------------- row
+
+tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_t N, const void* w,
+                    const void* bias, const void* residual, void* y, float* partials,
+                    cudaStream_t st) {
+  for (int r = 0; r < tp; ++r)
+    if (k_w[r] % 8 != 0) return TPL_ERR_ALIGN;
+  if (!aligned(h, 16) || !aligned(w, 16) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||
+      (residual && !aligned(residual, 2)) || (partials && !aligned(partials, 4)))
+    return TPL_ERR_ALIGN;
+  const int64_t Kr = k_w[0];
+  for (int r = 1; r < tp; ++r)
+    if (k_w[r] != Kr) return TPL_ERR_UNSUPPORTED;  // bf16 path: equal rank widths
+  DeviceInfo* dev = nullptr;
+  tpl_status s = device_info(&dev);
+  if (s != TPL_OK) return s;
+
+  tpl::GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(Kr), static_cast<uint64_t>(M),
+                              static_cast<uint64_t>(tp)};
+    const uint64_t str[2] = {static_cast<uint64_t>(Kr) * 2, static_cast<uint64_t>(M * Kr) * 2};
+    if ((s = encode_bf16(&a.tmA, h, 3, dims, str, tpl::kBM)) != TPL_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(Kr), static_cast<uint64_t>(N),
+                              static_cast<uint64_t>(tp)};
+    const uint64_t str[2] = {static_cast<uint64_t>(Kr) * 2, static_cast<uint64_t>(N * Kr) * 2};
+    if ((s = encode_bf16(&a.tmB, w, 3, dims, str, tpl::kHalfN)) != TPL_OK) return s;
+  }
+  a.mode = tpl::kModeRow;
+  a.M = static_cast<int32_t>(M);
+  a.N = static_cast<int32_t>(N);
+  a.k_iters = static_cast<int32_t>((Kr + tpl::kBK - 1) / tpl::kBK);
+  a.m_blocks = static_cast<int32_t>((M + tpl::kBM - 1) / tpl::kBM);
+  a.n_halves = static_cast<int32_t>((N + tpl::kHalfN - 1) / tpl::kHalfN);
+  a.n_tiles = (a.n_halves + 1) / 2;
+  a.group_m = 8;
+  const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
+  if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
+  a.num_tiles = static_cast<int32_t>(tiles);
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
+  a.y = static_cast<__nv_bfloat16*>(y);
+
+  // The fused path: all ranks accumulate into one accumulator.
+  a.r0 = 0;
+  a.r1 = tp;
+  a.bias = static_cast<const __nv_bfloat16*>(bias);
+  a.residual = static_cast<const __nv_bfloat16*>(residual);
+  a.partials = nullptr;
+  a.vec_store = (N % 8 == 0 && aligned(y, 16) && (residual == nullptr || aligned(residual, 16)));
+  tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
+  if ((s = launched()) != TPL_OK) return s;
+
+  if (partials != nullptr) {
+    a.bias = nullptr;
+    a.residual = nullptr;
+    a.vec_store = (N % 4 == 0 && aligned(partials, 16)) ? 1 : 0;
+    for (int r = 0; r < tp; ++r) {
+      a.r0 = r;
+      a.r1 = r + 1;
+      a.partials = partials + static_cast<int64_t>(r) * M * N;
+      tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
+      if ((s = launched()) != TPL_OK) return s;
+    }
+  }
+  return TPL_OK;
+}
+
+tpl_status row_fp32(const void* h, const int64_t* k_w, int tp, int64_t M, int64_t N, const void* w,
+                    const void* bias, const void* residual, void* y, float* partials,
+                    cudaStream_t st) {
+  if (!aligned(h, 4) || !aligned(w, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4)) ||
+      (residual && !aligned(residual, 4)) || (partials && !aligned(partials, 4)))
+    return TPL_ERR_ALIGN;
+  tpl::F32Args a;
+  std::memset(&a, 0, sizeof(a));
+  a.mode = 1;
+  a.M = M;
+  a.N = static_cast<int32_t>(N);
+  a.h = static_cast<const float*>(h);
+  a.w = static_cast<const float*>(w);
+  a.y = static_cast<float*>(y);
+  a.koff[0] = 0;
+  for (int r = 0; r < tp; ++r) a.koff[r + 1] = a.koff[r] + k_w[r];
+  a.n_tiles = static_cast<int32_t>((N + tpl::kF32BN - 1) / tpl::kF32BN);
+  const int64_t mb = (M + tpl::kF32BM - 1) / tpl::kF32BM;
+  if (mb > 65535) return TPL_ERR_SHAPE;
+  dim3 grid(a.n_tiles, static_cast<unsigned>(mb));
+  a.r0 = 0;
+  a.r1 = tp;
+  a.bias = static_cast<const float*>(bias);
+  a.residual = static_cast<const float*>(residual);
+  tpl::gemm_fp32_simt<<<grid, tpl::kF32Threads, 0, st>>>(a);
+  tpl_status s = launched();
+  if (s != TPL_OK) return s;
+  if (partials != nullptr) {
+    a.bias = nullptr;
+    a.residual = nullptr;
+    for (int r = 0; r < tp; ++r) {
+      a.r0 = r;
+      a.r1 = r + 1;
+      a.partials = partials + static_cast<int64_t>(r) * M * N;
+      tpl::gemm_fp32_simt<<<grid, tpl::kF32Threads, 0, st>>>(a);
+      if ((s = launched()) != TPL_OK) return s;
+    }
+  }
+  return TPL_OK;
+}
+
+// ----------------------------------------------------------------- rmsnorm
+
+template <typename T>
+tpl_status rmsnorm_launch(const void* x, int64_t M, int64_t H, const float* scale, int centered,
+                          float eps, void* y, cudaStream_t st) {
+  DeviceInfo* dev = nullptr;
+  tpl_status s = device_info(&dev);
+  if (s != TPL_OK) return s;
+  constexpr int P = tpl::VecTraits<T>::kPer;
+  const int64_t rows_per_block = tpl::kNormWarps;
+  const int64_t blocks = std::min<int64_t>((M + rows_per_block - 1) / rows_per_block,
+                                           static_cast<int64_t>(dev->sm_count) * 16);
+  const T* xp = static_cast<const T*>(x);
+  T* yp = static_cast<T*>(y);
+  const bool vec = (H % P == 0) && aligned(x, 16) && aligned(y, 16) &&
+                   (scale == nullptr || aligned(scale, 16));
+  const int64_t lanes_vec = (H / P + 31) / 32;  // vectors per lane
+  const int g = static_cast<int>(blocks);
+  const int t = tpl::kNormWarps * 32;
+  const int Hi = static_cast<int>(H);
+  if (vec && lanes_vec <= 32) {
+    if (lanes_vec <= 1)
+      tpl::rmsnorm_reg<T, 1><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else if (lanes_vec <= 2)
+      tpl::rmsnorm_reg<T, 2><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else if (lanes_vec <= 4)
+      tpl::rmsnorm_reg<T, 4><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else if (lanes_vec <= 8)
+      tpl::rmsnorm_reg<T, 8><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else if (lanes_vec <= 16)
+      tpl::rmsnorm_reg<T, 16><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else
+      tpl::rmsnorm_reg<T, 32><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+  } else {
+    tpl::rmsnorm_generic<T><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, H);
+  }
+  return launched();
+}
+
+}  // namespace
+
+// ======================================================================
+// extern "C" entry points
+// ======================================================================
+
+extern "C" {
+
+const char* tpl_status_string(tpl_status s) {
+  switch (s) {
+    case TPL_OK: return "TPL_OK";
+    case TPL_ERR_NULL: return "TPL_ERR_NULL: a required pointer is NULL";
+    case TPL_ERR_SHAPE: return "TPL_ERR_SHAPE: a size is out of range or sizes disagree";
+    case TPL_ERR_INDIVISIBLE: return "TPL_ERR_INDIVISIBLE: the partition leaves a rank empty";
+    case TPL_ERR_DTYPE: return "TPL_ERR_DTYPE: unknown dtype or activation";
+    case TPL_ERR_ALIGN: return "TPL_ERR_ALIGN: pointer or row stride breaks the 16-byte rule";
+    case TPL_ERR_CUDA: return "TPL_ERR_CUDA: a CUDA call failed";
+    case TPL_ERR_TIMEOUT: return "TPL_ERR_TIMEOUT: a kernel gave up waiting on its pipeline";
+    case TPL_ERR_UNSUPPORTED: return "TPL_ERR_UNSUPPORTED: outside what this build implements";
+  }
+  return "unknown tpl_status";
+}
+
+uint64_t tpl_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }
+
+tpl_status tpl_partition_subparams(const int64_t* sub_sizes, int32_t n_sub, int32_t tp_size,
+                                   int64_t align, tpl_partition* out) {
+  if (sub_sizes == nullptr || out == nullptr) return TPL_ERR_NULL;
+  if (tp_size < 1 || tp_size > TPL_MAX_TP || n_sub < 1 || n_sub > TPL_MAX_SUB || align < 1)
+    return TPL_ERR_SHAPE;
+  int64_t total = 0;
+  for (int j = 0; j < n_sub; ++j) {
+    if (sub_sizes[j] < 1 || sub_sizes[j] > INT32_MAX) return TPL_ERR_SHAPE;
+    if (sub_sizes[j] % align != 0) return TPL_ERR_INDIVISIBLE;
+    total += sub_sizes[j];
+  }
+  if (total > INT32_MAX) return TPL_ERR_SHAPE;
+  tpl_partition p;
+  std::memset(&p, 0, sizeof(p));
+  p.tp_size = tp_size;
+  p.n_sub = n_sub;
+  p.logical_out = total;
+  int64_t sub_start = 0;
+  for (int j = 0; j < n_sub; ++j) {
+    const int64_t units = sub_sizes[j] / align;
+    int64_t row = sub_start;
+    for (int r = 0; r < tp_size; ++r) {
+      const int64_t u = units / tp_size + (r < units % tp_size ? 1 : 0);
+      if (u == 0) return TPL_ERR_INDIVISIBLE;
+      p.width[r][j] = u * align;
+      p.src_off[r][j] = row;
+      row += p.width[r][j];
+    }
+    sub_start += sub_sizes[j];
+  }
+  int64_t base = 0;
+  for (int r = 0; r < tp_size; ++r) {
+    int64_t col = 0;
+    for (int j = 0; j < n_sub; ++j) {
+      p.dst_off[r][j] = col;
+      col += p.width[r][j];
+    }
+    p.shard_width[r] = col;
+    p.shard_base[r] = base;
+    base += col;
+  }
+  *out = p;
+  return TPL_OK;
+}
+
+tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                             const void* w, const void* bias, tpl_dtype dt, tpl_act act, void* y,
+                             void* stream) {
+  if (p == nullptr) return TPL_ERR_NULL;
+  if ((dt != TPL_FP32 && dt != TPL_BF16) || !act_ok(act)) return TPL_ERR_DTYPE;
+  tpl_status s = check_partition(p);
+  if (s != TPL_OK) return s;
+  if (M < 0 || K < 1 || M > INT32_MAX || K > INT32_MAX) return TPL_ERR_SHAPE;
+  if (M == 0) return TPL_OK;
+  if (x == nullptr || w == nullptr || y == nullptr) return TPL_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dt == TPL_BF16 ? column_bf16(p, x, M, K, w, bias, act, y, st)
+                        : column_fp32(p, x, M, K, w, bias, act, y, st);
+}
+
+tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
+                                 int64_t N, const void* w, const void* bias, const void* residual,
+                                 tpl_dtype dt, void* y, float* partials, void* stream) {
+  if (k_w == nullptr) return TPL_ERR_NULL;
+  if (dt != TPL_FP32 && dt != TPL_BF16) return TPL_ERR_DTYPE;
+  if (tp < 1 || tp > TPL_MAX_TP || M < 0 || N < 1 || M > INT32_MAX || N > INT32_MAX)
+    return TPL_ERR_SHAPE;
+  int64_t ktot = 0;
+  for (int r = 0; r < tp; ++r) {
+    if (k_w[r] < 1 || k_w[r] > INT32_MAX) return TPL_ERR_SHAPE;
+    ktot += k_w[r];
+  }
+  if (ktot > INT32_MAX) return TPL_ERR_SHAPE;
+  if (M == 0) return TPL_OK;
+  if (h == nullptr || w == nullptr || y == nullptr) return TPL_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dt == TPL_BF16 ? row_bf16(h, k_w, tp, M, N, w, bias, residual, y, partials, st)
+                        : row_fp32(h, k_w, tp, M, N, w, bias, residual, y, partials, st);
+}
+
+tpl_status tpl_rmsnorm(const void* x, int64_t M, int64_t H, const float* scale, int32_t centered,
+                       float eps, tpl_dtype dt, void* y, void* stream) {
+  if (dt != TPL_FP32 && dt != TPL_BF16) return TPL_ERR_DTYPE;
+  if (M < 0 || H < 1 || H > INT32_MAX || !(eps >= 0.0f)) return TPL_ERR_SHAPE;
+  if (M == 0) return TPL_OK;
+  if (x == nullptr || y == nullptr) return TPL_ERR_NULL;
+  if (!aligned(x, dt == TPL_BF16 ? 2 : 4) || !aligned(y, dt == TPL_BF16 ? 2 : 4) ||
+      (scale && !aligned(scale, 4)))
+    return TPL_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dt == TPL_BF16 ? rmsnorm_launch<__nv_bfloat16>(x, M, H, scale, centered, eps, y, st)
+                        : rmsnorm_launch<float>(x, M, H, scale, centered, eps, y, st);
+}
+
+static tpl_status lm_layout(int64_t B, int64_t V, int32_t tp, int32_t n_chunks, int64_t* shard) {
+  if (B < 1 || B > 256 || V < 1 || V > INT32_MAX || tp < 1 || tp > TPL_MAX_TP || n_chunks < 1)
+    return TPL_ERR_SHAPE;
+  const int64_t sh = (V + tp - 1) / tp;
+  const int64_t cap = (sh + n_chunks - 1) / n_chunks;
+  const int64_t num_splits = (sh + cap - 1) / cap;
+  const int64_t last = sh - std::min(sh, cap) * (num_splits - 1);
+  if (num_splits != n_chunks || last <= 0) return TPL_ERR_SHAPE;
+  *shard = sh;
+  return TPL_OK;
+}
+
+tpl_status tpl_lmhead_workspace_size(int64_t B, int64_t V, int32_t tp, int32_t n_chunks,
+                                     size_t* bytes) {
+  if (bytes == nullptr) return TPL_ERR_NULL;
+  int64_t shard = 0;
+  tpl_status s = lm_layout(B, V, tp, n_chunks, &shard);
+  if (s != TPL_OK) return s;
+  const size_t raw = static_cast<size_t>(tp) * static_cast<size_t>(B) * 8 + 16;
+  *bytes = (raw + 255) / 256 * 256;
+  return TPL_OK;
+}
+
+tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
+                             int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
+                             int32_t* shard_idx, int32_t* ids, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (x == nullptr || w == nullptr || shard_max == nullptr || shard_idx == nullptr ||
+      ids == nullptr || workspace == nullptr)
+    return TPL_ERR_NULL;
+  int64_t shard = 0;
+  tpl_status s = lm_layout(B, V, tp, n_chunks, &shard);
+  if (s != TPL_OK) return s;
+  if (K < 1 || K > INT32_MAX) return TPL_ERR_SHAPE;
+  size_t need = 0;
+  tpl_lmhead_workspace_size(B, V, tp, n_chunks, &need);
+  if (ws_bytes < need) return TPL_ERR_SHAPE;
+  if (K % 8 != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(workspace, 16) ||
+      (logits && !aligned(logits, 4)) || !aligned(shard_max, 4) || !aligned(shard_idx, 4) ||
+      !aligned(ids, 4))
+    return TPL_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  if ((s = device_info(&dev)) != TPL_OK) return s;
+
+  tpl::LmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = static_cast<int32_t>(B);
+  a.Npad = static_cast<int32_t>((B + 15) / 16 * 16);
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(V)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    if ((s = encode_bf16(&a.tmW, w, 2, dims, str, tpl::kLmRows)) != TPL_OK) return s;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(B)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    if ((s = encode_bf16(&a.tmX, x, 2, dims, str, static_cast<uint32_t>(a.Npad))) != TPL_OK)
+      return s;
+  }
+  a.K = static_cast<int32_t>(K);
+  a.k_iters = static_cast<int32_t>((K + tpl::kLmBK - 1) / tpl::kLmBK);
+  a.V = static_cast<int32_t>(V);
+  a.tp = tp;
+  a.shard = static_cast<int32_t>(shard);
+  a.n_slabs = static_cast<int32_t>((V + tpl::kLmRows - 1) / tpl::kLmRows);
+  a.stage_bytes = tpl::kLmABytes + a.Npad * tpl::kLmBK * 2;
+  const int budget = 227 * 1024 - 1024 - 256;
+  a.stages = std::min(tpl::kLmMaxStages, budget / a.stage_bytes);
+  if (a.stages < 2) return TPL_ERR_UNSUPPORTED;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(2 * a.Npad)) cols <<= 1;
+  a.tmem_cols = cols;
+  a.logits = logits;
+  a.shard_max = shard_max;
+  a.shard_idx = shard_idx;
+  a.ids = ids;
+  a.keys = static_cast<unsigned long long*>(workspace);
+  a.counter = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
+                                              static_cast<size_t>(tp) * B * 8);
+  const int smem = a.stages * a.stage_bytes + 1024 + 256;
+  const int grid = std::min(a.n_slabs, dev->sm_count);
+  tpl::lmhead_argmax_tcgen05<<<grid, tpl::kLmThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      a);
+  return launched();
+}
+
+tpl_status tpl_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TPL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, tpl::g_status_word, sizeof(int)) != cudaSuccess)
+    return TPL_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(tpl::g_status_word, &zero, sizeof(int)) != cudaSuccess)
+      return TPL_ERR_CUDA;
+    return static_cast<tpl_status>(v);
+  }
+  return TPL_OK;
+}
+
+}  // extern "C"

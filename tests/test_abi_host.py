@@ -1,0 +1,176 @@
+"""Host-side checks of libtpl.so that need no GPU.
+
+The library loads, exports every symbol include/tpl.h declares, computes the
+partition bit-exactly like the oracle, and rejects bad arguments on the host
+with the documented status before touching CUDA.  Every call below that passes
+a non-NULL fake pointer is one the host validation must reject, so nothing is
+ever launched (these tests are also safe on a GPU machine).
+"""
+import ctypes
+import os
+import random
+import re
+
+import pytest
+
+import oracle as O
+import tensor_transformer_linear_b200 as T
+from tensor_transformer_linear_b200 import _tpl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tpl.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const char\*|tpl_status|uint64_t)\s+(tpl_\w+)\(",
+                                 src, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = T.lib()
+    names = _declared()
+    assert len(names) == 9, names
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(names) == sorted(_tpl.EXPORTED)
+
+
+def test_status_strings():
+    for code, name in _tpl.STATUS.items():
+        assert T.tpl_status_string(code).startswith(name)
+
+
+def _oracle_kind(subs, tp, align):
+    try:
+        return O.partition_subparams(subs, tp, align)
+    except O.OracleError as e:
+        return e.kind
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_partition_bit_exact_against_oracle(seed):
+    rng = random.Random(seed)
+    cases = [([4096, 1024, 1024], 8, 128), ([1024], 4, 1), ([14336], 8, 1), ([28672], 8, 1),
+             ([128256], 8, 1)]
+    for _ in range(300):
+        n = rng.randint(1, 4)
+        align = rng.choice([1, 2, 8, 128])
+        cases.append(([align * rng.randint(1, 40) for _ in range(n)], rng.randint(1, 12), align))
+    for subs, tp, align in cases:
+        ref = _oracle_kind(subs, tp, align)
+        if isinstance(ref, str):
+            with pytest.raises(T.TplError) as e:
+                T.tpl_partition_subparams(subs, tp, align)
+            assert e.value.name == "TPL_ERR_" + ref, (subs, tp, align)
+            continue
+        got = T.tpl_partition_subparams(subs, tp, align).as_lists()
+        assert got["width"] == ref.width
+        assert got["src_off"] == ref.src_off
+        assert got["dst_off"] == ref.dst_off
+        assert got["shard_width"] == ref.shard_width
+        assert got["shard_base"] == ref.shard_base
+
+
+def test_partition_argument_errors():
+    L = T.lib()
+    p = _tpl.Partition()
+    arr = (ctypes.c_int64 * 2)(8, 8)
+    assert L.tpl_partition_subparams(None, 2, 2, 1, ctypes.byref(p)) == 1
+    assert L.tpl_partition_subparams(arr, 2, 2, 1, None) == 1
+    assert L.tpl_partition_subparams(arr, 0, 2, 1, ctypes.byref(p)) == 2
+    assert L.tpl_partition_subparams(arr, 9, 2, 1, ctypes.byref(p)) == 2
+    assert L.tpl_partition_subparams(arr, 2, 65, 1, ctypes.byref(p)) == 2
+    assert L.tpl_partition_subparams(arr, 2, 2, 0, ctypes.byref(p)) == 2
+
+
+FAKE = ctypes.c_void_p(0x10000)       # never dereferenced: every call below is rejected first
+FAKE_ODD = ctypes.c_void_p(0x10001)
+
+
+def test_column_linear_rejections():
+    L = T.lib()
+    p = T.tpl_partition_subparams([64, 32], 2, 8)
+    s = ctypes.c_void_p(0)
+    bp = ctypes.byref(p)
+    assert L.tpl_column_linear(None, FAKE, 4, 64, FAKE, None, 1, 0, FAKE, s) == 1
+    assert L.tpl_column_linear(bp, None, 4, 64, FAKE, None, 1, 0, FAKE, s) == 1
+    assert L.tpl_column_linear(bp, FAKE, 4, 64, FAKE, None, 7, 0, FAKE, s) == 4   # dtype
+    assert L.tpl_column_linear(bp, FAKE, 4, 64, FAKE, None, 1, 9, FAKE, s) == 4   # act
+    assert L.tpl_column_linear(bp, FAKE, -1, 64, FAKE, None, 1, 0, FAKE, s) == 2
+    assert L.tpl_column_linear(bp, FAKE, 4, 0, FAKE, None, 1, 0, FAKE, s) == 2
+    assert L.tpl_column_linear(bp, FAKE, 0, 64, FAKE, None, 1, 0, FAKE, s) == 0   # empty: no-op
+    assert L.tpl_column_linear(bp, None, 0, 64, None, None, 1, 0, None, s) == 0
+    assert L.tpl_column_linear(bp, FAKE, 4, 60, FAKE, None, 1, 0, FAKE, s) == 5   # K % 8
+    assert L.tpl_column_linear(bp, FAKE_ODD, 4, 64, FAKE, None, 1, 0, FAKE, s) == 5
+    assert L.tpl_column_linear(bp, FAKE, 4, 64, FAKE_ODD, None, 0, 0, FAKE, s) == 5  # fp32 align
+    bad = _tpl.Partition()
+    ctypes.memmove(ctypes.byref(bad), bp, ctypes.sizeof(p))
+    bad.src_off[1][1] = 90                                       # past the fused weight
+    assert L.tpl_column_linear(ctypes.byref(bad), FAKE, 4, 64, FAKE, None, 1, 0, FAKE, s) == 2
+    bad.src_off[1][1] = p.src_off[1][1]
+    bad.width[0][0] = 0
+    assert L.tpl_column_linear(ctypes.byref(bad), FAKE, 4, 64, FAKE, None, 1, 0, FAKE, s) == 2
+
+
+def test_row_linear_rejections():
+    L = T.lib()
+    s = ctypes.c_void_p(0)
+    kw = (ctypes.c_int64 * 2)(64, 64)
+    assert L.tpl_row_linear_reduce(None, kw, 2, 4, 8, FAKE, None, None, 1, FAKE, None, s) == 1
+    assert L.tpl_row_linear_reduce(None, kw, 2, 0, 8, None, None, None, 1, None, None, s) == 0
+    assert L.tpl_row_linear_reduce(FAKE, None, 2, 4, 8, FAKE, None, None, 1, FAKE, None, s) == 1
+    assert L.tpl_row_linear_reduce(FAKE, kw, 0, 4, 8, FAKE, None, None, 1, FAKE, None, s) == 2
+    assert L.tpl_row_linear_reduce(FAKE, kw, 2, 4, 0, FAKE, None, None, 1, FAKE, None, s) == 2
+    assert L.tpl_row_linear_reduce(FAKE, kw, 2, 4, 8, FAKE, None, None, 3, FAKE, None, s) == 4
+    assert L.tpl_row_linear_reduce(FAKE, kw, 2, 0, 8, FAKE, None, None, 1, FAKE, None, s) == 0
+    kw_bad = (ctypes.c_int64 * 2)(64, 0)
+    assert L.tpl_row_linear_reduce(FAKE, kw_bad, 2, 4, 8, FAKE, None, None, 1, FAKE, None, s) == 2
+    kw_odd = (ctypes.c_int64 * 2)(64, 60)
+    assert L.tpl_row_linear_reduce(FAKE, kw_odd, 2, 4, 8, FAKE, None, None, 1, FAKE, None, s) == 5
+    assert L.tpl_row_linear_reduce(FAKE_ODD, kw, 2, 4, 8, FAKE, None, None, 1, FAKE, None, s) == 5
+
+
+def test_rmsnorm_rejections():
+    L = T.lib()
+    s = ctypes.c_void_p(0)
+    f = ctypes.c_float(1e-6)
+    assert L.tpl_rmsnorm(None, 4, 8, None, 0, f, 1, FAKE, s) == 1
+    assert L.tpl_rmsnorm(FAKE, 4, 8, None, 0, f, 1, None, s) == 1
+    assert L.tpl_rmsnorm(FAKE, 4, 8, None, 0, f, 5, FAKE, s) == 4
+    assert L.tpl_rmsnorm(FAKE, -1, 8, None, 0, f, 1, FAKE, s) == 2
+    assert L.tpl_rmsnorm(FAKE, 4, 0, None, 0, f, 1, FAKE, s) == 2
+    assert L.tpl_rmsnorm(FAKE, 4, 8, None, 0, ctypes.c_float(-1.0), 1, FAKE, s) == 2
+    assert L.tpl_rmsnorm(FAKE, 0, 8, None, 0, f, 1, FAKE, s) == 0
+    assert L.tpl_rmsnorm(None, 0, 8, None, 0, f, 1, None, s) == 0
+    assert L.tpl_rmsnorm(FAKE_ODD, 4, 8, None, 0, f, 1, FAKE, s) == 5
+
+
+def test_lmhead_layout_and_rejections():
+    # the layout rule is the oracle's (LMHead1D.from_model_args with tile 1)
+    for V, tp, n in [(128256, 8, 4), (32000, 8, 3), (10, 4, 2), (72, 8, 4), (9, 8, 1), (1, 1, 1)]:
+        try:
+            O.vocab_layout(V, tp, n)
+            ok = True
+        except O.OracleError:
+            ok = False
+        if ok:
+            assert T.tpl_lmhead_workspace_size(32, V, tp, n) >= tp * 32 * 8 + 4
+        else:
+            with pytest.raises(T.TplError) as e:
+                T.tpl_lmhead_workspace_size(32, V, tp, n)
+            assert e.value.name == "TPL_ERR_SHAPE"
+    L = T.lib()
+    s = ctypes.c_void_p(0)
+    n = T.tpl_lmhead_workspace_size(32, 1000, 4, 2)
+    args = lambda **kw: [kw.get("x", FAKE), kw.get("B", 32), kw.get("K", 64), kw.get("w", FAKE),
+                         kw.get("V", 1000), kw.get("tp", 4), kw.get("nc", 2), None, FAKE, FAKE,
+                         FAKE, kw.get("ws", FAKE), kw.get("wsb", n), s]
+    assert L.tpl_lmhead_argmax(*args(x=None)) == 1
+    assert L.tpl_lmhead_argmax(*args(ws=None)) == 1
+    assert L.tpl_lmhead_argmax(*args(B=0)) == 2
+    assert L.tpl_lmhead_argmax(*args(B=257)) == 2
+    assert L.tpl_lmhead_argmax(*args(nc=0)) == 2
+    assert L.tpl_lmhead_argmax(*args(V=72, tp=8, nc=4)) == 2
+    assert L.tpl_lmhead_argmax(*args(wsb=n - 1)) == 2
+    assert L.tpl_lmhead_argmax(*args(K=60)) == 5
+    assert L.tpl_lmhead_argmax(*args(w=FAKE_ODD)) == 5

@@ -1,0 +1,273 @@
+"""GPU parity of every kernel against the fp64 oracle on small and ragged shapes.
+
+Inputs come from the seeded generator on the host and are copied to the GPU;
+the oracle reads the same (bf16-exact) values in float64.  Shapes span several
+tiles plus ragged tails in M, N and K, uneven sub-parameter pieces, empty
+inputs and tie cases.  All calls go through the C ABI (ctypes binding).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import tensor_transformer_linear_b200 as T
+from workloads import gen
+
+from ._parity import TOL_BF16, TOL_FP32, check_ids, check_shard_ids, f64, rel
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _t(shape, sigma, tid, dtype=torch.bfloat16, seed=0, mu=0.0):
+    return gen.normal(shape, sigma, tensor_id=tid, seed=seed, dtype=dtype, mu=mu)
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    yield
+    assert T.tpl_get_device_status() == 0
+
+
+# ---------------------------------------------------------------- generator
+
+def test_generator_device_matches_host_bitwise():
+    for dtype, sigma, mu in [(torch.bfloat16, 0.02, 0.0), (torch.float32, 0.1, 1.0)]:
+        h = gen.normal((1000, 77), sigma, tensor_id=5, dtype=dtype, mu=mu, chunk=4096)
+        d = gen.normal((1000, 77), sigma, tensor_id=5, dtype=dtype, mu=mu, device=DEV, chunk=4096)
+        assert torch.equal(h, d.cpu())
+
+
+# ------------------------------------------------------------------ RMSNorm
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("M,H", [(1, 64), (7, 4096), (133, 8192), (33, 72), (5, 12288),
+                                 (300, 256), (3, 1000)])
+@pytest.mark.parametrize("mode", ["none", "centered", "plain"])
+def test_rmsnorm(dtype, M, H, mode):
+    x = _t((M, H), 1.0, 0, dtype)
+    s = _t((H,), 0.1, 4, torch.float32) if mode != "none" else None
+    y = T.tpl_rmsnorm(x.to(DEV), s.to(DEV) if s is not None else None, mode == "centered")
+    torch.cuda.synchronize()
+    ref = O.rmsnorm(f64(x), None if s is None else f64(s), mode == "centered", 1e-6)
+    assert rel(y, ref) <= (TOL_BF16 if dtype == torch.bfloat16 else TOL_FP32)
+
+
+def test_rmsnorm_in_place_and_empty():
+    x = _t((64, 4096), 1.0, 0).to(DEV)
+    ref = O.rmsnorm(f64(x))
+    T.tpl_rmsnorm(x, None, False, 1e-6, y=x)
+    assert rel(x, ref) <= TOL_BF16
+    e = torch.empty((0, 4096), dtype=torch.bfloat16, device=DEV)
+    T.tpl_rmsnorm(e)
+
+
+# ------------------------------------------------------------ column linear
+
+COLUMN_CASES = [
+    # sub_sizes, tp, align, M, K, bias, act
+    ([4096 // 8, 1024 // 8, 1024 // 8], 8, 16, 130, 256, True, "none"),   # GQA-like, small
+    ([1024], 4, 1, 32, 256, False, "gelu_tanh"),
+    ([136, 24, 8], 1, 8, 257, 72, True, "gelu_erf"),                     # ragged pieces and K
+    ([256, 256, 256], 2, 128, 1, 64, True, "none"),                      # M = 1
+    ([1792 * 2], 2, 1, 200, 520, False, "gelu_erf"),                     # K ragged > 1 block
+    ([512, 384, 384], 3, 128, 129, 8, True, "gelu_tanh"),                # uneven ranks, K = 8
+    ([14336 // 16], 8, 1, 384, 4096, False, "gelu_erf"),                 # long K
+]
+
+
+@pytest.mark.parametrize("case", COLUMN_CASES)
+def test_column_linear_bf16(case):
+    subs, tp, align, M, K, with_bias, act = case
+    part = O.partition_subparams(subs, tp, align)
+    x = _t((M, K), 1.0, 0)
+    w = _t((sum(subs), K), 0.02, 1)
+    b = _t((sum(subs),), 0.02, 3) if with_bias else None
+    p = T.tpl_partition_subparams(subs, tp, align)
+    y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), b.to(DEV) if b is not None else None, act)
+    torch.cuda.synchronize()
+    ref = O.column_linear(f64(x), f64(w), None if b is None else f64(b), part, act)
+    got = [f64(v) for v in T.shard_views(y, p, M)]
+    err = O.rel_frobenius(np.concatenate([g.ravel() for g in got]),
+                          np.concatenate([r.ravel() for r in ref]))
+    assert err <= TOL_BF16, err
+    for g, r in zip(got, ref):
+        assert O.rel_frobenius(g, r) <= TOL_BF16
+
+
+def test_column_linear_fp32_tiny_mlp_shapes():
+    part = O.partition_subparams([1024], 4, 1)
+    x = _t((32, 256), 1.0, 0, torch.float32)
+    w = _t((1024, 256), 0.02, 1, torch.float32)
+    p = T.tpl_partition_subparams([1024], 4, 1)
+    y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), None, "gelu_tanh")
+    torch.cuda.synchronize()
+    ref = O.column_linear(f64(x), f64(w), None, part, "gelu_tanh")
+    for g, r in zip(T.shard_views(y, p, 32), ref):
+        assert rel(g, r) <= TOL_FP32
+
+
+def test_column_linear_fp32_ragged_with_bias():
+    subs, tp = [70, 30, 30], 3
+    part = O.partition_subparams(subs, tp, 10)
+    x = _t((67, 33), 1.0, 0, torch.float32)
+    w = _t((130, 33), 0.5, 1, torch.float32)
+    b = _t((130,), 0.5, 3, torch.float32)
+    p = T.tpl_partition_subparams(subs, tp, 10)
+    y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), b.to(DEV), "gelu_erf")
+    torch.cuda.synchronize()
+    ref = O.column_linear(f64(x), f64(w), f64(b), part, "gelu_erf")
+    for g, r in zip(T.shard_views(y, p, 67), ref):
+        assert rel(g, r) <= TOL_FP32
+
+
+def test_column_linear_many_pieces_two_launches():
+    # 16 ranks x 5 sub-parameters = 80 pieces: more than one launch's piece table
+    subs, tp = [16 * 16, 16 * 8, 16 * 8, 16 * 24, 16 * 8], 16
+    part = O.partition_subparams(subs, tp, 8)
+    x = _t((150, 128), 1.0, 0)
+    w = _t((sum(subs), 128), 0.05, 1)
+    b = _t((sum(subs),), 0.05, 3)
+    p = T.tpl_partition_subparams(subs, tp, 8)
+    y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), b.to(DEV), "none")
+    torch.cuda.synchronize()
+    ref = O.column_linear(f64(x), f64(w), f64(b), part)
+    for g, r in zip(T.shard_views(y, p, 150), ref):
+        assert rel(g, r) <= TOL_BF16
+
+
+def test_column_linear_empty_rows():
+    p = T.tpl_partition_subparams([256], 2, 1)
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
+    w = _t((256, 64), 0.02, 1).to(DEV)
+    y = torch.zeros(8, dtype=torch.bfloat16, device=DEV)
+    T.tpl_column_linear(p, x, w, None, "none", y=y)
+    assert int(y.abs().sum()) == 0
+
+
+# --------------------------------------------------------------- row linear
+
+ROW_CASES = [
+    # tp, Kr, M, N, bias, residual
+    (8, 64, 130, 256, False, False),
+    (2, 72, 257, 300, True, True),
+    (1, 4096, 128, 512, False, True),
+    (4, 8, 1, 8, True, False),
+    (8, 1792 // 4, 384, 4096 // 8, False, False),
+]
+
+
+@pytest.mark.parametrize("case", ROW_CASES)
+def test_row_linear_reduce_bf16(case):
+    tp, Kr, M, N, with_bias, with_res = case
+    k_w = [Kr] * tp
+    h = _t((M, Kr * tp), 1.0, 5)
+    w2 = _t((N, Kr * tp), 0.02, 2)
+    b = _t((N,), 0.02, 3) if with_bias else None
+    res = _t((M, N), 1.0, 6) if with_res else None
+    hp = T.pack_row_weight(h, k_w)           # rank-major H blocks [M][Kr]
+    wp = T.pack_row_weight(w2, k_w)
+    parts = torch.empty(tp * M * N, dtype=torch.float32, device=DEV)
+    y = T.tpl_row_linear_reduce(hp.to(DEV), k_w, M, wp.to(DEV),
+                                b.to(DEV) if b is not None else None,
+                                res.to(DEV) if res is not None else None, partials=parts)
+    torch.cuda.synchronize()
+    hs = O.row_weight_slices(f64(h), k_w)
+    ws = O.row_weight_slices(f64(w2), k_w)
+    ref = O.row_linear_reduce(hs, ws, None if b is None else f64(b), None if res is None else f64(res))
+    assert rel(y, ref) <= TOL_BF16
+    pref = O.row_partials(hs, ws)
+    pg = f64(parts).reshape(tp, M, N)
+    for r in range(tp):
+        assert O.rel_frobenius(pg[r], pref[r]) <= 1e-5   # fp32 partials of bf16 inputs
+
+
+def test_row_linear_residual_aliases_output():
+    tp, Kr, M, N = 4, 64, 200, 384
+    k_w = [Kr] * tp
+    h = _t((M, Kr * tp), 1.0, 5)
+    w2 = _t((N, Kr * tp), 0.02, 2)
+    x = _t((M, N), 1.0, 6)
+    xd = x.to(DEV)
+    T.tpl_row_linear_reduce(T.pack_row_weight(h, k_w).to(DEV), k_w, M,
+                            T.pack_row_weight(w2, k_w).to(DEV), None, xd, y=xd)
+    torch.cuda.synchronize()
+    ref = O.row_linear_reduce(O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w),
+                              None, f64(x))
+    assert rel(xd, ref) <= TOL_BF16
+
+
+def test_row_linear_fp32_uneven_ranks():
+    k_w = [40, 40, 24, 24]
+    M, N = 33, 70
+    h = _t((M, sum(k_w)), 1.0, 5, torch.float32)
+    w2 = _t((N, sum(k_w)), 0.1, 2, torch.float32)
+    b = _t((N,), 0.1, 3, torch.float32)
+    res = _t((M, N), 1.0, 6, torch.float32)
+    parts = torch.empty(4 * M * N, dtype=torch.float32, device=DEV)
+    y = T.tpl_row_linear_reduce(T.pack_row_weight(h, k_w).to(DEV), k_w, M,
+                                T.pack_row_weight(w2, k_w).to(DEV), b.to(DEV), res.to(DEV),
+                                partials=parts)
+    torch.cuda.synchronize()
+    hs, ws = O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w)
+    assert rel(y, O.row_linear_reduce(hs, ws, f64(b), f64(res))) <= TOL_FP32
+    pg = f64(parts).reshape(4, M, N)
+    for r, pr in enumerate(O.row_partials(hs, ws)):
+        assert O.rel_frobenius(pg[r], pr) <= TOL_FP32
+
+
+def test_row_linear_bf16_uneven_ranks_rejected():
+    h = torch.zeros(4 * 24, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(8 * 24, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(T.TplError) as e:
+        T.tpl_row_linear_reduce(h, [16, 8], 4, w)
+    assert e.value.name == "TPL_ERR_UNSUPPORTED"
+
+
+# ---------------------------------------------------------------- LM head
+
+LM_CASES = [
+    # B, K, V, tp, n_chunks, logits
+    (3, 64, 1000, 4, 2, True),
+    (32, 4096, 9000, 8, 4, True),
+    (17, 200, 37, 4, 2, True),          # shards of 10 ids: several shards inside one slab
+    (1, 8, 9, 8, 1, False),             # empty shards
+    (48, 128, 2000, 3, 5, True),        # B > 32, uneven
+]
+
+
+@pytest.mark.parametrize("case", LM_CASES)
+def test_lmhead_argmax(case):
+    B, K, V, tp, nc, with_logits = case
+    x = _t((B, K), 1.0, 0)
+    w = _t((V, K), 0.02, 1)
+    ws = T.lmhead_workspace(B, V, tp, nc)
+    logits = torch.empty(B * V, dtype=torch.float32, device=DEV) if with_logits else None
+    for rep in range(2):                 # the workspace is reused without clearing
+        ids, smax, sidx = T.tpl_lmhead_argmax(x.to(DEV), w.to(DEV), tp, nc, ws, logits=logits)
+        torch.cuda.synchronize()
+        res = O.lmhead_argmax(f64(x), f64(w), tp, nc)
+        check_ids(ids.cpu().numpy(), res)
+        check_shard_ids(sidx.cpu().numpy(), smax.cpu().numpy(), res)
+        if with_logits:
+            assert rel(logits.view(B, V), res.logits) <= 1e-5
+        assert int(ws.abs().sum()) == 0
+
+
+def test_lmhead_planted_ids_and_tie_break():
+    B, K, V, tp, nc = 4, 128, 4000, 8, 4
+    lay = O.vocab_layout(V, tp, nc)
+    x = _t((B, K), 1.0, 0)
+    w = _t((V, K), 0.01, 1).clone()
+    planted = [lay.shard - 1, lay.shard, V - 1, 3 * lay.shard + lay.split_sizes[0]]
+    for b, v in enumerate(planted):
+        w[v] = (2.0 * x[b].float() / x[b].float().norm()).to(torch.bfloat16)
+    w[7 * lay.shard - 5] = w[planted[1]]          # exact tie in a later shard
+    ws = T.lmhead_workspace(B, V, tp, nc)
+    ids, smax, sidx = T.tpl_lmhead_argmax(x.to(DEV), w.to(DEV), tp, nc, ws)
+    torch.cuda.synchronize()
+    assert ids.cpu().tolist() == planted
+    assert int(sidx[6, 1]) == 7 * lay.shard - 5
