@@ -1,0 +1,565 @@
+#!/usr/bin/env python
+"""Benchmark of the tensor-parallel sharded-linear path on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic input
+(workload ``block``, the default):
+
+  1. GQA fused-QKV column-parallel linear  x[4,1024,4096] bf16, 32 q + 8 kv
+     heads of 128, tp 8, bias                      (sub-parameter partition)
+  2. RMSNorm (eps 1e-6, centred scale) -> c_fc 4096->14336 column-parallel
+     + GELU(erf) -> c_proj 14336->4096 row-parallel with the partial-sum
+     reduction in the epilogue                     x[8,1024,4096] bf16, tp 8
+  3. decode LM head x[32,4096] over W[128256,4096] bf16, 8 vocab shards x 4
+     chunks, fp32 logits kept on chip, per-shard + global argmax
+
+``value`` is the sharded-linear FLOP rate of the step (algorithmic FLOPs of
+the three contractions / step time).  ``--workload stack`` runs the 4-layer
+residual stack x[4,4096,8192], 8192->28672->8192 instead.
+
+``--impl reference`` times the fp64 CPU oracle (the reference of this build)
+on a bounded sample of the same workload.  Under torchrun (N > 1) every rank
+runs an independent replica (the path is single-GPU; there is no exchange)
+and the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import configs as C  # noqa: E402
+from workloads import gen  # noqa: E402
+
+METRIC = "sharded-linear TFLOP/s (% bf16 peak); LM-head decode GB/s (% HBM) at 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ ncu traffic
+
+def _src_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "tensor_transformer_linear_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(kernel: str, workload: str, sources):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = _src_hash(sources)
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload:
+            return float(f[2]) if f[3] == cur else None
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ workloads
+
+class Block:
+    """The default step: fused QKV + RMSNorm/MLP + decode LM head (or a subset, for profiling)."""
+
+    def __init__(self, dev, parts=("qkv", "mlp", "lmhead")):
+        import tensor_transformer_linear_b200 as T
+        self.T = T
+        q, m, l = C.GQA_QKV, C.TP_MLP, C.LM_HEAD
+        self.q, self.m, self.l = q, m, l
+        self.sel = parts
+        names = {"qkv": q.name, "mlp": m.name, "lmhead": l.name}
+        self.name = ("tp-block: " if len(parts) > 1 else "") + " + ".join(names[p] for p in parts)
+        self.flops = 0.0
+        self.gemm_flops = 0.0
+        self.launches = []        # (part name, callable(stream)), in launch order
+        self.d_in, self.d_out = [], []
+        if "qkv" in parts:
+            # inputs and weights, generated on the device by the seeded generator
+            self.qx = C.qkv_x(q, dev)
+            self.qw = C.qkv_w(q, dev)
+            self.qb = C.qkv_bias(q, dev)
+            self.qpart = T.tpl_partition_subparams(q.sub_sizes, q.tp, q.align)
+            self.qy = torch.empty(q.M * q.out, dtype=torch.bfloat16, device=dev)
+            self.launches.append(("qkv_column", lambda s: T.tpl_column_linear(
+                self.qpart, self.qx, self.qw, self.qb, "none", y=self.qy, stream=s)))
+            self.flops += q.flops()
+            self.gemm_flops += q.flops()
+            self.d_in.append(self.qx)
+            self.d_out.append(self.qy)
+        if "mlp" in parts:
+            self.mx = C.mlp_x(m, dev)
+            self.mlp = T.TPMLP(C.mlp_w1(m, 0, dev), C.mlp_w2(m, 0, dev), m.tp, m.act,
+                               scale=C.mlp_scale(m, 0, dev), centered=True, norm=True)
+            self.my = torch.empty((m.M, m.hidden), dtype=torch.bfloat16, device=dev)
+            self.xn = torch.empty_like(self.mx)
+            self.h = torch.empty(m.M * m.inter, dtype=torch.bfloat16, device=dev)
+            mlp = self.mlp
+            self.launches += [
+                ("rmsnorm", lambda s: T.tpl_rmsnorm(self.mx, mlp.scale, True, 1e-6, y=self.xn,
+                                                    stream=s)),
+                ("mlp_column_gelu", lambda s: T.tpl_column_linear(mlp.part, self.xn, mlp.w1, None,
+                                                                  m.act, y=self.h, stream=s)),
+                ("mlp_row_reduce", lambda s: T.tpl_row_linear_reduce(
+                    self.h, mlp.k_w, m.M, mlp.w2, None, None, y=self.my, stream=s))]
+            self.flops += m.flops()
+            self.gemm_flops += m.flops()
+            self.d_in.append(self.mx)
+            self.d_out.append(self.my)
+        if "lmhead" in parts:
+            self.lx = C.lm_x(l, dev)
+            self.lw = C.lm_w(l, dev)
+            self.ws = T.lmhead_workspace(l.batch, l.vocab, l.tp, l.n_chunks, dev)
+            self.ids = torch.empty(l.batch, dtype=torch.int32, device=dev)
+            self.smax = torch.empty((l.tp, l.batch), dtype=torch.float32, device=dev)
+            self.sidx = torch.empty((l.tp, l.batch), dtype=torch.int32, device=dev)
+            self.launches.append(("lmhead_argmax", lambda s: T.tpl_lmhead_argmax(
+                self.lx, self.lw, l.tp, l.n_chunks, self.ws, ids=self.ids, shard_max=self.smax,
+                shard_idx=self.sidx, stream=s)))
+            self.flops += l.flops()
+            self.d_in.append(self.lx)
+            self.d_out += [self.ids, self.smax, self.sidx]
+        self.parts = [n for n, _ in self.launches]
+
+    def step(self, stream, events=None):
+        for i, (_, fn) in enumerate(self.launches):
+            if events is not None:
+                events[i].record(stream)
+            fn(stream)
+        if events is not None:
+            events[len(self.launches)].record(stream)
+
+    def gemm_part_ids(self):
+        return [i for i, n in enumerate(self.parts) if n in ("qkv_column", "mlp_column_gelu",
+                                                              "mlp_row_reduce")]
+
+    # --- end to end through host buffers
+    def host_io(self):
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+        self.h_in = [pin(t.cpu()) for t in self.d_in]
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in self.d_out]
+        b_in = sum(t.numel() * t.element_size() for t in self.h_in)
+        b_out = sum(t.numel() * t.element_size() for t in self.h_out)
+        return b_in, b_out
+
+    def step_e2e(self, stream):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.step(stream)
+        for h, d in zip(self.h_out, self.d_out):
+            h.copy_(d, non_blocking=True)
+
+    def lmhead_bytes(self):
+        return self.l.algorithmic_bytes() if "lmhead" in self.sel else None
+
+    def rmsnorm_bytes(self):
+        return 2 * 2 * self.m.M * self.m.hidden if "mlp" in self.sel else None
+
+    # --- the oracle on a bounded sample (CPU baseline / reference arm)
+    def oracle_sample(self, rows_qkv=256, rows_mlp=96, lm_rows=16032):
+        import numpy as np
+        import oracle as O
+        f64 = lambda t: t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
+        q, m, l = self.q, self.m, self.l
+        jobs, flops, desc = [], 0.0, []
+        if "qkv" in self.sel:
+            xq, wq, bq = f64(self.qx[:rows_qkv]), f64(self.qw), f64(self.qb)
+            part = O.partition_subparams(list(q.sub_sizes), q.tp, q.align)
+            jobs.append(lambda: O.column_linear(xq, wq, bq, part))
+            flops += 2.0 * rows_qkv * q.hidden * q.out
+            desc.append(f"{rows_qkv} token rows of the fused QKV")
+        if "mlp" in self.sel:
+            xm, w1 = f64(self.mx[:rows_mlp]), f64(self.mlp.w1)
+            w2, sc = f64(C.mlp_w2(m, 0, self.mx.device)), f64(self.mlp.scale)
+            jobs.append(lambda: O.tp_mlp(xm, w1, w2, m.tp, m.act, scale=sc, centered=True,
+                                         norm=True))
+            flops += 4.0 * rows_mlp * m.hidden * m.inter
+            desc.append(f"{rows_mlp} token rows of the RMSNorm+MLP")
+        if "lmhead" in self.sel:
+            xl, wl = f64(self.lx), f64(self.lw[:lm_rows])
+            jobs.append(lambda: O.lmhead_argmax(xl, wl, 1, 1))
+            flops += 2.0 * l.batch * l.hidden * lm_rows
+            desc.append(f"{lm_rows} vocab rows x {l.batch} batch rows of the LM head")
+
+        def run():
+            for j in jobs:
+                j()
+        return run, flops, ", ".join(desc)
+
+
+class Stack:
+    """The 4-layer residual TP stack."""
+
+    name = C.STACK4.name
+
+    def __init__(self, dev):
+        import tensor_transformer_linear_b200 as T
+        self.T = T
+        w = C.STACK4
+        self.w = w
+        self.x0 = C.mlp_x(w, dev)
+        self.x = self.x0.clone()
+        self.layers = [T.TPMLP(C.mlp_w1(w, l, dev), C.mlp_w2(w, l, dev), w.tp, w.act,
+                               norm=True, residual=True) for l in range(w.layers)]
+        self.flops = w.flops()
+        self.gemm_flops = w.flops()
+        self.launches_per_step = 3 * w.layers
+        self.parts = []
+        for l in range(w.layers):
+            self.parts += [f"l{l}_rmsnorm", f"l{l}_column_gelu", f"l{l}_row_reduce_residual"]
+
+    def step(self, stream, events=None):
+        T = self.T
+        i = 0
+        for layer in self.layers:
+            M = self.x.shape[0]
+            xn = layer._buf("xn", self.x.numel(), self.x).view(M, -1)
+            h = layer._buf("h", M * layer.inter, self.x)
+            if events is not None:
+                events[i].record(stream)
+            T.tpl_rmsnorm(self.x, None, False, 1e-6, y=xn, stream=stream)
+            if events is not None:
+                events[i + 1].record(stream)
+            T.tpl_column_linear(layer.part, xn, layer.w1, None, layer.act, y=h, stream=stream)
+            if events is not None:
+                events[i + 2].record(stream)
+            T.tpl_row_linear_reduce(h, layer.k_w, M, layer.w2, None, self.x, y=self.x,
+                                    stream=stream)
+            i += 3
+        if events is not None:
+            events[i].record(stream)
+
+    def host_io(self):
+        self.h_in = torch.empty(self.x.shape, dtype=self.x.dtype, pin_memory=True).copy_(self.x0.cpu())
+        self.h_out = torch.empty(self.x.shape, dtype=self.x.dtype, pin_memory=True)
+        n = self.x.numel() * self.x.element_size()
+        return n, n
+
+    def step_e2e(self, stream):
+        self.x.copy_(self.h_in, non_blocking=True)
+        self.step(stream)
+        self.h_out.copy_(self.x, non_blocking=True)
+
+    def lmhead_bytes(self):
+        return None
+
+    def rmsnorm_bytes(self):
+        return None
+
+    def gemm_part_ids(self):
+        return [i for i in range(len(self.parts)) if i % 3 != 0]
+
+    def oracle_sample(self, rows=8):
+        import numpy as np
+        import oracle as O
+        f64 = lambda t: t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
+        w = self.w
+        xs = f64(self.x0[:rows])
+        layers = [(f64(l.w1), f64(C.mlp_w2(w, i, self.x0.device)), None)
+                  for i, l in enumerate(self.layers)]
+
+        def run():
+            O.tp_stack(xs, layers, w.tp, w.act)
+        return run, w.layers * 4.0 * rows * w.hidden * w.inter, \
+            f"{rows} token rows through all {w.layers} layers"
+
+
+WORKLOADS = {"block": Block, "stack": Stack,
+             "qkv": lambda dev: Block(dev, ("qkv",)),
+             "mlp": lambda dev: Block(dev, ("mlp",)),
+             "lmhead": lambda dev: Block(dev, ("lmhead",))}
+
+
+# ------------------------------------------------------------------ timing
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else cpu_cores()
+    except Exception:
+        return cpu_cores()
+
+
+def time_oracle(run, flops, target_s=15.0, max_reps=50):
+    """Repeat the oracle sample for about target_s seconds; returns TFLOP/s and reps."""
+    t0 = time.perf_counter()
+    run()
+    one = time.perf_counter() - t0
+    reps = max(1, min(max_reps, int(target_s / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run()
+    dt = time.perf_counter() - t0
+    return flops * reps / dt / 1e12, reps, dt
+
+
+def run_reference(args, wl_cls, rank, world):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = wl_cls(dev)
+    run, flops, desc = wl.oracle_sample()
+    for _ in range(max(1, args.warmup)):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    v = flops * args.steps / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "parallelism": "oracle on host cores"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="block", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl_cls = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, wl_cls, rank, world)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    import tensor_transformer_linear_b200 as T
+    wl = wl_cls(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    n_ev = len(wl.parts) + 1
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            wl.step(stream)
+    torch.cuda.synchronize()
+    if T.tpl_get_device_status(stream) != 0:
+        raise RuntimeError("a kernel reported a pipeline timeout during warm-up")
+
+    # ---- device-timed region: K steps, per-launch events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device())
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    n0 = T.tpl_launch_count()
+    start.record(stream)
+    for k in range(args.steps):
+        wl.step(stream, evs[k])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    launches = T.tpl_launch_count() - n0
+    clk = clocks.stop()
+    if pg is not None:
+        pg.barrier()
+    ms = start.elapsed_time(stop)
+    if T.tpl_get_device_status(stream) != 0:
+        raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
+    part_ms = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
+               for i in range(n_ev - 1)]
+
+    # ---- end to end through host buffers (pinned), copies inside the timed region
+    b_in, b_out = wl.host_io()
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            wl.step_e2e(stream)
+    torch.cuda.synchronize()
+    e_steps = max(10, args.steps // 5)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e_steps):
+            wl.step_e2e(stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+
+    if pg is not None:
+        t = torch.tensor([ms, e_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms, e_ms = float(t[0]), float(t[1])
+
+    if rank == 0:
+        pk, pk_kind = peaks()
+        step_ms = ms / args.steps
+        value = world * wl.flops / (step_ms * 1e-3) / 1e12
+        e2e_val = world * wl.flops / (e_ms / e_steps * 1e-3) / 1e12
+        # dominant kernel: the tcgen05 GEMM (all launches of it in the step)
+        gids = wl.gemm_part_ids()
+        n_gemm = len(gids)
+        gemm_ms = sum(part_ms[i] for i in gids)
+        gemm_launch_flops = wl.gemm_flops / max(1, n_gemm)
+        gemm_achieved = wl.gemm_flops / (gemm_ms * 1e-3) / 1e12 if n_gemm else 0.0
+        peak_t = pk["bf16_tflops"]
+        traffic = ncu_traffic("gemm_bf16_tcgen05", args.workload,
+                              ["gemm_bf16.cuh", "ptx.cuh", "common.cuh"])
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded SplitMix64 / Irwin-Hall normal, the pages' shapes)",
+            "config": {"workload": wl.name,
+                       "parallelism": f"{world} replica(s); tp shards of each linear computed "
+                                      "on one GPU, cross-shard sum in the GEMM epilogue",
+                       "l2": "not flushed: one step streams ~1.5 GB (block) / ~4 GB (stack), "
+                             "far above the 126 MB L2"},
+            "roofline": {"kernel": "gemm_bf16_tcgen05", "bound": "tensor",
+                         "achieved": round(gemm_achieved, 2), "peak": peak_t,
+                         "unit": "TFLOP/s", "frac": round(gemm_achieved / peak_t, 4),
+                         "peak_kind": f"{pk_kind} bf16 burst",
+                         "frac_of_sustained": round(gemm_achieved / pk["bf16_tflops_sustained"], 4),
+                         "launches_per_step": n_gemm,
+                         "flops_per_launch_avg": gemm_launch_flops,
+                         "traffic": traffic},
+            "parts_ms": {n: round(v, 4) for n, v in zip(wl.parts, part_ms)},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_out)},
+        }
+        lb = wl.lmhead_bytes()
+        if lb is not None:
+            lm_ms = part_ms[wl.parts.index("lmhead_argmax")]
+            gbs = lb / (lm_ms * 1e-3) / 1e9
+            line["roofline_lmhead"] = {
+                "kernel": "lmhead_argmax_tcgen05", "bound": "hbm", "achieved": round(gbs, 1),
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                "frac_of_8000": round(gbs / 8000.0, 4), "bytes_per_launch": lb,
+                "traffic": ncu_traffic("lmhead_argmax_tcgen05", "lmhead",
+                                       ["lmhead.cuh", "ptx.cuh", "common.cuh"])}
+        rb = wl.rmsnorm_bytes()
+        if rb is not None:
+            r_ms = part_ms[wl.parts.index("rmsnorm")]
+            line["roofline_rmsnorm"] = {"kernel": "rmsnorm_reg", "bound": "hbm",
+                                        "achieved": round(rb / (r_ms * 1e-3) / 1e9, 1),
+                                        "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                        "frac": round(rb / (r_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        if not gids:
+            line["roofline"] = line.pop("roofline_lmhead")
+        if world == 1 and not args.no_cpu_baseline:
+            run, flops, desc = wl.oracle_sample()
+            v, reps, dt = time_oracle(run, flops)
+            line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s",
+                                    "cores": blas_threads(), "kind": "oracle",
+                                    "sample": f"{desc}; {reps} reps in {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
