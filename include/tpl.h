@@ -206,6 +206,36 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
                              void* stream);
 
 /*
+ * tpl_lmhead_argmax with no workspace argument, for callers that cannot
+ * allocate device memory.  (No counterpart on the pages: this is an
+ * integration entry point of this library.)  Some callers cannot call
+ * cudaMalloc: a plugin inside a host framework that owns all device memory
+ * and hands the plugin only its input and output buffers, or a
+ * latency-critical decode loop where an allocation (which can synchronise the
+ * device) is not allowed.  This entry point allocates nothing: its scratch
+ * (per-shard keys and a completion counter) lives in a fixed array of
+ * TPL_LMHEAD_STATIC_SCRATCH_BYTES bytes inside the library, which every GPU
+ * that loads the library holds until the process exits.
+ *
+ * Arguments, layout, outputs and ties are as for tpl_lmhead_argmax; the
+ * caller still passes x, w and every output buffer.
+ *   - Sizes whose scratch (tp * B * 8 + 16 bytes, rounded up to 256) exceeds
+ *     TPL_LMHEAD_STATIC_SCRATCH_BYTES are rejected with TPL_ERR_SHAPE.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - Every call on a device shares the one array and clears the part it uses
+ *     (cudaMemsetAsync on `stream`) before the kernel.  Calls whose work
+ *     overlaps on the GPU (different streams, or different host threads)
+ *     race on it: order them on one stream.
+ */
+#define TPL_LMHEAD_STATIC_SCRATCH_BYTES 65536
+
+tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
+                                    int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
+                                    int32_t* shard_idx, int32_t* ids, void* stream);
+
+/*
  * Synchronises `stream`, then returns TPL_ERR_TIMEOUT if any kernel of this
  * library on the current device recorded a pipeline timeout since the last
  * call (and clears it), TPL_ERR_CUDA if the stream reports an error, else

@@ -6,6 +6,6 @@ script (``build``).
 """
 from ._tpl import (EXPORTED, Partition, TplError, lib, lmhead_workspace,  # noqa: F401
                    tpl_column_linear, tpl_get_device_status, tpl_launch_count,
-                   tpl_lmhead_argmax, tpl_lmhead_workspace_size, tpl_partition_subparams,
+                   tpl_lmhead_argmax, tpl_lmhead_argmax_static, tpl_lmhead_workspace_size, tpl_partition_subparams,
                    tpl_rmsnorm, tpl_row_linear_reduce, tpl_status_string, LIB_PATH)
 from .path import TPMLP, TPStack, pack_row_weight, shard_views  # noqa: F401

@@ -29,7 +29,8 @@ DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 
 EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_reduce",
             "tpl_rmsnorm", "tpl_lmhead_workspace_size", "tpl_lmhead_argmax",
-            "tpl_get_device_status", "tpl_status_string", "tpl_launch_count")
+            "tpl_get_device_status", "tpl_status_string", "tpl_launch_count",
+            "tpl_lmhead_argmax_static")
 
 
 class TplError(RuntimeError):
@@ -79,6 +80,8 @@ def lib():
         L.tpl_lmhead_workspace_size.argtypes = [i64, i64, i32, i32, ctypes.POINTER(sz)]
         L.tpl_lmhead_argmax.argtypes = [vp, i64, i64, vp, i64, i32, i32, vp, vp, vp, vp, vp, sz,
                                         vp]
+        L.tpl_lmhead_argmax_static.argtypes = [vp, i64, i64, vp, i64, i32, i32, vp, vp, vp, vp,
+                                               vp]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -237,6 +240,38 @@ def tpl_lmhead_argmax(x: torch.Tensor, w: torch.Tensor, tp: int, n_chunks: int,
                                    _ptr(logits), _ptr(shard_max), _ptr(shard_idx), _ptr(ids),
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream)), "tpl_lmhead_argmax")
+    return ids, shard_max, shard_idx
+
+
+def tpl_lmhead_argmax_static(x: torch.Tensor, w: torch.Tensor, tp: int, n_chunks: int,
+                             logits: Optional[torch.Tensor] = None,
+                             ids: Optional[torch.Tensor] = None,
+                             shard_max: Optional[torch.Tensor] = None,
+                             shard_idx: Optional[torch.Tensor] = None, stream=None):
+    """tpl_lmhead_argmax without a workspace: the library's own fixed scratch is used.
+
+    For callers that cannot allocate device memory.  Calls that overlap on the
+    GPU share that scratch and race; order them on one stream.
+    """
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(w, "w", torch.bfloat16)
+    B, K = x.shape
+    V = w.shape[0]
+    dev = x.device
+    if ids is None:
+        ids = torch.empty(B, dtype=torch.int32, device=dev)
+    if shard_max is None:
+        shard_max = torch.empty((tp, B), dtype=torch.float32, device=dev)
+    if shard_idx is None:
+        shard_idx = torch.empty((tp, B), dtype=torch.int32, device=dev)
+    if logits is not None:
+        _cuda(logits, "logits", torch.float32)
+        if logits.numel() != B * V:
+            raise ValueError("logits must hold B * V floats")
+    _check(lib().tpl_lmhead_argmax_static(_ptr(x), B, K, _ptr(w), V, int(tp), int(n_chunks),
+                                          _ptr(logits), _ptr(shard_max), _ptr(shard_idx),
+                                          _ptr(ids), _stream(stream)),
+           "tpl_lmhead_argmax_static")
     return ids, shard_max, shard_idx
 
 

@@ -612,3 +612,62 @@ tpl_status tpl_get_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ======================================================================
+// LM head with library-owned scratch, for callers that cannot allocate
+// ======================================================================
+
+// Scratch of tpl_lmhead_argmax_static: per-(shard, row) keys and the
+// completion counter.  A device global, so no call allocates; every GPU that
+// loads the library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_lmhead_scratch[TPL_LMHEAD_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices];
+
+// Device address of g_lmhead_scratch on the current device, looked up once per
+// device.  In host code the array's name is only a host-side stand-in, so the
+// kernel must be given this address instead.
+tpl_status lmhead_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TPL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_lmhead_scratch) != cudaSuccess || p == nullptr)
+      return TPL_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return TPL_OK;
+}
+
+}  // namespace
+
+extern "C" tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t K, const void* w,
+                                               int64_t V, int32_t tp, int32_t n_chunks,
+                                               float* logits, float* shard_max,
+                                               int32_t* shard_idx, int32_t* ids, void* stream) {
+  // The checks tpl_lmhead_argmax makes, repeated here so that a rejected call
+  // enqueues nothing (not even the scratch clear).
+  if (x == nullptr || w == nullptr || shard_max == nullptr || shard_idx == nullptr ||
+      ids == nullptr)
+    return TPL_ERR_NULL;
+  size_t need = 0;
+  tpl_status s = tpl_lmhead_workspace_size(B, V, tp, n_chunks, &need);
+  if (s != TPL_OK) return s;
+  if (need > static_cast<size_t>(TPL_LMHEAD_STATIC_SCRATCH_BYTES)) return TPL_ERR_SHAPE;
+  if (K < 1 || K > INT32_MAX) return TPL_ERR_SHAPE;
+  if (K % 8 != 0 || !aligned(x, 16) || !aligned(w, 16) || (logits && !aligned(logits, 4)) ||
+      !aligned(shard_max, 4) || !aligned(shard_idx, 4) || !aligned(ids, 4))
+    return TPL_ERR_ALIGN;
+  void* scratch = nullptr;
+  if ((s = lmhead_scratch_address(&scratch)) != TPL_OK) return s;
+  // The array keeps the previous call's contents: start this call from zero.
+  if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TPL_ERR_CUDA;
+  return tpl_lmhead_argmax(x, B, K, w, V, tp, n_chunks, logits, shard_max, shard_idx, ids, scratch,
+                           static_cast<size_t>(TPL_LMHEAD_STATIC_SCRATCH_BYTES), stream);
+}
