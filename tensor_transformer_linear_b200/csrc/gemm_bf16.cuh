@@ -18,11 +18,12 @@
 // adds bias and residual and stores bf16 (or, for the unreduced check, stores
 // one rank's fp32 partial).
 //
-// Roles (192 threads, one CTA per SM): warp 0 issues TMA loads into a
+// Roles (320 threads, one CTA per SM): warp 0 issues TMA loads into a
 // kStages-deep shared-memory ring; warp 1 issues tcgen05.mma (one elected
-// lane) into one of two TMEM accumulators; warps 2..5 drain the other
-// accumulator through tcgen05.ld, so the epilogue of tile i overlaps the MMAs
-// of tile i+1.
+// lane) into one of two TMEM accumulators; warps 2..9 drain the other
+// accumulator through tcgen05.ld -- each owns one TMEM lane quarter (32 rows)
+// and one 128-column half -- so the epilogue of tile i overlaps the MMAs of
+// tile i+1, with two epilogue warps per SM sub-partition to hide latency.
 #pragma once
 
 #include "common.cuh"
@@ -38,9 +39,11 @@ constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBHalfBytes = kHalfN * kBK * 2;
 constexpr int kStageBytes = kABytes + 2 * kBHalfBytes;
 constexpr int kMaxPieces = 64;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter: one per 128-column half
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kAccCols = 256;  // fp32 columns of one accumulator
-constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kBiasSmemBytes = kEpiWarps * kHalfN * 4;
+constexpr int kGemmSmemBytes = kStages * kStageBytes + kBiasSmemBytes + 1024 + 256;
 
 enum GemmMode : int { kModeColumn = 0, kModeRow = 1 };
 
@@ -115,7 +118,7 @@ __device__ __forceinline__ void tile_coords(const GemmArgs& a, int t, int& mb, i
 
 // Epilogue of 32 accumulator columns of one row.
 __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h, int m, int col0,
-                                            const uint32_t (&r)[32]) {
+                                            const uint32_t (&r)[32], const float* bias_s) {
   const int nvalid = min(32, h.valid - col0);
   float v[32];
 #pragma unroll
@@ -136,14 +139,12 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h
   }
 
   if (a.bias != nullptr) {
-    const __nv_bfloat16* b = a.bias + h.bias_off + col0;
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < nvalid) v[j] += bf16_to_f(b[j]);
+    for (int j = 0; j < 32; ++j) v[j] += bias_s[col0 + j];
   }
   if (a.act != TPL_ACT_NONE) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = apply_act(v[j], a.act);
+    for (int j = 0; j < 32; ++j) v[j] = apply_act_fast(v[j], a.act);
   }
   const int64_t off = static_cast<int64_t>(m) * h.ld + h.out_off + col0;
   if (a.residual != nullptr) {
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  float* bias_smem = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kBiasSmemBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&tfull[i], 1);
-      ptx::mbar_init(&tempty[i], 4);
+      ptx::mbar_init(&tempty[i], kEpiWarps);
     }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
@@ -284,34 +286,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    bool any_mma = false;
-    int it = 0;
-    for (int t = blockIdx.x; ok && t < a.num_tiles; t += gridDim.x, ++it) {
-      int mb, nt;
-      tile_coords(a, t, mb, nt);
-      const bool has1 = 2 * nt + 1 < a.n_halves;
-      const uint32_t idesc = has1 ? ptx::idesc_bf16(kBM, 2 * kHalfN) : ptx::idesc_bf16(kBM, kHalfN);
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
-      int w_ok = 1;
-      if (lane == 0) w_ok = ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag);
-      if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
-        ok = false;
-        break;
-      }
-      ptx::tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * kAccCols;
-      for (int ki = 0; ki < k_total; ++ki) {
-        if (lane == 0) w_ok = ptx::mbar_wait(&full[stage], phase, abort_flag);
-        if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+    // One thread issues every MMA: no warp-wide synchronisation per stage.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      bool any_mma = false;
+      int it = 0;
+      for (int t = blockIdx.x; ok && t < a.num_tiles; t += gridDim.x, ++it) {
+        int mb, nt;
+        tile_coords(a, t, mb, nt);
+        const bool has1 = 2 * nt + 1 < a.n_halves;
+        const uint32_t idesc =
+            has1 ? ptx::idesc_bf16(kBM, 2 * kHalfN) : ptx::idesc_bf16(kBM, kHalfN);
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        if (lane == 0) {
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        for (int ki = 0; ki < k_total; ++ki) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
           const uint32_t sA = ptx::smem_u32(smem + stage * kStageBytes);
           const uint64_t adesc = ptx::sdesc_kmajor_sw128(sA);
           const uint64_t bdesc = ptx::sdesc_kmajor_sw128(sA + kABytes);
@@ -320,38 +321,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptx::umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ki | kk) != 0);
           ptx::umma_commit(&empty[stage]);
           any_mma = true;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
+        if (!ok) break;
+        ptx::umma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_timeout();
+        if (any_mma) {
+          volatile int no_abort = 0;
+          ptx::umma_commit(drain);
+          ptx::mbar_wait(drain, 0, &no_abort, 200000000ull);
         }
       }
-      if (!ok) break;
-      if (lane == 0) ptx::umma_commit(&tfull[acc]);
-      __syncwarp();
     }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      record_timeout();
-      if (any_mma) {
-        volatile int no_abort = 0;
-        ptx::umma_commit(drain);
-        ptx::mbar_wait(drain, 0, &no_abort, 200000000ull);
-      }
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int ew = warp - 2;    // 0 .. kEpiWarps-1
+    const int q = warp & 3;     // TMEM lane quarter this warp may access
+    const int hh = ew >> 2;     // 128-column half of the accumulator it drains
     const int row = q * 32 + lane;
+    float* bias_s = bias_smem + ew * kHalfN;
     int it = 0;
     for (int t = blockIdx.x; t < a.num_tiles; t += gridDim.x, ++it) {
       int mb, nt;
       tile_coords(a, t, mb, nt);
-      const bool has1 = 2 * nt + 1 < a.n_halves;
+      const bool active = (hh == 0) || (2 * nt + 1 < a.n_halves);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      HalfInfo h;
+      if (active) {
+        h = decode_half(a, 2 * nt + hh);
+        if (a.bias != nullptr) {
+          // This warp's 128 bias values, read once per tile while the MMAs run.
+          for (int i = lane; i < kHalfN; i += 32)
+            bias_s[i] = (i < h.valid) ? bf16_to_f(a.bias[h.bias_off + i]) : 0.0f;
+          __syncwarp();
+        }
+      }
       int w_ok = 1;
       if (lane == 0) w_ok = ptx::mbar_wait(&tfull[acc], acc_phase, abort_flag);
       if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
@@ -362,14 +373,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       ptx::tc_fence_after();
-      const int m = mb * kBM + row;
-      for (int hh = 0; hh < (has1 ? 2 : 1); ++hh) {
-        const HalfInfo h = decode_half(a, 2 * nt + hh);
+      if (active) {
+        const int m = mb * kBM + row;
         for (int c = 0; c < kHalfN / 32; ++c) {
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
           ptx::tmem_ld_wait();
-          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, c * 32, r);
+          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, c * 32, r, bias_s);
         }
       }
       ptx::tc_fence_before();

@@ -11,8 +11,12 @@
 // through a deep TMA ring; the epilogue warps turn each finished slab into
 // per-(shard, row) 64-bit keys (order-preserving logit bits, inverted id) and
 // fold them into the workspace with atomicMax, which also resolves ties to the
-// lowest id.  The last CTA to finish writes shard_max / shard_idx / ids and
-// zeroes the workspace for the next call.
+// lowest id.  Each epilogue warp transposes its 32 x 16 logit tiles through
+// shared memory so that one lane scans one batch row with float compares, and
+// folds its winners into the workspace with one atomic instruction per tile:
+// the epilogue stays a small fraction of a slab's streaming time and leaves
+// issue slots to the producer and MMA warps.  The last CTA to finish writes
+// shard_max / shard_idx / ids and zeroes the workspace for the next call.
 #pragma once
 
 #include "common.cuh"
@@ -25,13 +29,16 @@ constexpr int kLmBK = 64;
 constexpr int kLmThreads = 192;
 constexpr int kLmABytes = kLmRows * kLmBK * 2;
 constexpr int kLmMaxStages = 12;
+constexpr int kLmTbufWarp = 16 * 33;  // floats of one epilogue warp's transpose tile
+constexpr int kLmTbufBytes = 4 * kLmTbufWarp * 4;
 
 struct LmArgs {
-  CUtensorMap tmW;  // {K, V}, box {64, 128}
+  CUtensorMap tmW;  // {K, V}, box {64, slab_rows}
   CUtensorMap tmX;  // {K, B}, box {64, Npad}
   int32_t B, Npad, K, k_iters;
   int32_t V, tp, shard;
   int32_t n_slabs;
+  int32_t slab_rows;  // vocab rows per slab (<= 128; the MMA tile rows beyond it are ignored)
   int32_t stages, stage_bytes;
   uint32_t tmem_cols;
   float* logits;
@@ -79,6 +86,7 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;
+  float* tbuf = reinterpret_cast<float*>(smem + a.stages * a.stage_bytes + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -113,7 +121,8 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
     if (lane == 0) {
       const uint64_t pol_w = ptx::policy_evict_first();
       const uint64_t pol_x = ptx::policy_evict_last();
-      const uint32_t bytes = static_cast<uint32_t>(a.stage_bytes);
+      const uint32_t bytes =
+          static_cast<uint32_t>(a.slab_rows * kLmBK * 2 + a.stage_bytes - kLmABytes);
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -125,7 +134,7 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
           }
           uint8_t* sW = smem + stage * a.stage_bytes;
           ptx::mbar_arrive_expect_tx(&full[stage], bytes);
-          ptx::tma_load_2d(sW, &a.tmW, &full[stage], kb * kLmBK, slab * kLmRows, pol_w);
+          ptx::tma_load_2d(sW, &a.tmW, &full[stage], kb * kLmBK, slab * a.slab_rows, pol_w);
           ptx::tma_load_2d(sW + kLmABytes, &a.tmX, &full[stage], kb * kLmBK, 0, pol_x);
           ++issued;
           if (++stage == S) {
@@ -151,29 +160,27 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
       }
     }
   } else if (warp == 1) {
-    const uint32_t idesc = ptx::idesc_bf16(kLmRows, a.Npad);
-    int stage = 0, it = 0;
-    uint32_t phase = 0;
-    bool ok = true, any_mma = false;
-    for (int slab = blockIdx.x; ok && slab < a.n_slabs; slab += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
-      int w_ok = 1;
-      if (lane == 0) w_ok = ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag);
-      if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
-        ok = false;
-        break;
-      }
-      ptx::tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * (a.tmem_cols / 2);
-      for (int kb = 0; kb < a.k_iters; ++kb) {
-        if (lane == 0) w_ok = ptx::mbar_wait(&full[stage], phase, abort_flag);
-        if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+    // One thread issues every MMA: no warp-wide synchronisation per stage.
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_bf16(kLmRows, a.Npad);
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true, any_mma = false;
+      for (int slab = blockIdx.x; ok && slab < a.n_slabs; slab += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        if (lane == 0) {
+        const uint32_t d_tmem = tmem_base + acc * (a.tmem_cols / 2);
+        for (int kb = 0; kb < a.k_iters; ++kb) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
           const uint32_t sW = ptx::smem_u32(smem + stage * a.stage_bytes);
           const uint64_t adesc = ptx::sdesc_kmajor_sw128(sW);
           const uint64_t bdesc = ptx::sdesc_kmajor_sw128(sW + kLmABytes);
@@ -182,27 +189,24 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
             ptx::umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
           ptx::umma_commit(&empty[stage]);
           any_mma = true;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
+        if (!ok) break;
+        ptx::umma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_timeout();
+        if (any_mma) {
+          volatile int no_abort = 0;
+          ptx::umma_commit(drain);
+          ptx::mbar_wait(drain, 0, &no_abort, 200000000ull);
         }
       }
-      if (!ok) break;
-      if (lane == 0) ptx::umma_commit(&tfull[acc]);
-      __syncwarp();
     }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      record_timeout();
-      if (any_mma) {
-        volatile int no_abort = 0;
-        ptx::umma_commit(drain);
-        ptx::mbar_wait(drain, 0, &no_abort, 200000000ull);
-      }
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
@@ -222,34 +226,72 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
         break;
       }
       ptx::tc_fence_after();
-      const int row0 = slab * kLmRows + q * 32;  // first vocab id of this warp
+      const int slab0 = slab * a.slab_rows;              // first vocab id of the slab
+      const int row0 = slab0 + q * 32;                   // first vocab id of this warp
+      const int row_end = min(slab0 + a.slab_rows, a.V);  // ids at or past it are not this slab's
       const int v = row0 + lane;
-      const bool valid = v < a.V;
-      const int s_first = min(row0, a.V - 1) / a.shard;
-      const int s_last = min(row0 + 31, a.V - 1) / a.shard;
-      const bool warp_live = row0 < a.V;
+      const bool valid = v < row_end;
+      const bool warp_live = row0 < row_end;
+      const int s_first = min(row0, row_end - 1) / a.shard;
+      const int s_last = min(row0 + 31, row_end - 1) / a.shard;
+      const int split = (s_first + 1) * a.shard;  // first id of the next shard
+      float* tb = tbuf + (warp - 2) * kLmTbufWarp;
+      const int col = lane & 15, half = lane >> 4;
       for (int c = 0; c < a.Npad; c += 16) {
         uint32_t r[16];
         tmem_ld16(tmem_base + ((q * 32u) << 16) + acc * (a.tmem_cols / 2) + c, r);
         ptx::tmem_ld_wait();
         if (!warp_live) continue;
+        if (a.logits != nullptr && valid) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int b = c + j;
-          if (b >= a.B) continue;
-          const float f = __uint_as_float(r[j]);
-          if (a.logits != nullptr && valid) a.logits[static_cast<int64_t>(b) * a.V + v] = f;
-          unsigned long long key = valid ? make_key(f, v) : 0ull;
-          if (s_first == s_last) {
+          for (int j = 0; j < 16; ++j)
+            if (c + j < a.B) a.logits[static_cast<int64_t>(c + j) * a.V + v] = __uint_as_float(r[j]);
+        }
+        if (s_last > s_first + 1) {
+          // Shards narrower than a warp (tiny vocabularies): one atomic per logit.
+          if (valid) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
-              key = other > key ? other : key;
-            }
-            if (lane == 0) atomicMax(&a.keys[s_first * a.B + b], key);
-          } else if (valid) {
-            atomicMax(&a.keys[(v / a.shard) * a.B + b], key);
+            for (int j = 0; j < 16; ++j)
+              if (c + j < a.B)
+                atomicMax(&a.keys[(v / a.shard) * a.B + c + j], make_key(__uint_as_float(r[j]), v));
           }
+          continue;
+        }
+        // Transpose the warp's 32 rows x 16 columns through shared memory so that
+        // each lane scans one column (batch row) over 16 vocab rows with plain
+        // float compares, ascending ids first (ties keep the lowest id).
+#pragma unroll
+        for (int j = 0; j < 16; ++j) tb[j * 33 + lane] = __uint_as_float(r[j]);
+        __syncwarp();
+        float bv0 = 0.0f, bv1 = 0.0f;
+        int bi0 = -1, bi1 = -1;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int rr = half * 16 + i;
+          const int vv = row0 + rr;
+          const float f = tb[col * 33 + rr];
+          if (vv < row_end) {
+            if (vv < split) {
+              if (bi0 < 0 || f > bv0) { bv0 = f; bi0 = vv; }
+            } else {
+              if (bi1 < 0 || f > bv1) { bv1 = f; bi1 = vv; }
+            }
+          }
+        }
+        __syncwarp();
+        // Lanes l and l ^ 16 hold the two row halves of the same column.
+        {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv0, 16);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi0, 16);
+          if (oi >= 0 && (bi0 < 0 || ov > bv0 || (ov == bv0 && oi < bi0))) { bv0 = ov; bi0 = oi; }
+          const float ov1 = __shfl_xor_sync(0xffffffffu, bv1, 16);
+          const int oi1 = __shfl_xor_sync(0xffffffffu, bi1, 16);
+          if (oi1 >= 0 && (bi1 < 0 || ov1 > bv1 || (ov1 == bv1 && oi1 < bi1))) { bv1 = ov1; bi1 = oi1; }
+        }
+        const int b = c + col;
+        if (half == 0 && b < a.B) {
+          if (bi0 >= 0) atomicMax(&a.keys[s_first * a.B + b], make_key(bv0, bi0));
+          if (bi1 >= 0) atomicMax(&a.keys[(s_first + 1) * a.B + b], make_key(bv1, bi1));
         }
       }
       ptx::tc_fence_before();

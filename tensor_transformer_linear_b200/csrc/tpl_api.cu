@@ -13,7 +13,7 @@
 #include <mutex>
 #include <vector>
 
-#include "../../include/tpl.h"
+#include "tpl.h"
 #include "common.cuh"
 #include "gemm_bf16.cuh"
 #include "gemm_fp32.cuh"
@@ -155,7 +155,7 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
   a.M = static_cast<int32_t>(M);
   a.k_iters = static_cast<int32_t>((K + tpl::kBK - 1) / tpl::kBK);
   a.m_blocks = static_cast<int32_t>((M + tpl::kBM - 1) / tpl::kBM);
-  a.group_m = 8;
+  a.group_m = 16;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
   a.y = static_cast<__nv_bfloat16*>(y);
 
@@ -279,7 +279,7 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   a.m_blocks = static_cast<int32_t>((M + tpl::kBM - 1) / tpl::kBM);
   a.n_halves = static_cast<int32_t>((N + tpl::kHalfN - 1) / tpl::kHalfN);
   a.n_tiles = (a.n_halves + 1) / 2;
-  a.group_m = 8;
+  a.group_m = 16;
   const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
   if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
   a.num_tiles = static_cast<int32_t>(tiles);
@@ -558,10 +558,19 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
   std::memset(&a, 0, sizeof(a));
   a.B = static_cast<int32_t>(B);
   a.Npad = static_cast<int32_t>((B + 15) / 16 * 16);
+  // Slab height: the fewest rounds of at most 128-row slabs over the SMs, then
+  // the shortest slab that still covers V in that many rounds, so every CTA
+  // streams (nearly) the same number of rows.
+  {
+    const int64_t sms = dev->sm_count;
+    const int64_t rounds = (V + sms * tpl::kLmRows - 1) / (sms * tpl::kLmRows);
+    a.slab_rows = static_cast<int32_t>((V + sms * rounds - 1) / (sms * rounds));
+  }
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(V)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
-    if ((s = encode_bf16(&a.tmW, w, 2, dims, str, tpl::kLmRows)) != TPL_OK) return s;
+    if ((s = encode_bf16(&a.tmW, w, 2, dims, str, static_cast<uint32_t>(a.slab_rows))) != TPL_OK)
+      return s;
   }
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(B)};
@@ -574,9 +583,9 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
   a.V = static_cast<int32_t>(V);
   a.tp = tp;
   a.shard = static_cast<int32_t>(shard);
-  a.n_slabs = static_cast<int32_t>((V + tpl::kLmRows - 1) / tpl::kLmRows);
+  a.n_slabs = static_cast<int32_t>((V + a.slab_rows - 1) / a.slab_rows);
   a.stage_bytes = tpl::kLmABytes + a.Npad * tpl::kLmBK * 2;
-  const int budget = 227 * 1024 - 1024 - 256;
+  const int budget = 227 * 1024 - 1024 - 256 - tpl::kLmTbufBytes;
   a.stages = std::min(tpl::kLmMaxStages, budget / a.stage_bytes);
   if (a.stages < 2) return TPL_ERR_UNSUPPORTED;
   uint32_t cols = 32;
@@ -589,7 +598,7 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
   a.keys = static_cast<unsigned long long*>(workspace);
   a.counter = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
                                               static_cast<size_t>(tp) * B * 8);
-  const int smem = a.stages * a.stage_bytes + 1024 + 256;
+  const int smem = a.stages * a.stage_bytes + 1024 + 256 + tpl::kLmTbufBytes;
   const int grid = std::min(a.n_slabs, dev->sm_count);
   tpl::lmhead_argmax_tcgen05<<<grid, tpl::kLmThreads, smem, static_cast<cudaStream_t>(stream)>>>(
       a);
