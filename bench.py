@@ -359,6 +359,19 @@ def blas_threads():
         return cpu_cores()
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (every rank calls this at the same point)."""
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def replica_rate(world, flops_per_step, step_ms):
+    """Whole-job TFLOP/s of ``world`` replicas that each ran one step in ``step_ms`` (max)."""
+    return world * flops_per_step / (step_ms * 1e-3) / 1e12
+
+
 def time_oracle(run, flops, target_s=15.0, max_reps=50):
     """Repeat the oracle sample for about target_s seconds; returns TFLOP/s and reps."""
     t0 = time.perf_counter()
@@ -487,15 +500,13 @@ def main():
     e_ms = e0.elapsed_time(e1)
 
     if pg is not None:
-        t = torch.tensor([ms, e_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms, e_ms = float(t[0]), float(t[1])
+        ms, e_ms = max_over_ranks([ms, e_ms], dev)
 
     if rank == 0:
         pk, pk_kind = peaks()
         step_ms = ms / args.steps
-        value = world * wl.flops / (step_ms * 1e-3) / 1e12
-        e2e_val = world * wl.flops / (e_ms / e_steps * 1e-3) / 1e12
+        value = replica_rate(world, wl.flops, step_ms)
+        e2e_val = replica_rate(world, wl.flops, e_ms / e_steps)
         # dominant kernel: the tcgen05 GEMM (all launches of it in the step)
         gids = wl.gemm_part_ids()
         n_gemm = len(gids)
