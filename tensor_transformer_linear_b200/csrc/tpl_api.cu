@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -16,6 +17,7 @@
 #include "tpl.h"
 #include "common.cuh"
 #include "gemm_bf16.cuh"
+#include "gemm_bf16_pair.cuh"
 #include "gemm_fp32.cuh"
 #include "lmhead.cuh"
 #include "rmsnorm.cuh"
@@ -56,6 +58,10 @@ tpl_status device_info(DeviceInfo** out) {
   if (!d.gemm_attr) {
     if (cudaFuncSetAttribute(tpl::gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tpl::kGemmSmemBytes) != cudaSuccess)
+      return TPL_ERR_CUDA;
+    if (cudaFuncSetAttribute(tpl::gemm_bf16_tcgen05_pair,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tpl::kGemmPairSmemBytes) != cudaSuccess)
       return TPL_ERR_CUDA;
     d.gemm_attr = true;
   }
@@ -107,6 +113,34 @@ tpl_status launched() {
   return cudaGetLastError() == cudaSuccess ? TPL_OK : TPL_ERR_CUDA;
 }
 
+// CTA pairs (tcgen05 cta_group::2, 256-row tiles) unless M fits one 128-row
+// block or TPL_GEMM_CTA_PAIRS=0 asks for the single-CTA kernel.
+bool use_cta_pairs(int64_t M) {
+  const char* e = std::getenv("TPL_GEMM_CTA_PAIRS");
+  if (e != nullptr && e[0] == '0') return false;
+  return M > tpl::kBM;
+}
+
+// Fills the tile counts of `a` (n_tiles / n_halves already set) and launches
+// the GEMM on a single CTA per tile or on CTA pairs.
+tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, const DeviceInfo* dev, cudaStream_t st) {
+  const bool pairs = use_cta_pairs(M) && dev->sm_count >= 2;
+  const int64_t bm = pairs ? tpl::kPairBM : tpl::kBM;
+  a.m_blocks = static_cast<int32_t>((M + bm - 1) / bm);
+  a.group_m = pairs ? 8 : 16;
+  const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
+  if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
+  a.num_tiles = static_cast<int32_t>(tiles);
+  if (pairs) {
+    const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, dev->sm_count / 2));
+    tpl::gemm_bf16_tcgen05_pair<<<grid, tpl::kGemmThreads, tpl::kGemmPairSmemBytes, st>>>(a);
+  } else {
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
+    tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
+  }
+  return launched();
+}
+
 tpl_status check_partition(const tpl_partition* p) {
   if (p->tp_size < 1 || p->tp_size > TPL_MAX_TP || p->n_sub < 1 || p->n_sub > TPL_MAX_SUB)
     return TPL_ERR_SHAPE;
@@ -154,8 +188,6 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
   a.act = act;
   a.M = static_cast<int32_t>(M);
   a.k_iters = static_cast<int32_t>((K + tpl::kBK - 1) / tpl::kBK);
-  a.m_blocks = static_cast<int32_t>((M + tpl::kBM - 1) / tpl::kBM);
-  a.group_m = 16;
   a.bias = static_cast<const __nv_bfloat16*>(bias);
   a.y = static_cast<__nv_bfloat16*>(y);
 
@@ -185,12 +217,7 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
     a.n_halves = hb;
     a.vec_store = vec ? 1 : 0;
     a.n_tiles = (hb + 1) / 2;
-    const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
-    if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
-    a.num_tiles = static_cast<int32_t>(tiles);
-    const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
-    tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
-    if ((s = launched()) != TPL_OK) return s;
+    if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
   }
   return TPL_OK;
 }
@@ -276,14 +303,8 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   a.M = static_cast<int32_t>(M);
   a.N = static_cast<int32_t>(N);
   a.k_iters = static_cast<int32_t>((Kr + tpl::kBK - 1) / tpl::kBK);
-  a.m_blocks = static_cast<int32_t>((M + tpl::kBM - 1) / tpl::kBM);
   a.n_halves = static_cast<int32_t>((N + tpl::kHalfN - 1) / tpl::kHalfN);
   a.n_tiles = (a.n_halves + 1) / 2;
-  a.group_m = 16;
-  const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
-  if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
-  a.num_tiles = static_cast<int32_t>(tiles);
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
   a.y = static_cast<__nv_bfloat16*>(y);
 
   // The fused path: all ranks accumulate into one accumulator.
@@ -293,8 +314,7 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   a.residual = static_cast<const __nv_bfloat16*>(residual);
   a.partials = nullptr;
   a.vec_store = (N % 8 == 0 && aligned(y, 16) && (residual == nullptr || aligned(residual, 16)));
-  tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
-  if ((s = launched()) != TPL_OK) return s;
+  if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
 
   if (partials != nullptr) {
     a.bias = nullptr;
@@ -304,8 +324,7 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
       a.r0 = r;
       a.r1 = r + 1;
       a.partials = partials + static_cast<int64_t>(r) * M * N;
-      tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
-      if ((s = launched()) != TPL_OK) return s;
+      if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
     }
   }
   return TPL_OK;
