@@ -553,7 +553,7 @@ def main():
         rb = wl.rmsnorm_bytes()
         if rb is not None:
             r_ms = part_ms[wl.parts.index("rmsnorm")]
-            line["roofline_rmsnorm"] = {"kernel": "rmsnorm_reg", "bound": "hbm",
+            line["roofline_rmsnorm"] = {"kernel": "rmsnorm_cta", "bound": "hbm",
                                         "achieved": round(rb / (r_ms * 1e-3) / 1e9, 1),
                                         "peak": pk["hbm_gbs"], "unit": "GB/s",
                                         "frac": round(rb / (r_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}

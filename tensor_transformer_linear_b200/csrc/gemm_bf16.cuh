@@ -116,9 +116,31 @@ __device__ __forceinline__ void tile_coords(const GemmArgs& a, int t, int& mb, i
   nt = tin / gsize;
 }
 
-// Epilogue of 32 accumulator columns of one row.
+// Bias of the 32 output columns of a half block starting at col0 (0 past its
+// valid columns), read straight from global memory: every lane of a warp asks
+// for the same addresses, so the loads are broadcasts.
+__device__ __forceinline__ void load_bias_chunk(const GemmArgs& a, const HalfInfo& h, int col0,
+                                                float (&bv)[32]) {
+  const int nvalid = min(32, h.valid - col0);
+  const __nv_bfloat16* b = a.bias + h.bias_off + col0;
+  if (nvalid == 32 && (reinterpret_cast<uintptr_t>(b) & 15u) == 0) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(b + j));
+      bv[j + 0] = bf16_lo(q.x); bv[j + 1] = bf16_hi(q.x);
+      bv[j + 2] = bf16_lo(q.y); bv[j + 3] = bf16_hi(q.y);
+      bv[j + 4] = bf16_lo(q.z); bv[j + 5] = bf16_hi(q.z);
+      bv[j + 6] = bf16_lo(q.w); bv[j + 7] = bf16_hi(q.w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) bv[j] = (j < nvalid) ? bf16_to_f(b[j]) : 0.0f;
+  }
+}
+
+// Epilogue of 32 accumulator columns of one row; bv holds the chunk's bias.
 __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h, int m, int col0,
-                                            const uint32_t (&r)[32], const float* bias_s) {
+                                            const uint32_t (&r)[32], const float (&bv)[32]) {
   const int nvalid = min(32, h.valid - col0);
   float v[32];
 #pragma unroll
@@ -140,7 +162,7 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h
 
   if (a.bias != nullptr) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] += bias_s[col0 + j];
+    for (int j = 0; j < 32; ++j) v[j] += bv[j];
   }
   if (a.act != TPL_ACT_NONE) {
 #pragma unroll
@@ -379,7 +401,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
           ptx::tmem_ld_wait();
-          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, c * 32, r, bias_s);
+          if (m < a.M && c * 32 < h.valid) {
+            float bv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) bv[j] = bias_s[c * 32 + j];
+            store_chunk(a, h, m, c * 32, r, bv);
+          }
         }
       }
       ptx::tc_fence_before();

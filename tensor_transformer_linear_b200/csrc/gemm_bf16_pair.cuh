@@ -23,19 +23,17 @@
 
 namespace tpl {
 
-constexpr int kPairStages = 6;
+constexpr int kPairStages = 7;
 constexpr int kPairStageBytes = kABytes + kBHalfBytes;  // per CTA
 constexpr int kPairBM = 2 * kBM;                        // tile rows over the pair
-constexpr int kGemmPairSmemBytes = kPairStages * kPairStageBytes + kBiasSmemBytes + 1024 + 256;
+constexpr int kGemmPairSmemBytes = kPairStages * kPairStageBytes + 1024 + 256;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tcgen05_pair(const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* bias_smem = reinterpret_cast<float*>(smem + kPairStages * kPairStageBytes);
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes + kBiasSmemBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
   uint64_t* tempty = tfull + 2;
@@ -179,7 +177,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int hh = ew >> 2;
     const int row = q * 32 + lane;
-    float* bias_s = bias_smem + ew * kHalfN;
     int it = 0;
     for (int t = pair; t < a.num_tiles; t += npairs, ++it) {
       int mb, nt;
@@ -188,14 +185,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       HalfInfo h;
-      if (active) {
-        h = decode_half(a, 2 * nt + hh);
-        if (a.bias != nullptr) {
-          for (int i = lane; i < kHalfN; i += 32)
-            bias_s[i] = (i < h.valid) ? bf16_to_f(a.bias[h.bias_off + i]) : 0.0f;
-          __syncwarp();
-        }
-      }
+      if (active) h = decode_half(a, 2 * nt + hh);
       int w_ok = 1;
       if (lane == 0) w_ok = ptx::mbar_wait(&tfull[acc], acc_phase, abort_flag);
       if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
@@ -209,10 +199,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (active) {
         const int m = mb * kPairBM + static_cast<int>(rank) * kBM + row;
         for (int c = 0; c < kHalfN / 32; ++c) {
+          float bv[32];
+          if (a.bias != nullptr && c * 32 < h.valid) load_bias_chunk(a, h, c * 32, bv);
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
           ptx::tmem_ld_wait();
-          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, c * 32, r, bias_s);
+          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, c * 32, r, bv);
         }
       }
       ptx::tc_fence_before();

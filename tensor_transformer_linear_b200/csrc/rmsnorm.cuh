@@ -112,6 +112,75 @@ __global__ void __launch_bounds__(kNormWarps * 32)
   }
 }
 
+constexpr int kNormCtaThreads = 128;
+
+// Wide rows: one 128-thread CTA per row, VPT 16-byte vectors per thread held in
+// registers (about 40 registers), so an SM keeps 16 CTAs -- 64 warps of loads --
+// in flight.  Sum of squares: shuffles within each warp, then 4 partials through
+// shared memory.  y may alias x (each thread rewrites only what it read).
+template <typename T, int VPT>
+__global__ void __launch_bounds__(kNormCtaThreads)
+    rmsnorm_cta(const T* x, T* y, const float* __restrict__ scale, int centered, float eps,
+                int64_t M, int H) {
+  using VT = VecTraits<T>;
+  constexpr int P = VT::kPer;
+  __shared__ float part[kNormCtaThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int nvec = H / P;
+  const float inv_h = 1.0f / static_cast<float>(H);
+  for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * H);
+    uint4 q[VPT];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = tid + kNormCtaThreads * i;
+      if (v < nvec) {
+        q[i] = __ldcs(xr + v);
+        float f[P];
+        VT::unpack(q[i], f);
+#pragma unroll
+        for (int e = 0; e < P; ++e) ss = fmaf(f[e], f[e], ss);
+      }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) part[w] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNormCtaThreads / 32; ++i) tot += part[i];
+    __syncthreads();  // part[] is rewritten by the next row
+    const float rinv = rsqrtf(tot * inv_h + eps);
+    uint4* yr = reinterpret_cast<uint4*>(y + row * H);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = tid + kNormCtaThreads * i;
+      if (v < nvec) {
+        float f[P];
+        VT::unpack(q[i], f);
+        if (scale != nullptr) {
+          const float4* s4 = reinterpret_cast<const float4*>(scale + v * P);
+#pragma unroll
+          for (int e4 = 0; e4 < P / 4; ++e4) {
+            float4 s = __ldg(s4 + e4);
+            if (centered) {
+              s.x += 1.f; s.y += 1.f; s.z += 1.f; s.w += 1.f;
+            }
+            f[4 * e4 + 0] = f[4 * e4 + 0] * rinv * s.x;
+            f[4 * e4 + 1] = f[4 * e4 + 1] * rinv * s.y;
+            f[4 * e4 + 2] = f[4 * e4 + 2] * rinv * s.z;
+            f[4 * e4 + 3] = f[4 * e4 + 3] * rinv * s.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < P; ++e) f[e] *= rinv;
+        }
+        __stcs(yr + v, VT::pack(f));
+      }
+    }
+  }
+}
+
 // Any width and alignment: pass 1 sums squares, pass 2 rescales (re-read from L2).
 template <typename T>
 __global__ void __launch_bounds__(kNormWarps * 32)

@@ -388,10 +388,23 @@ tpl_status rmsnorm_launch(const void* x, int64_t M, int64_t H, const float* scal
   const bool vec = (H % P == 0) && aligned(x, 16) && aligned(y, 16) &&
                    (scale == nullptr || aligned(scale, 16));
   const int64_t lanes_vec = (H / P + 31) / 32;  // vectors per lane
+  const int64_t cta_vec = (H / P + tpl::kNormCtaThreads - 1) / tpl::kNormCtaThreads;
   const int g = static_cast<int>(blocks);
   const int t = tpl::kNormWarps * 32;
   const int Hi = static_cast<int>(H);
-  if (vec && lanes_vec <= 32) {
+  if (vec && H / P >= 2 * tpl::kNormCtaThreads && cta_vec <= 16) {
+    // Wide rows: a CTA per row, up to 16 CTAs resident per SM.
+    const int gc = static_cast<int>(std::min<int64_t>(M, static_cast<int64_t>(dev->sm_count) * 16));
+    const int tc = tpl::kNormCtaThreads;
+    if (cta_vec <= 2)
+      tpl::rmsnorm_cta<T, 2><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else if (cta_vec <= 4)
+      tpl::rmsnorm_cta<T, 4><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else if (cta_vec <= 8)
+      tpl::rmsnorm_cta<T, 8><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+    else
+      tpl::rmsnorm_cta<T, 16><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+  } else if (vec && lanes_vec <= 32) {
     if (lanes_vec <= 1)
       tpl::rmsnorm_reg<T, 1><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
     else if (lanes_vec <= 2)
