@@ -396,3 +396,102 @@ def rel_frobenius(got: np.ndarray, ref: np.ndarray) -> float:
     g = np.asarray(got, dtype=np.float64)
     o = np.asarray(ref, dtype=np.float64)
     return float(np.linalg.norm((g - o).ravel()) / np.linalg.norm(o.ravel()))
+
+
+# --------------------------------------------------------------------------
+# Next rows: sequence-parallel layouts, SwiGLU, vocab-sharded embedding
+# --------------------------------------------------------------------------
+
+def seq_scatter(y: np.ndarray, batch: int, seq: int, tp: int) -> np.ndarray:
+    """Rank-major sequence slices ``[tp][batch][seq/tp][N]`` of ``y [batch*seq, N]``.
+
+    nanotron "MLP Module": the row-parallel c_proj hands each rank the output
+    rows ``[batch, seq // tp, hidden]`` -- after the sum over ranks, rank r
+    keeps tokens ``r*seq/tp .. (r+1)*seq/tp`` of every sequence (a
+    reduce-scatter along the sequence).
+    """
+    y = np.asarray(y)
+    if seq % tp != 0:
+        raise OracleError("INDIVISIBLE", f"seq {seq} not divisible by tp {tp}")
+    n = y.shape[1]
+    return y.reshape(batch, tp, seq // tp, n).transpose(1, 0, 2, 3).copy()
+
+
+def seq_gather(x_sp: np.ndarray, batch: int, seq: int, tp: int) -> np.ndarray:
+    """Inverse of :func:`seq_scatter`: ``[batch*seq, N]`` from rank-major slices
+    (the all-gather along the sequence ahead of a column-parallel linear)."""
+    x_sp = np.asarray(x_sp)
+    n = x_sp.shape[-1]
+    return x_sp.reshape(tp, batch, seq // tp, n).transpose(1, 0, 2, 3).reshape(batch * seq, n)
+
+
+def row_linear_reduce_scatter(h, w2, batch: int, seq: int, bias=None,
+                              residual_sp=None) -> np.ndarray:
+    """Row-parallel linear whose summed output is scattered along the sequence.
+
+    Returns ``[tp][batch][seq/tp][N]``; a residual is given in the same layout.
+    """
+    tp = len(h)
+    y = row_linear_reduce(h, w2, bias, None)
+    out = seq_scatter(y, batch, seq, tp)
+    if residual_sp is not None:
+        out = out + np.asarray(residual_sp, dtype=np.float64)
+    return out
+
+
+def column_linear_allgather(x_sp, batch: int, seq: int, w, bias, part: Partition,
+                            act: str = "none") -> List[np.ndarray]:
+    """Column-parallel linear of sequence-sharded activations (gather, then a3)."""
+    return column_linear(seq_gather(x_sp, batch, seq, part.tp), w, bias, part, act)
+
+
+def silu(a: np.ndarray) -> np.ndarray:
+    """Swish with beta = 1: a * sigmoid(a) (the gate of SwiGLU)."""
+    a = np.asarray(a, dtype=np.float64)
+    return a / (1.0 + np.exp(-a))
+
+
+def swiglu_column_linear(x: np.ndarray, w: np.ndarray, F: int, tp: int) -> List[np.ndarray]:
+    """Column-parallel fused SwiGLU projection (google-research "SwiGLU" section).
+
+    ``w`` is the fused ``[wi0; wi1]`` weight ``[2F, K]``; it is partitioned as
+    two equal sub-parameters, rank r holding its slice of each, and returns
+    ``h_r = silu(X wi0_r^T) * (X wi1_r^T)``, ``[M, F_r]`` per rank.
+    Reading: "swish2" is taken as swish with beta = 1 (SiLU).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    if w.shape[0] != 2 * F:
+        raise OracleError("SHAPE", f"fused weight has {w.shape[0]} rows, expected {2 * F}")
+    part = partition_subparams([F, F], tp, 1)
+    out = []
+    for r in range(tp):
+        s0, n = part.src_off[r][0], part.width[r][0]
+        s1 = part.src_off[r][1]
+        a = x @ w[s0:s0 + n].T
+        b = x @ w[s1:s1 + n].T
+        out.append(silu(a) * b)
+    return out
+
+
+def embedding_lookup(ids: np.ndarray, table: np.ndarray, tp: int) -> np.ndarray:
+    """Vocab-sharded embedding (google-research ``embed_manual``, 'embed' scope).
+
+    Each rank r holds rows ``r*shard .. (r+1)*shard`` of the table; it looks up
+    ``one_x = x - vocab_start`` and keeps the row only where
+    ``0 <= one_x < shard_rows``; the sum over ranks is the embedding.  Ids
+    outside ``[0, V)`` embed to zeros.
+    """
+    ids = np.asarray(ids).reshape(-1)
+    table = np.asarray(table, dtype=np.float64)
+    V, H = table.shape
+    shard = -(-V // tp)
+    out = np.zeros((ids.size, H))
+    for r in range(tp):
+        start = r * shard
+        rows = max(0, min(shard, V - start))
+        for i, tok in enumerate(ids):
+            local = int(tok) - start
+            if 0 <= local < rows:
+                out[i] += table[start + local]
+    return out

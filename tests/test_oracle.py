@@ -392,3 +392,80 @@ def test_mlp_tp_invariance_and_stack_composition():
 def test_rel_frobenius():
     o = np.array([3.0, 4.0])
     assert O.rel_frobenius(o + np.array([0.0, 0.5]), o) == pytest.approx(0.1)
+
+
+# ------------------------------------------------- next rows (seq-parallel, SwiGLU, embed)
+
+def test_seq_scatter_gather_invariants():
+    rng = np.random.default_rng(11)
+    batch, seq, tp, n = 3, 8, 4, 5
+    y = rng.standard_normal((batch * seq, n))
+    sp = O.seq_scatter(y, batch, seq, tp)
+    assert sp.shape == (tp, batch, seq // tp, n)
+    # brute force: rank r holds tokens r*seq/tp .. of every sequence
+    for r in range(tp):
+        for b in range(batch):
+            for t in range(seq // tp):
+                np.testing.assert_array_equal(sp[r, b, t], y[b * seq + r * (seq // tp) + t])
+    np.testing.assert_array_equal(O.seq_gather(sp, batch, seq, tp), y)
+    with pytest.raises(O.OracleError):
+        O.seq_scatter(y, batch, seq, 3)
+
+
+def test_reduce_scatter_and_allgather_linears():
+    rng = np.random.default_rng(12)
+    batch, seq, tp, K, N = 2, 6, 3, 9, 4
+    M = batch * seq
+    hfull = rng.standard_normal((M, K))
+    w2 = rng.standard_normal((N, K))
+    kw = [3, 3, 3]
+    h = [hfull[:, 3 * r:3 * r + 3] for r in range(tp)]
+    res = rng.standard_normal((tp, batch, seq // tp, N))
+    got = O.row_linear_reduce_scatter(h, O.row_weight_slices(w2, kw), batch, seq, None, res)
+    full = hfull @ w2.T
+    for r in range(tp):
+        for b in range(batch):
+            for t in range(seq // tp):
+                np.testing.assert_allclose(got[r, b, t], full[b * seq + r * 2 + t] + res[r, b, t],
+                                           rtol=1e-13)
+    x = rng.standard_normal((M, K))
+    w = rng.standard_normal((6, K))
+    part = O.partition_subparams([6], tp, 1)
+    a = O.column_linear_allgather(O.seq_scatter(x, batch, seq, tp), batch, seq, w, None, part)
+    b = O.column_linear(x, w, None, part)
+    for u, v in zip(a, b):
+        np.testing.assert_allclose(u, v, rtol=1e-14)
+
+
+def test_silu_and_swiglu():
+    y = np.linspace(-20, 20, 801)
+    s = O.silu(y)
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    np.testing.assert_allclose(s - O.silu(-y), y, atol=1e-12)     # sigma(y) + sigma(-y) = 1
+    assert O.silu(np.array([1.0]))[0] == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
+    rng = np.random.default_rng(13)
+    M, K, F, tp = 4, 5, 6, 3
+    x = rng.standard_normal((M, K))
+    w = rng.standard_normal((2 * F, K))
+    got = O.swiglu_column_linear(x, w, F, tp)
+    # brute force: rank r's column c is output column r*F/tp + c of the unsharded SwiGLU
+    for r in range(tp):
+        for m in range(M):
+            for c in range(F // tp):
+                j = r * (F // tp) + c
+                a = sum(x[m][k] * w[j][k] for k in range(K))
+                b = sum(x[m][k] * w[F + j][k] for k in range(K))
+                assert got[r][m, c] == pytest.approx(a / (1 + math.exp(-a)) * b, rel=1e-12)
+
+
+def test_embedding_lookup_masks_and_sums():
+    rng = np.random.default_rng(14)
+    V, H, tp = 11, 4, 4                      # shard 3: ranks hold 3, 3, 3, 2 rows
+    table = rng.standard_normal((V, H))
+    ids = np.array([0, 2, 3, 10, 5, -1, 11, 40])
+    out = O.embedding_lookup(ids, table, tp)
+    for i, tok in enumerate(ids):
+        if 0 <= tok < V:
+            np.testing.assert_array_equal(out[i], table[tok])
+        else:
+            np.testing.assert_array_equal(out[i], 0.0)
