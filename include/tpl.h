@@ -170,6 +170,62 @@ tpl_status tpl_rmsnorm(const void* x, int64_t M, int64_t H, const float* scale, 
                        float eps, tpl_dtype dt, void* y, void* stream);
 
 /*
+ * Sequence parallelism around the TP linears (nanotron "MLP Module": the
+ * row-parallel c_proj hands rank r the rows [batch, seq // tp, hidden]).
+ * Activations of a sequence-parallel region are stored rank-major: rank r's
+ * slice [batch][seq/tp][*] (tokens r*seq/tp .. (r+1)*seq/tp of every sequence)
+ * starts at row r*batch*(seq/tp).  On one GPU the reduce-scatter and the
+ * all-gather are row remaps inside the GEMMs; no data moves twice.
+ *
+ * tpl_row_linear_reduce_scatter: as tpl_row_linear_reduce with M = batch*seq,
+ * but y (and residual, if given) are in the rank-major layout, so rank r's
+ * slice holds the summed output of its tokens.  seq % tp != 0 ->
+ * TPL_ERR_INDIVISIBLE.
+ */
+tpl_status tpl_row_linear_reduce_scatter(const void* h, const int64_t* k_w, int32_t tp,
+                                         int64_t batch, int64_t seq, int64_t N, const void* w,
+                                         const void* bias, const void* residual, tpl_dtype dt,
+                                         void* y, void* stream);
+
+/*
+ * tpl_column_linear_allgather: as tpl_column_linear with M = batch*seq, but x
+ * is read from the rank-major layout (the all-gather along the sequence that
+ * precedes a column-parallel linear), tp = p->tp_size.  The bf16 path needs
+ * (seq/tp) % 128 == 0 (else TPL_ERR_UNSUPPORTED).
+ */
+tpl_status tpl_column_linear_allgather(const tpl_partition* p, const void* x, int64_t batch,
+                                       int64_t seq, int64_t K, const void* w, const void* bias,
+                                       tpl_dtype dt, tpl_act act, void* y, void* stream);
+
+/*
+ * Column-parallel fused SwiGLU projection (google-research, "SwiGLU" section
+ * and the fused q_wi projection: swish(wi0) * wi1).
+ *
+ *   x   device bf16 [M][K].
+ *   w   device bf16 [2F][K]: the F rows of wi0, then the F rows of wi1.
+ *   h   device bf16; rank r's block [M][F_r] starts at element M*sum_{q<r} F_q,
+ *       F_r = F/tp + (r < F%tp); h_r = silu(X wi0_r^T) * (X wi1_r^T),
+ *       silu(a) = a / (1 + exp(-a)).
+ * Each 256-wide tile pairs a 128-column block of wi0 with the same block of
+ * wi1, so the gate is applied in the epilogue.  bf16 only (fp32 ->
+ * TPL_ERR_UNSUPPORTED); F < tp -> TPL_ERR_INDIVISIBLE.
+ */
+tpl_status tpl_swiglu_column_linear(const void* x, int64_t M, int64_t K, const void* w, int64_t F,
+                                    int32_t tp, tpl_dtype dt, void* h, void* stream);
+
+/*
+ * Vocab-sharded embedding lookup (google-research embed_manual, 'embed'
+ * scope): rank r holds table rows r*shard .. (r+1)*shard (shard = ceil(V/tp)),
+ * keeps its row where 0 <= id - r*shard < its row count, and the embedding is
+ * the sum over ranks (fp32, one rounding).  Ids outside [0, V) give zeros.
+ *
+ *   ids    device int32 [n].     table  device [V][H] (dtype dt).
+ *   out    device [n][H].        n == 0 is a no-op.
+ */
+tpl_status tpl_embedding_lookup(const int32_t* ids, int64_t n, const void* table, int64_t V,
+                                int64_t H, int32_t tp, tpl_dtype dt, void* out, void* stream);
+
+/*
  * Bytes of device workspace tpl_lmhead_argmax needs for B rows and tp shards.
  * Errors as for tpl_lmhead_argmax's shape checks.
  */

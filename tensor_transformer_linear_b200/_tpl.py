@@ -30,7 +30,8 @@ DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_reduce",
             "tpl_rmsnorm", "tpl_lmhead_workspace_size", "tpl_lmhead_argmax",
             "tpl_get_device_status", "tpl_status_string", "tpl_launch_count",
-            "tpl_lmhead_argmax_static")
+            "tpl_lmhead_argmax_static", "tpl_row_linear_reduce_scatter",
+            "tpl_column_linear_allgather", "tpl_swiglu_column_linear", "tpl_embedding_lookup")
 
 
 class TplError(RuntimeError):
@@ -82,6 +83,12 @@ def lib():
                                         vp]
         L.tpl_lmhead_argmax_static.argtypes = [vp, i64, i64, vp, i64, i32, i32, vp, vp, vp, vp,
                                                vp]
+        L.tpl_row_linear_reduce_scatter.argtypes = [vp, ctypes.POINTER(i64), i32, i64, i64, i64,
+                                                    vp, vp, vp, i32, vp, vp]
+        L.tpl_column_linear_allgather.argtypes = [ctypes.POINTER(Partition), vp, i64, i64, i64,
+                                                  vp, vp, i32, i32, vp, vp]
+        L.tpl_swiglu_column_linear.argtypes = [vp, i64, i64, vp, i64, i32, i32, vp, vp]
+        L.tpl_embedding_lookup.argtypes = [vp, i64, vp, i64, i64, i32, i32, vp, vp]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -273,6 +280,93 @@ def tpl_lmhead_argmax_static(x: torch.Tensor, w: torch.Tensor, tp: int, n_chunks
                                           _ptr(ids), _stream(stream)),
            "tpl_lmhead_argmax_static")
     return ids, shard_max, shard_idx
+
+
+def tpl_row_linear_reduce_scatter(h: torch.Tensor, k_w: Sequence[int], batch: int, seq: int,
+                                  w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                                  residual: Optional[torch.Tensor] = None,
+                                  y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Row-parallel linear; the summed output is returned rank-major ``[tp, batch, seq/tp, N]``."""
+    _cuda(h, "h")
+    dt = h.dtype
+    _cuda(w, "w", dt)
+    tp = len(k_w)
+    ktot = sum(int(k) for k in k_w)
+    M = batch * seq
+    if h.numel() != M * ktot or w.numel() % ktot != 0:
+        raise ValueError("h or w has the wrong size")
+    N = w.numel() // ktot
+    if y is None:
+        y = torch.empty((tp, batch, seq // tp, N), dtype=dt, device=h.device)
+    _cuda(y, "y", dt)
+    if residual is not None:
+        _cuda(residual, "residual", dt)
+    if bias is not None:
+        _cuda(bias, "bias", dt)
+    kw = (ctypes.c_int64 * tp)(*[int(k) for k in k_w])
+    _check(lib().tpl_row_linear_reduce_scatter(_ptr(h), kw, tp, int(batch), int(seq), int(N),
+                                               _ptr(w), _ptr(bias), _ptr(residual), DTYPE[dt],
+                                               _ptr(y), _stream(stream)),
+           "tpl_row_linear_reduce_scatter")
+    return y
+
+
+def tpl_column_linear_allgather(p: Partition, x_sp: torch.Tensor, batch: int, seq: int,
+                                w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                                act: str = "none", y: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """Column-parallel linear reading sequence-sharded, rank-major activations."""
+    _cuda(x_sp, "x")
+    dt = x_sp.dtype
+    _cuda(w, "w", dt)
+    K = x_sp.shape[-1]
+    M = batch * seq
+    if x_sp.numel() != M * K or w.numel() != p.logical_out * K:
+        raise ValueError("x or w has the wrong size")
+    if bias is not None:
+        _cuda(bias, "bias", dt)
+    if y is None:
+        y = torch.empty(M * p.logical_out, dtype=dt, device=x_sp.device)
+    _cuda(y, "y", dt)
+    _check(lib().tpl_column_linear_allgather(ctypes.byref(p), _ptr(x_sp), int(batch), int(seq),
+                                             int(K), _ptr(w), _ptr(bias), DTYPE[dt], ACT[act],
+                                             _ptr(y), _stream(stream)),
+           "tpl_column_linear_allgather")
+    return y
+
+
+def tpl_swiglu_column_linear(x: torch.Tensor, w: torch.Tensor, F: int, tp: int,
+                             h: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Fused SwiGLU column projection; rank r's ``[M, F_r]`` block at M * sum(F_q, q < r)."""
+    _cuda(x, "x")
+    dt = x.dtype
+    _cuda(w, "w", dt)
+    M, K = x.shape
+    if w.numel() != 2 * F * K:
+        raise ValueError("w must be [2F, K]")
+    if h is None:
+        h = torch.empty(M * F, dtype=dt, device=x.device)
+    _cuda(h, "h", dt)
+    _check(lib().tpl_swiglu_column_linear(_ptr(x), int(M), int(K), _ptr(w), int(F), int(tp),
+                                          DTYPE[dt], _ptr(h), _stream(stream)),
+           "tpl_swiglu_column_linear")
+    return h
+
+
+def tpl_embedding_lookup(ids: torch.Tensor, table: torch.Tensor, tp: int,
+                         out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Vocab-sharded embedding: ``[n, H]`` rows of ``table``, zeros for ids outside [0, V)."""
+    _cuda(ids, "ids", torch.int32)
+    _cuda(table, "table")
+    V, H = table.shape
+    n = ids.numel()
+    if out is None:
+        out = torch.empty((n, H), dtype=table.dtype, device=table.device)
+    _cuda(out, "out", table.dtype)
+    _check(lib().tpl_embedding_lookup(_ptr(ids), int(n), _ptr(table), int(V), int(H), int(tp),
+                                      DTYPE[table.dtype], _ptr(out), _stream(stream)),
+           "tpl_embedding_lookup")
+    return out
 
 
 def tpl_get_device_status(stream=None) -> int:

@@ -45,14 +45,20 @@ constexpr int kAccCols = 256;  // fp32 columns of one accumulator
 constexpr int kBiasSmemBytes = kEpiWarps * kHalfN * 4;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + kBiasSmemBytes + 1024 + 256;
 
-enum GemmMode : int { kModeColumn = 0, kModeRow = 1 };
+// kModeSwiglu: a column-parallel projection over a fused [wi0; wi1] weight
+// whose tiles pair a 128-column half block of wi0 with the same half block of
+// wi1, so the epilogue holds both operands of silu(a) * b (google-research
+// "SwiGLU" section) and writes 128 output columns per tile.
+enum GemmMode : int { kModeColumn = 0, kModeRow = 1, kModeSwiglu = 2 };
 
 struct ColPiece {
   int64_t out_off;   // element offset in y of (row 0, first column of the piece)
   int32_t src_row;   // first fused-weight row; also the fused-bias index
+  int32_t src_row1;  // SwiGLU mode: first wi1 row of the piece
   int32_t width;     // columns in the piece
   int32_t ld;        // row stride (elements) of the rank's shard
-  int32_t hb_begin;  // index of the piece's first 128-column half block
+  int32_t hb_begin;  // first 128-column half block (SwiGLU mode: first tile)
+  int32_t pad_;
 };
 
 struct GemmArgs {
@@ -73,7 +79,19 @@ struct GemmArgs {
   int32_t N;  // row mode output width
   const __nv_bfloat16* residual;
   float* partials;  // row mode: store this launch's fp32 sum here instead of y
+  // Sequence parallelism (nanotron "MLP Module": [batch, seq // tp, hidden] per
+  // rank): logical row m = b * seq + t lives at physical row
+  // (t / seg * batch + b) * seg + t % seg, seg = seq / tp (rank-major slices).
+  int32_t sp_batch, sp_seq, sp_seg;
+  int32_t a_remap;    // A rows are read from the rank-major layout (all-gather)
+  int32_t out_remap;  // output (and residual) rows use it (reduce-scatter)
 };
+
+__device__ __forceinline__ int64_t seq_row(const GemmArgs& a, int64_t m) {
+  const int64_t b = m / a.sp_seq, t = m - b * a.sp_seq;
+  const int64_t r = t / a.sp_seg, tl = t - r * a.sp_seg;
+  return (r * a.sp_batch + b) * a.sp_seg + tl;
+}
 
 struct HalfInfo {
   int32_t brow;     // weight row (column mode) or output column (row mode) of column 0
@@ -85,7 +103,19 @@ struct HalfInfo {
 
 __device__ __forceinline__ HalfInfo decode_half(const GemmArgs& a, int hb) {
   HalfInfo h;
-  if (a.mode == kModeColumn) {
+  if (a.mode == kModeSwiglu) {
+    // Half 0 of tile t is the wi0 block, half 1 the matching wi1 block.
+    const int t = hb >> 1;
+    int p = 0;
+    while (p + 1 < a.n_pieces && a.pieces[p + 1].hb_begin <= t) ++p;
+    const ColPiece& pc = a.pieces[p];
+    const int local = (t - pc.hb_begin) * kHalfN;
+    h.brow = ((hb & 1) ? pc.src_row1 : pc.src_row) + local;
+    h.valid = min(kHalfN, pc.width - local);
+    h.out_off = pc.out_off + local;
+    h.ld = pc.ld;
+    h.bias_off = 0;
+  } else if (a.mode == kModeColumn) {
     int p = 0;
     while (p + 1 < a.n_pieces && a.pieces[p + 1].hb_begin <= hb) ++p;
     const ColPiece& pc = a.pieces[p];
@@ -168,7 +198,8 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = apply_act_fast(v[j], a.act);
   }
-  const int64_t off = static_cast<int64_t>(m) * h.ld + h.out_off + col0;
+  const int64_t prow = a.out_remap ? seq_row(a, m) : static_cast<int64_t>(m);
+  const int64_t off = prow * h.ld + h.out_off + col0;
   if (a.residual != nullptr) {
     const __nv_bfloat16* res = a.residual + off;
     if (nvalid == 32 && a.vec_store) {
@@ -201,6 +232,52 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       if (j < nvalid) dst[j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+__device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
+
+// SwiGLU epilogue of 32 output columns of one row: silu(a) * b, stored bf16.
+__device__ __forceinline__ void store_swiglu_chunk(const GemmArgs& a, const HalfInfo& h, int m,
+                                                   int col0, const uint32_t (&ra)[32],
+                                                   const uint32_t (&rb)[32]) {
+  const int nvalid = min(32, h.valid - col0);
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = silu_fast(__uint_as_float(ra[j])) * __uint_as_float(rb[j]);
+  __nv_bfloat16* dst = a.y + static_cast<int64_t>(m) * h.ld + h.out_off + col0;
+  if (nvalid == 32 && a.vec_store) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint4 q;
+      q.x = pack_bf16x2(v[j + 0], v[j + 1]);
+      q.y = pack_bf16x2(v[j + 2], v[j + 3]);
+      q.z = pack_bf16x2(v[j + 4], v[j + 5]);
+      q.w = pack_bf16x2(v[j + 6], v[j + 7]);
+      *reinterpret_cast<uint4*>(dst + j) = q;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) dst[j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+// SwiGLU tile epilogue for one warp: TMEM columns 0..127 hold a = X wi0^T and
+// 128..255 hold b = X wi1^T for the same 128 output columns; epilogue warp
+// half hh writes output columns 64 hh .. 64 hh + 63.
+__device__ __forceinline__ void swiglu_epilogue(const GemmArgs& a, int nt, int m, int hh,
+                                                uint32_t tmem_row) {
+  const HalfInfo h0 = decode_half(a, 2 * nt);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int col0 = hh * 64 + c * 32;
+    if (col0 >= h0.valid) continue;
+    uint32_t ra[32], rb[32];
+    ptx::tmem_ld32(tmem_row + col0, ra);
+    ptx::tmem_ld32(tmem_row + kHalfN + col0, rb);
+    ptx::tmem_ld_wait();
+    if (m < a.M) store_swiglu_chunk(a, h0, m, col0, ra, rb);
   }
 }
 
@@ -271,8 +348,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sB = sA + kABytes;
           ptx::mbar_arrive_expect_tx(&full[stage], bytes);
           const int kc = (ki % a.k_iters) * kBK;
-          if (a.mode == kModeColumn) {
-            ptx::tma_load_2d_nohint(sA, &a.tmA, &full[stage], kc, mb * kBM);
+          if (a.mode != kModeRow) {
+            const int arow = a.a_remap ? static_cast<int>(seq_row(a, mb * kBM)) : mb * kBM;
+            ptx::tma_load_2d_nohint(sA, &a.tmA, &full[stage], kc, arow);
             ptx::tma_load_2d_nohint(sB, &a.tmB, &full[stage], kc, h0.brow);
             if (has1) ptx::tma_load_2d_nohint(sB + kBHalfBytes, &a.tmB, &full[stage], kc, h1.brow);
           } else {
@@ -395,7 +473,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       ptx::tc_fence_after();
-      if (active) {
+      if (a.mode == kModeSwiglu) {
+        swiglu_epilogue(a, nt, mb * kBM + row, hh,
+                        tmem_base + ((q * 32u) << 16) + acc * kAccCols);
+      } else if (active) {
         const int m = mb * kBM + row;
         for (int c = 0; c < kHalfN / 32; ++c) {
           uint32_t r[32];

@@ -101,8 +101,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           uint8_t* sB = sA + kABytes;
           const uint32_t bar = full_lead + 8u * stage;
           const int kc = (ki % a.k_iters) * kBK;
-          if (a.mode == kModeColumn) {
-            ptx::tma_load_2d_pair(sA, &a.tmA, bar, kc, m_row);
+          if (a.mode != kModeRow) {
+            const int arow = a.a_remap ? static_cast<int>(seq_row(a, m_row)) : m_row;
+            ptx::tma_load_2d_pair(sA, &a.tmA, bar, kc, arow);
             ptx::tma_load_2d_pair(sB, &a.tmB, bar, kc, h.brow);
           } else {
             const int r = a.r0 + ki / a.k_iters;
@@ -196,7 +197,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         break;
       }
       ptx::tc_fence_after();
-      if (active) {
+      if (a.mode == kModeSwiglu) {
+        swiglu_epilogue(a, nt, mb * kPairBM + static_cast<int>(rank) * kBM + row, hh,
+                        tmem_base + ((q * 32u) << 16) + acc * kAccCols);
+      } else if (active) {
         const int m = mb * kPairBM + static_cast<int>(rank) * kBM + row;
         for (int c = 0; c < kHalfN / 32; ++c) {
           float bv[32];

@@ -44,7 +44,17 @@ struct F32Args {
   const float* h;
   const float* residual;
   float* partials;  // when set: write this launch's fp32 sum here (no bias/residual)
+  // Sequence parallelism, as in GemmArgs: rank-major rows for A (a_remap) or for
+  // the output and residual (out_remap).
+  int32_t sp_batch, sp_seq, sp_seg;
+  int32_t a_remap, out_remap;
 };
+
+__device__ __forceinline__ int64_t seq_row_f32(const F32Args& a, int64_t m) {
+  const int64_t b = m / a.sp_seq, t = m - b * a.sp_seq;
+  const int64_t r = t / a.sp_seg, tl = t - r * a.sp_seg;
+  return (r * a.sp_batch + b) * a.sp_seg + tl;
+}
 
 __global__ void __launch_bounds__(kF32Threads) gemm_fp32_simt(const __grid_constant__ F32Args a) {
   __shared__ float As[kF32BK][kF32BM + 4];
@@ -102,7 +112,8 @@ __global__ void __launch_bounds__(kF32Threads) gemm_fp32_simt(const __grid_const
       for (int i = threadIdx.x; i < kF32BM * kF32BK; i += kF32Threads) {
         const int mm = i / kF32BK, kk = i % kF32BK;
         const int64_t gm = m0 + mm;
-        As[kk][mm] = (gm < a.M && k0 + kk < Kr) ? A[gm * lda + k0 + kk] : 0.f;
+        const int64_t am = (a.a_remap && gm < a.M) ? seq_row_f32(a, gm) : gm;
+        As[kk][mm] = (gm < a.M && k0 + kk < Kr) ? A[am * lda + k0 + kk] : 0.f;
       }
       for (int i = threadIdx.x; i < kF32BN * kF32BK; i += kF32Threads) {
         const int nn = i / kF32BK, kk = i % kF32BK;
@@ -135,7 +146,8 @@ __global__ void __launch_bounds__(kF32Threads) gemm_fp32_simt(const __grid_const
       const int c = tx * 4 + j;
       if (c >= valid) continue;
       float v = acc[i][j];
-      const int64_t off = m * ld + out0 + c;
+      const int64_t prow = a.out_remap ? seq_row_f32(a, m) : m;
+      const int64_t off = prow * ld + out0 + c;
       if (a.partials != nullptr) {
         a.partials[off] = v;
         continue;

@@ -161,10 +161,26 @@ int act_ok(int act) {
   return act == TPL_ACT_NONE || act == TPL_ACT_GELU_ERF || act == TPL_ACT_GELU_TANH;
 }
 
+// Sequence-parallel row layout (rank-major token slices); all zero = plain rows.
+struct SeqPar {
+  int32_t batch = 0, seq = 0, seg = 0;
+  int32_t a_remap = 0, out_remap = 0;
+};
+
+template <typename Args>
+void set_seqpar(Args& a, const SeqPar& sp) {
+  a.sp_batch = sp.batch;
+  a.sp_seq = sp.seq;
+  a.sp_seg = sp.seg;
+  a.a_remap = sp.a_remap;
+  a.out_remap = sp.out_remap;
+}
+
 // ------------------------------------------------------------------ column
 
 tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
-                       const void* bias, int act, void* y, cudaStream_t st) {
+                       const void* bias, int act, void* y, cudaStream_t st,
+                       const SeqPar& sp = SeqPar{}) {
   if ((K % 8) != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 2) ||
       (bias != nullptr && !aligned(bias, 2)))
     return TPL_ERR_ALIGN;
@@ -187,6 +203,7 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
   a.mode = tpl::kModeColumn;
   a.act = act;
   a.M = static_cast<int32_t>(M);
+  set_seqpar(a, sp);
   a.k_iters = static_cast<int32_t>((K + tpl::kBK - 1) / tpl::kBK);
   a.bias = static_cast<const __nv_bfloat16*>(bias);
   a.y = static_cast<__nv_bfloat16*>(y);
@@ -223,7 +240,8 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
 }
 
 tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
-                       const void* bias, int act, void* y, cudaStream_t st) {
+                       const void* bias, int act, void* y, cudaStream_t st,
+                       const SeqPar& sp = SeqPar{}) {
   if (!aligned(x, 4) || !aligned(w, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4)))
     return TPL_ERR_ALIGN;
   tpl::F32Args a;
@@ -231,6 +249,7 @@ tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t
   a.mode = 0;
   a.act = act;
   a.M = M;
+  set_seqpar(a, sp);
   a.K = static_cast<int32_t>(K);
   a.x = static_cast<const float*>(x);
   a.w = static_cast<const float*>(w);
@@ -272,7 +291,7 @@ tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t
 
 tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_t N, const void* w,
                     const void* bias, const void* residual, void* y, float* partials,
-                    cudaStream_t st) {
+                    cudaStream_t st, const SeqPar& sp = SeqPar{}) {
   for (int r = 0; r < tp; ++r)
     if (k_w[r] % 8 != 0) return TPL_ERR_ALIGN;
   if (!aligned(h, 16) || !aligned(w, 16) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||
@@ -301,6 +320,7 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   }
   a.mode = tpl::kModeRow;
   a.M = static_cast<int32_t>(M);
+  set_seqpar(a, sp);
   a.N = static_cast<int32_t>(N);
   a.k_iters = static_cast<int32_t>((Kr + tpl::kBK - 1) / tpl::kBK);
   a.n_halves = static_cast<int32_t>((N + tpl::kHalfN - 1) / tpl::kHalfN);
@@ -332,7 +352,7 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
 
 tpl_status row_fp32(const void* h, const int64_t* k_w, int tp, int64_t M, int64_t N, const void* w,
                     const void* bias, const void* residual, void* y, float* partials,
-                    cudaStream_t st) {
+                    cudaStream_t st, const SeqPar& sp = SeqPar{}) {
   if (!aligned(h, 4) || !aligned(w, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4)) ||
       (residual && !aligned(residual, 4)) || (partials && !aligned(partials, 4)))
     return TPL_ERR_ALIGN;
@@ -340,6 +360,7 @@ tpl_status row_fp32(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   std::memset(&a, 0, sizeof(a));
   a.mode = 1;
   a.M = M;
+  set_seqpar(a, sp);
   a.N = static_cast<int32_t>(N);
   a.h = static_cast<const float*>(h);
   a.w = static_cast<const float*>(w);
@@ -712,3 +733,6 @@ extern "C" tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t
   return tpl_lmhead_argmax(x, B, K, w, V, tp, n_chunks, logits, shard_max, shard_idx, ids, scratch,
                            static_cast<size_t>(TPL_LMHEAD_STATIC_SCRATCH_BYTES), stream);
 }
+
+// Entry points of the next rows (same translation unit).
+#include "tpl_next.cuh"

@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 10, names
+    assert len(names) == 14, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -174,3 +174,28 @@ def test_lmhead_layout_and_rejections():
     assert L.tpl_lmhead_argmax(*args(wsb=n - 1)) == 2
     assert L.tpl_lmhead_argmax(*args(K=60)) == 5
     assert L.tpl_lmhead_argmax(*args(w=FAKE_ODD)) == 5
+
+
+def test_next_rows_rejections():
+    L = T.lib()
+    s = ctypes.c_void_p(0)
+    kw = (ctypes.c_int64 * 4)(64, 64, 64, 64)
+    # seq not divisible by tp
+    assert L.tpl_row_linear_reduce_scatter(FAKE, kw, 4, 2, 10, 8, FAKE, None, None, 1, FAKE, s) == 3
+    assert L.tpl_row_linear_reduce_scatter(FAKE, None, 4, 2, 8, 8, FAKE, None, None, 1, FAKE, s) == 1
+    assert L.tpl_row_linear_reduce_scatter(FAKE, kw, 4, 0, 8, 8, FAKE, None, None, 1, FAKE, s) == 2
+    p = T.tpl_partition_subparams([256], 4, 1)
+    bp = ctypes.byref(p)
+    assert L.tpl_column_linear_allgather(bp, FAKE, 2, 6, 64, FAKE, None, 1, 0, FAKE, s) == 3
+    assert L.tpl_column_linear_allgather(bp, FAKE, 2, 64, 64, FAKE, None, 1, 0, FAKE, s) == 8
+    assert L.tpl_column_linear_allgather(None, FAKE, 2, 64, 64, FAKE, None, 1, 0, FAKE, s) == 1
+    # SwiGLU: bf16 only; ranks without rows; bad sizes
+    assert L.tpl_swiglu_column_linear(FAKE, 4, 64, FAKE, 256, 4, 0, FAKE, s) == 8
+    assert L.tpl_swiglu_column_linear(FAKE, 4, 64, FAKE, 2, 4, 1, FAKE, s) == 3
+    assert L.tpl_swiglu_column_linear(FAKE, 4, 60, FAKE, 256, 4, 1, FAKE, s) == 5
+    assert L.tpl_swiglu_column_linear(None, 0, 64, None, 256, 4, 1, None, s) == 0
+    # embedding
+    assert L.tpl_embedding_lookup(FAKE, -1, FAKE, 10, 8, 2, 1, FAKE, s) == 2
+    assert L.tpl_embedding_lookup(None, 0, None, 10, 8, 2, 1, None, s) == 0
+    assert L.tpl_embedding_lookup(FAKE, 4, FAKE, 10, 8, 65, 1, FAKE, s) == 2
+    assert L.tpl_embedding_lookup(FAKE, 4, FAKE_ODD, 10, 8, 2, 1, FAKE, s) == 5
