@@ -224,8 +224,10 @@ class Block:
     def lmhead_bytes(self):
         return self.l.algorithmic_bytes() if "lmhead" in self.sel else None
 
-    def rmsnorm_bytes(self):
-        return 2 * 2 * self.m.M * self.m.hidden if "mlp" in self.sel else None
+    def hbm_parts(self):
+        if "mlp" not in self.sel:
+            return []
+        return [("roofline_rmsnorm", "rmsnorm_cta", "rmsnorm", 2 * 2 * self.m.M * self.m.hidden)]
 
     # --- the oracle on a bounded sample (CPU baseline / reference arm)
     def oracle_sample(self, rows_qkv=256, rows_mlp=96, lm_rows=16032):
@@ -315,8 +317,8 @@ class Stack:
     def lmhead_bytes(self):
         return None
 
-    def rmsnorm_bytes(self):
-        return None
+    def hbm_parts(self):
+        return []
 
     def gemm_part_ids(self):
         return [i for i in range(len(self.parts)) if i % 3 != 0]
@@ -336,10 +338,144 @@ class Stack:
             f"{rows} token rows through all {w.layers} layers"
 
 
+class NextRows:
+    """Workloads of the path's next rows, one at a time (measured like the block).
+
+    swiglu: fused [wi0; wi1] column projection x[8192,4096] -> 2 x 14336, tp 8
+            (full d_ff per gate, as the PaLM note on the page says).
+    embed:  vocab-sharded lookup of 8192 token ids in W[128256,4096] bf16, tp 8.
+    seqpar: the RMSNorm + TP MLP block in sequence-parallel form (x[8,1024,4096],
+            tp 8): RMSNorm of the rank-major slices -> all-gather c_fc + GELU ->
+            c_proj with the reduce-scatter and residual.
+    """
+
+    def __init__(self, dev, kind):
+        import tensor_transformer_linear_b200 as T
+        self.T, self.kind = T, kind
+        m, l = C.TP_MLP, C.LM_HEAD
+        self.m, self.l = m, l
+        self.flops = 0.0
+        self.gemm_flops = 0.0
+        self.hbm_bytes = 0
+        self.launches = []
+        if kind == "swiglu":
+            self.F = m.inter
+            self.name = (f"fused-swiglu-column x[8,1024,4096] bf16 4096->2x{self.F} tp{m.tp}")
+            self.x = C.mlp_x(m, dev)
+            self.w = gen.normal((2 * self.F, m.hidden), m.w_sigma, tensor_id=gen.TID_W1,
+                                device=dev)
+            self.h = torch.empty(m.M * self.F, dtype=torch.bfloat16, device=dev)
+            self.launches.append(("swiglu_column", lambda s: T.tpl_swiglu_column_linear(
+                self.x, self.w, self.F, m.tp, h=self.h, stream=s)))
+            self.flops = self.gemm_flops = 2.0 * m.M * m.hidden * 2 * self.F
+            self.d_in, self.d_out = [self.x], [self.h]
+        elif kind == "embed":
+            self.name = (f"vocab-sharded-embedding ids[8,1024] W[{l.vocab},{l.hidden}] bf16 "
+                         f"tp{l.tp}")
+            g = torch.Generator(device=dev)
+            g.manual_seed(0)
+            self.ids = torch.randint(0, l.vocab, (m.M,), generator=g, device=dev,
+                                     dtype=torch.int32)
+            self.table = C.lm_w(l, dev)
+            self.out = torch.empty((m.M, l.hidden), dtype=torch.bfloat16, device=dev)
+            self.launches.append(("embed_lookup", lambda s: T.tpl_embedding_lookup(
+                self.ids, self.table, l.tp, out=self.out, stream=s)))
+            self.hbm_bytes = m.M * l.hidden * 2 * 2 + m.M * 4
+            self.d_in, self.d_out = [self.ids], [self.out]
+        elif kind == "seqpar":
+            b, sq = m.batch, m.seq
+            self.name = (f"sequence-parallel rmsnorm-tp-mlp x[{b},{sq},{m.hidden}] bf16 "
+                         f"{m.hidden}->{m.inter}->{m.hidden} tp{m.tp}")
+            self.x = C.mlp_x(m, dev)      # read as the rank-major [tp][b][s/tp][H] layout
+            self.scale = C.mlp_scale(m, 0, dev)
+            self.w1 = C.mlp_w1(m, 0, dev)
+            self.part = T.tpl_partition_subparams([m.inter], m.tp, 1)
+            self.k_w = [self.part.shard_width[r] for r in range(m.tp)]
+            self.w2 = T.pack_row_weight(C.mlp_w2(m, 0, dev), self.k_w)
+            self.xn = torch.empty_like(self.x)
+            self.hbuf = torch.empty(m.M * m.inter, dtype=torch.bfloat16, device=dev)
+            self.y = torch.empty_like(self.x)
+            self.launches += [
+                ("sp_rmsnorm", lambda s: T.tpl_rmsnorm(self.x, self.scale, True, 1e-6,
+                                                       y=self.xn, stream=s)),
+                ("sp_column_gelu", lambda s: T.tpl_column_linear_allgather(
+                    self.part, self.xn, b, sq, self.w1, None, m.act, y=self.hbuf, stream=s)),
+                ("sp_row_scatter", lambda s: T.tpl_row_linear_reduce_scatter(
+                    self.hbuf, self.k_w, b, sq, self.w2, None, self.x, y=self.y, stream=s))]
+            self.flops = self.gemm_flops = m.flops()
+            self.d_in, self.d_out = [self.x], [self.y]
+        else:
+            raise ValueError(kind)
+        self.parts = [n for n, _ in self.launches]
+
+    def step(self, stream, events=None):
+        for i, (_, fn) in enumerate(self.launches):
+            if events is not None:
+                events[i].record(stream)
+            fn(stream)
+        if events is not None:
+            events[len(self.launches)].record(stream)
+
+    def gemm_part_ids(self):
+        return [i for i, n in enumerate(self.parts)
+                if n in ("swiglu_column", "sp_column_gelu", "sp_row_scatter")]
+
+    def lmhead_bytes(self):
+        return None
+
+    def hbm_parts(self):
+        if self.kind == "embed":
+            return [("roofline_embed", "embedding_lookup_kernel", "embed_lookup", self.hbm_bytes)]
+        if self.kind == "seqpar":
+            return [("roofline_rmsnorm", "rmsnorm_cta", "sp_rmsnorm",
+                     2 * 2 * self.m.M * self.m.hidden)]
+        return []
+
+    def host_io(self):
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+        self.h_in = [pin(t.cpu()) for t in self.d_in]
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in self.d_out]
+        return (sum(t.numel() * t.element_size() for t in self.h_in),
+                sum(t.numel() * t.element_size() for t in self.h_out))
+
+    def step_e2e(self, stream):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.step(stream)
+        for h, d in zip(self.h_out, self.d_out):
+            h.copy_(d, non_blocking=True)
+
+    def oracle_sample(self, rows=64):
+        import numpy as np
+        import oracle as O
+        f64 = lambda t: t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
+        m, l = self.m, self.l
+        if self.kind == "swiglu":
+            xs, w = f64(self.x[:rows]), f64(self.w)
+            return (lambda: O.swiglu_column_linear(xs, w, self.F, m.tp),
+                    2.0 * rows * m.hidden * 2 * self.F, f"{rows} token rows")
+        if self.kind == "embed":
+            sub = 16032
+            table = f64(self.table[:sub])
+            ids = (self.ids[:4096] % sub).cpu().numpy()
+            return (lambda: O.embedding_lookup(ids, table, l.tp),
+                    ids.size * l.hidden * 2 * 2 + ids.size * 4,
+                    f"{ids.size} ids over a {sub}-row slice of the table")
+        xs = f64(self.x[:rows])
+        w1, w2 = f64(self.w1), f64(C.mlp_w2(m, 0, self.x.device))
+        sc = f64(self.scale)
+        return (lambda: O.tp_mlp(xs, w1, w2, m.tp, m.act, scale=sc, centered=True, norm=True,
+                                 residual=True),
+                4.0 * rows * m.hidden * m.inter, f"{rows} tokens through the block")
+
+
 WORKLOADS = {"block": Block, "stack": Stack,
              "qkv": lambda dev: Block(dev, ("qkv",)),
              "mlp": lambda dev: Block(dev, ("mlp",)),
-             "lmhead": lambda dev: Block(dev, ("lmhead",))}
+             "lmhead": lambda dev: Block(dev, ("lmhead",)),
+             "swiglu": lambda dev: NextRows(dev, "swiglu"),
+             "embed": lambda dev: NextRows(dev, "embed"),
+             "seqpar": lambda dev: NextRows(dev, "seqpar")}
 
 
 # ------------------------------------------------------------------ timing
@@ -577,15 +713,21 @@ def main():
                     "frac_of_8000": round(dg / 8000.0, 4), "ms_per_launch": round(decode_ms, 4),
                     "measured": f"{DECODE_LAUNCHES} back-to-back launches (a decode loop), "
                                 "CUDA events on the launching stream"}
-        rb = wl.rmsnorm_bytes()
-        if rb is not None:
-            r_ms = part_ms[wl.parts.index("rmsnorm")]
-            line["roofline_rmsnorm"] = {"kernel": "rmsnorm_cta", "bound": "hbm",
-                                        "achieved": round(rb / (r_ms * 1e-3) / 1e9, 1),
-                                        "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                        "frac": round(rb / (r_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        for key, kern, part, nbytes in wl.hbm_parts():
+            p_ms = part_ms[wl.parts.index(part)]
+            gb = nbytes / (p_ms * 1e-3) / 1e9
+            line[key] = {"kernel": kern, "bound": "hbm", "achieved": round(gb, 1),
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gb / pk["hbm_gbs"], 4), "bytes_per_launch": nbytes}
         if not gids:
-            line["roofline"] = line.pop("roofline_lmhead")
+            first = "roofline_lmhead" if "roofline_lmhead" in line else wl.hbm_parts()[0][0]
+            line["roofline"] = line.pop(first)
+        if wl.flops == 0:
+            # a bandwidth-only workload: the rate is bytes moved per second
+            line["value"] = round(wl.hbm_bytes / (step_ms * 1e-3) / 1e9 * world, 1)
+            line["unit"] = "GB/s"
+            line["e2e"]["value"] = round(wl.hbm_bytes / (e_ms / e_steps * 1e-3) / 1e9 * world, 1)
+            line["e2e"]["unit"] = "GB/s"
         if world == 1 and not args.no_cpu_baseline:
             run, flops, desc = wl.oracle_sample()
             v, reps, dt = time_oracle(run, flops)

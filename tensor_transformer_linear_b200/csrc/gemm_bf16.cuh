@@ -87,10 +87,18 @@ struct GemmArgs {
   int32_t out_remap;  // output (and residual) rows use it (reduce-scatter)
 };
 
-__device__ __forceinline__ int64_t seq_row(const GemmArgs& a, int64_t m) {
-  const int64_t b = m / a.sp_seq, t = m - b * a.sp_seq;
-  const int64_t r = t / a.sp_seg, tl = t - r * a.sp_seg;
-  return (r * a.sp_batch + b) * a.sp_seg + tl;
+__device__ __forceinline__ int seq_row(const GemmArgs& a, int m) {
+  const unsigned b = static_cast<unsigned>(m) / static_cast<unsigned>(a.sp_seq);
+  const unsigned t = static_cast<unsigned>(m) - b * static_cast<unsigned>(a.sp_seq);
+  const unsigned r = t / static_cast<unsigned>(a.sp_seg);
+  const unsigned tl = t - r * static_cast<unsigned>(a.sp_seg);
+  return static_cast<int>((r * static_cast<unsigned>(a.sp_batch) + b) *
+                              static_cast<unsigned>(a.sp_seg) + tl);
+}
+
+// Physical output row of logical row m (rank-major when the output is scattered).
+__device__ __forceinline__ int out_row(const GemmArgs& a, int m) {
+  return a.out_remap ? seq_row(a, m) : m;
 }
 
 struct HalfInfo {
@@ -169,8 +177,9 @@ __device__ __forceinline__ void load_bias_chunk(const GemmArgs& a, const HalfInf
 }
 
 // Epilogue of 32 accumulator columns of one row; bv holds the chunk's bias.
-__device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h, int m, int col0,
-                                            const uint32_t (&r)[32], const float (&bv)[32]) {
+__device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h, int m, int prow,
+                                            int col0, const uint32_t (&r)[32],
+                                            const float (&bv)[32]) {
   const int nvalid = min(32, h.valid - col0);
   float v[32];
 #pragma unroll
@@ -198,8 +207,7 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = apply_act_fast(v[j], a.act);
   }
-  const int64_t prow = a.out_remap ? seq_row(a, m) : static_cast<int64_t>(m);
-  const int64_t off = prow * h.ld + h.out_off + col0;
+  const int64_t off = static_cast<int64_t>(prow) * h.ld + h.out_off + col0;
   if (a.residual != nullptr) {
     const __nv_bfloat16* res = a.residual + off;
     if (nvalid == 32 && a.vec_store) {
@@ -339,6 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const HalfInfo h0 = decode_half(a, 2 * nt);
         const HalfInfo h1 = has1 ? decode_half(a, 2 * nt + 1) : h0;
         const uint32_t bytes = kABytes + (has1 ? 2 : 1) * kBHalfBytes;
+        const int arow = a.a_remap ? seq_row(a, mb * kBM) : mb * kBM;
         for (int ki = 0; ki < k_total; ++ki) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -349,7 +358,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ptx::mbar_arrive_expect_tx(&full[stage], bytes);
           const int kc = (ki % a.k_iters) * kBK;
           if (a.mode != kModeRow) {
-            const int arow = a.a_remap ? static_cast<int>(seq_row(a, mb * kBM)) : mb * kBM;
             ptx::tma_load_2d_nohint(sA, &a.tmA, &full[stage], kc, arow);
             ptx::tma_load_2d_nohint(sB, &a.tmB, &full[stage], kc, h0.brow);
             if (has1) ptx::tma_load_2d_nohint(sB + kBHalfBytes, &a.tmB, &full[stage], kc, h1.brow);
@@ -478,6 +486,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tmem_base + ((q * 32u) << 16) + acc * kAccCols);
       } else if (active) {
         const int m = mb * kBM + row;
+        const int prow = out_row(a, m);
         for (int c = 0; c < kHalfN / 32; ++c) {
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
@@ -486,7 +495,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float bv[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) bv[j] = bias_s[c * 32 + j];
-            store_chunk(a, h, m, c * 32, r, bv);
+            store_chunk(a, h, m, prow, c * 32, r, bv);
           }
         }
       }

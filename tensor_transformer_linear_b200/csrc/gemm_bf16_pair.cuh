@@ -91,6 +91,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // This CTA's half of B; an odd last half is padded with the even one.
         const HalfInfo h = decode_half(a, (rank == 1 && has1) ? 2 * nt + 1 : 2 * nt);
         const int m_row = mb * kPairBM + static_cast<int>(rank) * kBM;
+        const int arow = a.a_remap ? seq_row(a, m_row) : m_row;
         for (int ki = 0; ki < k_total; ++ki) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -102,7 +103,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t bar = full_lead + 8u * stage;
           const int kc = (ki % a.k_iters) * kBK;
           if (a.mode != kModeRow) {
-            const int arow = a.a_remap ? static_cast<int>(seq_row(a, m_row)) : m_row;
             ptx::tma_load_2d_pair(sA, &a.tmA, bar, kc, arow);
             ptx::tma_load_2d_pair(sB, &a.tmB, bar, kc, h.brow);
           } else {
@@ -202,13 +202,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         tmem_base + ((q * 32u) << 16) + acc * kAccCols);
       } else if (active) {
         const int m = mb * kPairBM + static_cast<int>(rank) * kBM + row;
+        const int prow = out_row(a, m);
         for (int c = 0; c < kHalfN / 32; ++c) {
           float bv[32];
           if (a.bias != nullptr && c * 32 < h.valid) load_bias_chunk(a, h, c * 32, bv);
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
           ptx::tmem_ld_wait();
-          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, c * 32, r, bv);
+          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, prow, c * 32, r, bv);
         }
       }
       ptx::tc_fence_before();
