@@ -619,7 +619,7 @@ def main():
 
     # ---- the LM head in a decode loop: back-to-back launches, as once per decode step
     decode_ms = None
-    lm = dict(wl.launches).get("lmhead_argmax")
+    lm = dict(getattr(wl, "launches", [])).get("lmhead_argmax")
     if lm is not None:
         for _ in range(3):
             lm(stream)

@@ -31,7 +31,8 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_rmsnorm", "tpl_lmhead_workspace_size", "tpl_lmhead_argmax",
             "tpl_get_device_status", "tpl_status_string", "tpl_launch_count",
             "tpl_lmhead_argmax_static", "tpl_row_linear_reduce_scatter",
-            "tpl_column_linear_allgather", "tpl_swiglu_column_linear", "tpl_embedding_lookup")
+            "tpl_column_linear_allgather", "tpl_swiglu_column_linear", "tpl_embedding_lookup",
+            "tpl_selftest_wait_timeout")
 
 
 class TplError(RuntimeError):
@@ -89,6 +90,7 @@ def lib():
                                                   vp, vp, i32, i32, vp, vp]
         L.tpl_swiglu_column_linear.argtypes = [vp, i64, i64, vp, i64, i32, i32, vp, vp]
         L.tpl_embedding_lookup.argtypes = [vp, i64, vp, i64, i64, i32, i32, vp, vp]
+        L.tpl_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -367,6 +369,15 @@ def tpl_embedding_lookup(ids: torch.Tensor, table: torch.Tensor, tp: int,
                                       DTYPE[table.dtype], _ptr(out), _stream(stream)),
            "tpl_embedding_lookup")
     return out
+
+
+def tpl_selftest_wait_timeout(limit_ns: int, waited_us: Optional[torch.Tensor] = None,
+                              stream=None) -> None:
+    """Run the bounded-wait failure path once (see include/tpl.h)."""
+    if waited_us is not None:
+        _cuda(waited_us, "waited_us", torch.int32)
+    _check(lib().tpl_selftest_wait_timeout(int(limit_ns), _ptr(waited_us), _stream(stream)),
+           "tpl_selftest_wait_timeout")
 
 
 def tpl_get_device_status(stream=None) -> int:

@@ -62,8 +62,10 @@ struct ColPiece {
 };
 
 struct GemmArgs {
-  CUtensorMap tmA;  // column: X {K, M};      row: H  {Kr, M, tp}
-  CUtensorMap tmB;  // column: W {K, rows};   row: W2 {Kr, N, tp}
+  CUtensorMap tmA;  // column: X {K, M};      row: H  {Kr, M, tp} of ranks 0 .. r_split-1
+  CUtensorMap tmB;  // column: W {K, rows};   row: W2 {Kr, N, tp} of ranks 0 .. r_split-1
+  CUtensorMap tmA2;  // row mode, ranks r_split .. tp-1 (a second contraction width)
+  CUtensorMap tmB2;
   int32_t mode;
   int32_t act;
   int32_t M;
@@ -85,7 +87,18 @@ struct GemmArgs {
   int32_t sp_batch, sp_seq, sp_seg;
   int32_t a_remap;    // A rows are read from the rank-major layout (all-gather)
   int32_t out_remap;  // output (and residual) rows use it (reduce-scatter)
+  // Row mode with two contraction widths: ranks below r_split use tmA/tmB and
+  // k_iters K blocks, the others tmA2/tmB2 and k_iters2 (r_split = tp if equal).
+  int32_t r_split, k_iters2;
 };
+
+// Number of 64-wide K steps of one tile.
+__device__ __forceinline__ int k_steps(const GemmArgs& a) {
+  if (a.mode != kModeRow) return a.k_iters;
+  const int n1 = max(0, min(a.r1, a.r_split) - a.r0);
+  const int n2 = max(0, a.r1 - max(a.r0, a.r_split));
+  return n1 * a.k_iters + n2 * a.k_iters2;
+}
 
 __device__ __forceinline__ int seq_row(const GemmArgs& a, int m) {
   const unsigned b = static_cast<unsigned>(m) / static_cast<unsigned>(a.sp_seq);
@@ -320,6 +333,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&a.tmA);
     ptx::prefetch_tmap(&a.tmB);
+    if (a.mode == kModeRow && a.r_split < a.r1) {
+      ptx::prefetch_tmap(&a.tmA2);
+      ptx::prefetch_tmap(&a.tmB2);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, 2 * kAccCols);
@@ -330,8 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int nr = (a.mode == kModeRow) ? (a.r1 - a.r0) : 1;
-  const int k_total = nr * a.k_iters;
+  const int k_total = k_steps(a);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -348,6 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const HalfInfo h1 = has1 ? decode_half(a, 2 * nt + 1) : h0;
         const uint32_t bytes = kABytes + (has1 ? 2 : 1) * kBHalfBytes;
         const int arow = a.a_remap ? seq_row(a, mb * kBM) : mb * kBM;
+        int rr = a.r0, kb = 0;  // row mode: rank and K block of the next step
         for (int ki = 0; ki < k_total; ++ki) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -356,17 +373,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sA = smem + stage * kStageBytes;
           uint8_t* sB = sA + kABytes;
           ptx::mbar_arrive_expect_tx(&full[stage], bytes);
-          const int kc = (ki % a.k_iters) * kBK;
           if (a.mode != kModeRow) {
+            const int kc = ki * kBK;
             ptx::tma_load_2d_nohint(sA, &a.tmA, &full[stage], kc, arow);
             ptx::tma_load_2d_nohint(sB, &a.tmB, &full[stage], kc, h0.brow);
             if (has1) ptx::tma_load_2d_nohint(sB + kBHalfBytes, &a.tmB, &full[stage], kc, h1.brow);
           } else {
-            const int r = a.r0 + ki / a.k_iters;
-            ptx::tma_load_3d_nohint(sA, &a.tmA, &full[stage], kc, mb * kBM, r);
-            ptx::tma_load_3d_nohint(sB, &a.tmB, &full[stage], kc, h0.brow, r);
+            const bool g2 = rr >= a.r_split;  // second contraction width
+            const CUtensorMap* mA = g2 ? &a.tmA2 : &a.tmA;
+            const CUtensorMap* mB = g2 ? &a.tmB2 : &a.tmB;
+            const int rc = g2 ? rr - a.r_split : rr;
+            ptx::tma_load_3d_nohint(sA, mA, &full[stage], kb * kBK, mb * kBM, rc);
+            ptx::tma_load_3d_nohint(sB, mB, &full[stage], kb * kBK, h0.brow, rc);
             if (has1)
-              ptx::tma_load_3d_nohint(sB + kBHalfBytes, &a.tmB, &full[stage], kc, h1.brow, r);
+              ptx::tma_load_3d_nohint(sB + kBHalfBytes, mB, &full[stage], kb * kBK, h1.brow, rc);
+            if (++kb == (g2 ? a.k_iters2 : a.k_iters)) {
+              kb = 0;
+              ++rr;
+            }
           }
           ++issued;
           if (++stage == kStages) {

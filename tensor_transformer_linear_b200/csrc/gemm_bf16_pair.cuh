@@ -62,6 +62,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&a.tmA);
     ptx::prefetch_tmap(&a.tmB);
+    if (a.mode == kModeRow && a.r_split < a.r1) {
+      ptx::prefetch_tmap(&a.tmA2);
+      ptx::prefetch_tmap(&a.tmB2);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(tmem_slot, 2 * kAccCols);
@@ -73,8 +77,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int nr = (a.mode == kModeRow) ? (a.r1 - a.r0) : 1;
-  const int k_total = nr * a.k_iters;
+  const int k_total = k_steps(a);
   const uint32_t full_lead = ptx::mapa_shared(&full[0], 0);      // full[s] at + 8 s
   const uint32_t tempty_lead = ptx::mapa_shared(&tempty[0], 0);  // tempty[a] at + 8 a
 
@@ -92,6 +95,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const HalfInfo h = decode_half(a, (rank == 1 && has1) ? 2 * nt + 1 : 2 * nt);
         const int m_row = mb * kPairBM + static_cast<int>(rank) * kBM;
         const int arow = a.a_remap ? seq_row(a, m_row) : m_row;
+        int rr = a.r0, kb = 0;  // row mode: rank and K block of the next step
         for (int ki = 0; ki < k_total; ++ki) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -101,14 +105,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           uint8_t* sA = smem + stage * kPairStageBytes;
           uint8_t* sB = sA + kABytes;
           const uint32_t bar = full_lead + 8u * stage;
-          const int kc = (ki % a.k_iters) * kBK;
           if (a.mode != kModeRow) {
+            const int kc = ki * kBK;
             ptx::tma_load_2d_pair(sA, &a.tmA, bar, kc, arow);
             ptx::tma_load_2d_pair(sB, &a.tmB, bar, kc, h.brow);
           } else {
-            const int r = a.r0 + ki / a.k_iters;
-            ptx::tma_load_3d_pair(sA, &a.tmA, bar, kc, m_row, r);
-            ptx::tma_load_3d_pair(sB, &a.tmB, bar, kc, h.brow, r);
+            const bool g2 = rr >= a.r_split;  // second contraction width
+            const CUtensorMap* mA = g2 ? &a.tmA2 : &a.tmA;
+            const CUtensorMap* mB = g2 ? &a.tmB2 : &a.tmB;
+            const int rc = g2 ? rr - a.r_split : rr;
+            ptx::tma_load_3d_pair(sA, mA, bar, kb * kBK, m_row, rc);
+            ptx::tma_load_3d_pair(sB, mB, bar, kb * kBK, h.brow, rc);
+            if (++kb == (g2 ? a.k_iters2 : a.k_iters)) {
+              kb = 0;
+              ++rr;
+            }
           }
           if (++stage == kPairStages) {
             stage = 0;

@@ -297,32 +297,48 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   if (!aligned(h, 16) || !aligned(w, 16) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||
       (residual && !aligned(residual, 2)) || (partials && !aligned(partials, 4)))
     return TPL_ERR_ALIGN;
+  // Up to two contiguous groups of equal contraction width: the shape of every
+  // partition from tpl_partition_subparams (remainder units on the lowest ranks).
   const int64_t Kr = k_w[0];
+  int split = tp;
   for (int r = 1; r < tp; ++r)
-    if (k_w[r] != Kr) return TPL_ERR_UNSUPPORTED;  // bf16 path: equal rank widths
+    if (k_w[r] != Kr) {
+      split = r;
+      break;
+    }
+  const int64_t Kr2 = split < tp ? k_w[split] : Kr;
+  for (int r = split; r < tp; ++r)
+    if (k_w[r] != Kr2) return TPL_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
   tpl_status s = device_info(&dev);
   if (s != TPL_OK) return s;
 
   tpl::GemmArgs a;
   std::memset(&a, 0, sizeof(a));
-  {
-    const uint64_t dims[3] = {static_cast<uint64_t>(Kr), static_cast<uint64_t>(M),
-                              static_cast<uint64_t>(tp)};
-    const uint64_t str[2] = {static_cast<uint64_t>(Kr) * 2, static_cast<uint64_t>(M * Kr) * 2};
-    if ((s = encode_bf16(&a.tmA, h, 3, dims, str, tpl::kBM)) != TPL_OK) return s;
-  }
-  {
-    const uint64_t dims[3] = {static_cast<uint64_t>(Kr), static_cast<uint64_t>(N),
-                              static_cast<uint64_t>(tp)};
-    const uint64_t str[2] = {static_cast<uint64_t>(Kr) * 2, static_cast<uint64_t>(N * Kr) * 2};
-    if ((s = encode_bf16(&a.tmB, w, 3, dims, str, tpl::kHalfN)) != TPL_OK) return s;
-  }
+  auto encode_group = [&](CUtensorMap* mh, CUtensorMap* mw, int64_t kr, int64_t ranks,
+                          int64_t first) -> tpl_status {
+    const char* hb = static_cast<const char*>(h) + M * first * Kr * 2;
+    const char* wb = static_cast<const char*>(w) + N * first * Kr * 2;
+    const uint64_t dh[3] = {static_cast<uint64_t>(kr), static_cast<uint64_t>(M),
+                            static_cast<uint64_t>(ranks)};
+    const uint64_t sh[2] = {static_cast<uint64_t>(kr) * 2, static_cast<uint64_t>(M * kr) * 2};
+    tpl_status st2 = encode_bf16(mh, hb, 3, dh, sh, tpl::kBM);
+    if (st2 != TPL_OK) return st2;
+    const uint64_t dw[3] = {static_cast<uint64_t>(kr), static_cast<uint64_t>(N),
+                            static_cast<uint64_t>(ranks)};
+    const uint64_t sw[2] = {static_cast<uint64_t>(kr) * 2, static_cast<uint64_t>(N * kr) * 2};
+    return encode_bf16(mw, wb, 3, dw, sw, tpl::kHalfN);
+  };
+  if ((s = encode_group(&a.tmA, &a.tmB, Kr, split, 0)) != TPL_OK) return s;
+  if (split < tp && (s = encode_group(&a.tmA2, &a.tmB2, Kr2, tp - split, split)) != TPL_OK)
+    return s;
   a.mode = tpl::kModeRow;
   a.M = static_cast<int32_t>(M);
   set_seqpar(a, sp);
   a.N = static_cast<int32_t>(N);
   a.k_iters = static_cast<int32_t>((Kr + tpl::kBK - 1) / tpl::kBK);
+  a.k_iters2 = static_cast<int32_t>((Kr2 + tpl::kBK - 1) / tpl::kBK);
+  a.r_split = split;
   a.n_halves = static_cast<int32_t>((N + tpl::kHalfN - 1) / tpl::kHalfN);
   a.n_tiles = (a.n_halves + 1) / 2;
   a.y = static_cast<__nv_bfloat16*>(y);

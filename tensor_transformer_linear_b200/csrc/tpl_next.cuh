@@ -160,3 +160,39 @@ tpl_status tpl_embedding_lookup(const int32_t* ids, int64_t n, const void* table
 }
 
 }  // extern "C"
+
+// ======================================================================
+// Self-test of the bounded pipeline waits
+// ======================================================================
+
+namespace tpl {
+
+// One thread waits, with the same bounded wait every pipeline of this library
+// uses, on an mbarrier that nothing ever arrives on; when the limit runs out
+// it records TPL_ERR_TIMEOUT in the status word and returns normally.
+__global__ void selftest_wait_timeout_kernel(uint64_t limit_ns, int* waited) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = ptx::globaltimer();
+    if (!ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns)) record_timeout();
+    if (waited != nullptr) *waited = static_cast<int>((ptx::globaltimer() - t0) / 1000);
+  }
+}
+
+}  // namespace tpl
+
+extern "C" tpl_status tpl_selftest_wait_timeout(uint64_t limit_ns, int32_t* waited_us,
+                                                void* stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return TPL_ERR_SHAPE;
+  if (waited_us != nullptr && !aligned(waited_us, 4)) return TPL_ERR_ALIGN;
+  tpl::selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      limit_ns, waited_us);
+  return launched();
+}

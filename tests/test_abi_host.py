@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 14, names
+    assert len(names) == 15, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -199,3 +199,10 @@ def test_next_rows_rejections():
     assert L.tpl_embedding_lookup(None, 0, None, 10, 8, 2, 1, None, s) == 0
     assert L.tpl_embedding_lookup(FAKE, 4, FAKE, 10, 8, 65, 1, FAKE, s) == 2
     assert L.tpl_embedding_lookup(FAKE, 4, FAKE_ODD, 10, 8, 2, 1, FAKE, s) == 5
+
+
+def test_selftest_rejections():
+    L = T.lib()
+    assert L.tpl_selftest_wait_timeout(0, None, None) == 2
+    assert L.tpl_selftest_wait_timeout(2_000_000_000, None, None) == 2
+    assert L.tpl_selftest_wait_timeout(1000, FAKE_ODD, None) == 5

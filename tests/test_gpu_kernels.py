@@ -219,12 +219,47 @@ def test_row_linear_fp32_uneven_ranks():
         assert O.rel_frobenius(pg[r], pr) <= TOL_FP32
 
 
-def test_row_linear_bf16_uneven_ranks_rejected():
-    h = torch.zeros(4 * 24, dtype=torch.bfloat16, device=DEV)
-    w = torch.zeros(8 * 24, dtype=torch.bfloat16, device=DEV)
+@pytest.mark.parametrize("k_w,M,N", [([16, 16, 8], 200, 136), ([72, 64, 64, 64], 300, 256),
+                                     ([336, 336, 328], 1, 40)])
+def test_row_linear_bf16_two_rank_widths(k_w, M, N):
+    # remainder units on the lowest ranks: two contiguous groups of equal width
+    h = _t((M, sum(k_w)), 1.0, 5)
+    w2 = _t((N, sum(k_w)), 0.05, 2)
+    tp = len(k_w)
+    parts = torch.empty(tp * M * N, dtype=torch.float32, device=DEV)
+    y = T.tpl_row_linear_reduce(T.pack_row_weight(h, k_w).to(DEV), k_w, M,
+                                T.pack_row_weight(w2, k_w).to(DEV), partials=parts)
+    torch.cuda.synchronize()
+    hs, ws = O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w)
+    assert rel(y, O.row_linear_reduce(hs, ws)) <= TOL_BF16
+    pg = f64(parts).reshape(tp, M, N)
+    for r, pr in enumerate(O.row_partials(hs, ws)):
+        assert O.rel_frobenius(pg[r], pr) <= 1e-5
+
+
+def test_row_linear_bf16_three_rank_widths_rejected():
+    h = torch.zeros(4 * 40, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(8 * 40, dtype=torch.bfloat16, device=DEV)
     with pytest.raises(T.TplError) as e:
-        T.tpl_row_linear_reduce(h, [16, 8], 4, w)
+        T.tpl_row_linear_reduce(h, [16, 8, 16], 4, w)
     assert e.value.name == "TPL_ERR_UNSUPPORTED"
+
+
+def test_tp_mlp_uneven_partition_end_to_end():
+    # intermediate 1000 over tp 3 in units of 8: widths 336, 336, 328
+    M, H, I, tp = 257, 256, 1000, 3
+    x = _t((M, H), 1.0, 0)
+    w1, w2 = _t((I, H), 0.05, 1), _t((H, I), 0.05, 2)
+    p = T.tpl_partition_subparams([I], tp, 8)
+    k_w = [p.shard_width[r] for r in range(tp)]
+    hbuf = T.tpl_column_linear(p, x.to(DEV), w1.to(DEV), None, "gelu_erf")
+    y = T.tpl_row_linear_reduce(hbuf, k_w, M, T.pack_row_weight(w2, k_w).to(DEV))
+    torch.cuda.synchronize()
+    part = O.partition_subparams([I], tp, 8)
+    ref = O.row_linear_reduce(O.column_linear(f64(x), f64(w1), None, part, "gelu_erf"),
+                              O.row_weight_slices(f64(w2), part.shard_width))
+    assert part.shard_width == [336, 336, 328]
+    assert rel(y, ref) <= TOL_BF16
 
 
 # ---------------------------------------------------------------- LM head
