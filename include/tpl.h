@@ -292,6 +292,16 @@ tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t K, const v
                                     int32_t* shard_idx, int32_t* ids, void* stream);
 
 /*
+ * Self-test of the failure path.  (No counterpart on the pages: a diagnostic
+ * of this library.)  Launches one thread that waits, with the bounded wait the
+ * pipelines use, on an mbarrier nothing arrives on; after limit_ns (1 ns .. 1 s)
+ * it records TPL_ERR_TIMEOUT in the status word and returns, leaving the
+ * context usable.  waited_us (device int32, or NULL) receives the time waited.
+ * tpl_get_device_status then reports and clears TPL_ERR_TIMEOUT.
+ */
+tpl_status tpl_selftest_wait_timeout(uint64_t limit_ns, int32_t* waited_us, void* stream);
+
+/*
  * Synchronises `stream`, then returns TPL_ERR_TIMEOUT if any kernel of this
  * library on the current device recorded a pipeline timeout since the last
  * call (and clears it), TPL_ERR_CUDA if the stream reports an error, else
