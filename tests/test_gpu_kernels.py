@@ -271,6 +271,9 @@ LM_CASES = [
     (17, 200, 37, 4, 2, True),          # shards of 10 ids: several shards inside one slab
     (1, 8, 9, 8, 1, False),             # empty shards
     (48, 128, 2000, 3, 5, True),        # B > 32, uneven
+    (128, 256, 5000, 4, 2, True),       # one full 128-row batch tile
+    (129, 128, 3000, 2, 3, True),       # two batch tiles, the second with one row
+    (256, 192, 40000, 8, 4, True),      # two full batch tiles of 160 columns: one TMEM buffer
 ]
 
 
