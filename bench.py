@@ -129,6 +129,70 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+
+# ------------------------------------------------------------------ end to end
+
+E2E_SETS = 3
+
+
+class E2EPipeline:
+    """Steps end to end through pinned host buffers, as a serving loop runs them.
+
+    Step k uploads its inputs from pinned host memory on an upload stream,
+    computes on the launching stream and downloads its results into pinned host
+    memory on a download stream, using device buffer set k % E2E_SETS.  Step
+    k+1's upload and step k-1's download therefore overlap step k's compute;
+    events order the reuse of each set (its upload waits for the download
+    E2E_SETS steps back).  Every step's copies are inside the timed region.
+    """
+
+    def __init__(self, wl, stream):
+        self.wl, self.stream = wl, stream
+        names = list(dict.fromkeys(wl.io_in + wl.io_out))
+        base = {a: getattr(wl, a) for a in names}
+        self.sets = [base] + [{a: torch.empty_like(t) for a, t in base.items()}
+                              for _ in range(E2E_SETS - 1)]
+        src = wl.host_inputs() if hasattr(wl, "host_inputs") else base
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+        self.h_in = {a: pin(src[a]) for a in wl.io_in}
+        self.h_out = [{a: torch.empty(base[a].shape, dtype=base[a].dtype, pin_memory=True)
+                       for a in wl.io_out} for _ in range(E2E_SETS)]
+        self.bytes_in = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        self.bytes_out = sum(t.numel() * t.element_size() for t in self.h_out[0].values())
+        self.up, self.down = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: [torch.cuda.Event() for _ in range(E2E_SETS)]
+        self.ev_up, self.ev_cmp, self.ev_down = ev(), ev(), ev()
+        self.k = 0
+
+    def step(self):
+        wl, b = self.wl, self.k % E2E_SETS
+        bufs = self.sets[b]
+        if self.k >= E2E_SETS:
+            self.up.wait_event(self.ev_down[b])
+        with torch.cuda.stream(self.up):
+            for a, h in self.h_in.items():
+                bufs[a].copy_(h, non_blocking=True)
+        self.ev_up[b].record(self.up)
+        self.stream.wait_event(self.ev_up[b])
+        if self.k >= E2E_SETS:
+            self.stream.wait_event(self.ev_down[b])
+        for a, t in bufs.items():
+            setattr(wl, a, t)
+        wl.step(self.stream)
+        self.ev_cmp[b].record(self.stream)
+        self.down.wait_event(self.ev_cmp[b])
+        with torch.cuda.stream(self.down):
+            for a, h in self.h_out[b].items():
+                h.copy_(bufs[a], non_blocking=True)
+        self.ev_down[b].record(self.down)
+        self.k += 1
+
+    def close(self):
+        torch.cuda.synchronize()
+        for a, t in self.sets[0].items():
+            setattr(self.wl, a, t)
+
+
 # ------------------------------------------------------------------ workloads
 
 class Block:
@@ -145,7 +209,9 @@ class Block:
         self.flops = 0.0
         self.gemm_flops = 0.0
         self.launches = []        # (part name, callable(stream)), in launch order
-        self.d_in, self.d_out = [], []
+        # Attributes holding each step's inputs and results; every launch reads
+        # them at call time, so the end-to-end pipeline can rotate buffer sets.
+        self.io_in, self.io_out = [], []
         if "qkv" in parts:
             # inputs and weights, generated on the device by the seeded generator
             self.qx = C.qkv_x(q, dev)
@@ -157,8 +223,8 @@ class Block:
                 self.qpart, self.qx, self.qw, self.qb, "none", y=self.qy, stream=s)))
             self.flops += q.flops()
             self.gemm_flops += q.flops()
-            self.d_in.append(self.qx)
-            self.d_out.append(self.qy)
+            self.io_in.append("qx")
+            self.io_out.append("qy")
         if "mlp" in parts:
             self.mx = C.mlp_x(m, dev)
             self.mlp = T.TPMLP(C.mlp_w1(m, 0, dev), C.mlp_w2(m, 0, dev), m.tp, m.act,
@@ -176,8 +242,8 @@ class Block:
                     self.h, mlp.k_w, m.M, mlp.w2, None, None, y=self.my, stream=s))]
             self.flops += m.flops()
             self.gemm_flops += m.flops()
-            self.d_in.append(self.mx)
-            self.d_out.append(self.my)
+            self.io_in.append("mx")
+            self.io_out.append("my")
         if "lmhead" in parts:
             self.lx = C.lm_x(l, dev)
             self.lw = C.lm_w(l, dev)
@@ -189,8 +255,8 @@ class Block:
                 self.lx, self.lw, l.tp, l.n_chunks, self.ws, ids=self.ids, shard_max=self.smax,
                 shard_idx=self.sidx, stream=s)))
             self.flops += l.flops()
-            self.d_in.append(self.lx)
-            self.d_out += [self.ids, self.smax, self.sidx]
+            self.io_in.append("lx")
+            self.io_out += ["ids", "smax", "sidx"]
         self.parts = [n for n, _ in self.launches]
 
     def step(self, stream, events=None):
@@ -204,22 +270,6 @@ class Block:
     def gemm_part_ids(self):
         return [i for i, n in enumerate(self.parts) if n in ("qkv_column", "mlp_column_gelu",
                                                               "mlp_row_reduce")]
-
-    # --- end to end through host buffers
-    def host_io(self):
-        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
-        self.h_in = [pin(t.cpu()) for t in self.d_in]
-        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in self.d_out]
-        b_in = sum(t.numel() * t.element_size() for t in self.h_in)
-        b_out = sum(t.numel() * t.element_size() for t in self.h_out)
-        return b_in, b_out
-
-    def step_e2e(self, stream):
-        for h, d in zip(self.h_in, self.d_in):
-            d.copy_(h, non_blocking=True)
-        self.step(stream)
-        for h, d in zip(self.h_out, self.d_out):
-            h.copy_(d, non_blocking=True)
 
     def lmhead_bytes(self):
         return self.l.algorithmic_bytes() if "lmhead" in self.sel else None
@@ -273,6 +323,7 @@ class Stack:
         self.w = w
         self.x0 = C.mlp_x(w, dev)
         self.x = self.x0.clone()
+        self.io_in, self.io_out = ["x"], ["x"]   # the residual stream is updated in place
         self.layers = [T.TPMLP(C.mlp_w1(w, l, dev), C.mlp_w2(w, l, dev), w.tp, w.act,
                                norm=True, residual=True) for l in range(w.layers)]
         self.flops = w.flops()
@@ -303,16 +354,8 @@ class Stack:
         if events is not None:
             events[i].record(stream)
 
-    def host_io(self):
-        self.h_in = torch.empty(self.x.shape, dtype=self.x.dtype, pin_memory=True).copy_(self.x0.cpu())
-        self.h_out = torch.empty(self.x.shape, dtype=self.x.dtype, pin_memory=True)
-        n = self.x.numel() * self.x.element_size()
-        return n, n
-
-    def step_e2e(self, stream):
-        self.x.copy_(self.h_in, non_blocking=True)
-        self.step(stream)
-        self.h_out.copy_(self.x, non_blocking=True)
+    def host_inputs(self):
+        return {"x": self.x0}
 
     def lmhead_bytes(self):
         return None
@@ -368,7 +411,7 @@ class NextRows:
             self.launches.append(("swiglu_column", lambda s: T.tpl_swiglu_column_linear(
                 self.x, self.w, self.F, m.tp, h=self.h, stream=s)))
             self.flops = self.gemm_flops = 2.0 * m.M * m.hidden * 2 * self.F
-            self.d_in, self.d_out = [self.x], [self.h]
+            self.io_in, self.io_out = ["x"], ["h"]
         elif kind == "embed":
             self.name = (f"vocab-sharded-embedding ids[8,1024] W[{l.vocab},{l.hidden}] bf16 "
                          f"tp{l.tp}")
@@ -381,7 +424,7 @@ class NextRows:
             self.launches.append(("embed_lookup", lambda s: T.tpl_embedding_lookup(
                 self.ids, self.table, l.tp, out=self.out, stream=s)))
             self.hbm_bytes = m.M * l.hidden * 2 * 2 + m.M * 4
-            self.d_in, self.d_out = [self.ids], [self.out]
+            self.io_in, self.io_out = ["ids"], ["out"]
         elif kind == "seqpar":
             b, sq = m.batch, m.seq
             self.name = (f"sequence-parallel rmsnorm-tp-mlp x[{b},{sq},{m.hidden}] bf16 "
@@ -403,7 +446,7 @@ class NextRows:
                 ("sp_row_scatter", lambda s: T.tpl_row_linear_reduce_scatter(
                     self.hbuf, self.k_w, b, sq, self.w2, None, self.x, y=self.y, stream=s))]
             self.flops = self.gemm_flops = m.flops()
-            self.d_in, self.d_out = [self.x], [self.y]
+            self.io_in, self.io_out = ["x"], ["y"]
         else:
             raise ValueError(kind)
         self.parts = [n for n, _ in self.launches]
@@ -430,20 +473,6 @@ class NextRows:
             return [("roofline_rmsnorm", "rmsnorm_cta", "sp_rmsnorm",
                      2 * 2 * self.m.M * self.m.hidden)]
         return []
-
-    def host_io(self):
-        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
-        self.h_in = [pin(t.cpu()) for t in self.d_in]
-        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in self.d_out]
-        return (sum(t.numel() * t.element_size() for t in self.h_in),
-                sum(t.numel() * t.element_size() for t in self.h_out))
-
-    def step_e2e(self, stream):
-        for h, d in zip(self.h_in, self.d_in):
-            d.copy_(h, non_blocking=True)
-        self.step(stream)
-        for h, d in zip(self.h_out, self.d_out):
-            h.copy_(d, non_blocking=True)
 
     def oracle_sample(self, rows=64):
         import numpy as np
@@ -633,24 +662,24 @@ def main():
         if pg is not None:
             decode_ms = max_over_ranks([decode_ms], dev)[0]
 
-    # ---- end to end through host buffers (pinned), copies inside the timed region
-    b_in, b_out = wl.host_io()
-    for _ in range(3):
-        with torch.cuda.stream(stream):
-            wl.step_e2e(stream)
+    # ---- end to end through pinned host buffers, copies inside the timed region
+    e2e = E2EPipeline(wl, stream)
+    b_in, b_out = e2e.bytes_in, e2e.bytes_out
+    for _ in range(E2E_SETS + 1):
+        e2e.step()
     torch.cuda.synchronize()
     e_steps = max(10, args.steps // 5)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if pg is not None:
         pg.barrier()
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e_steps):
-            wl.step_e2e(stream)
-        e1.record(stream)
+    e0.record(e2e.up)
+    for _ in range(e_steps):
+        e2e.step()
+    e1.record(e2e.down)
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
+    e2e.close()
 
     if pg is not None:
         ms, e_ms = max_over_ranks([ms, e_ms], dev)
@@ -691,7 +720,11 @@ def main():
             "gpu_launches": int(launches),
             "clocks": clk,
             "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_out)},
+                    "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_out),
+                    "steps": e_steps,
+                    "method": f"pinned host buffers; upload, compute and download on three "
+                              f"streams over {E2E_SETS} device buffer sets, so step k+1's "
+                              "upload and step k-1's download overlap step k's compute"},
         }
         lb = wl.lmhead_bytes()
         if lb is not None:
