@@ -24,6 +24,7 @@ and the step time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -83,7 +84,7 @@ def ncu_traffic(kernel: str, workload: str, sources):
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -103,7 +104,9 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
+        """Median SM clock and the throttle reasons seen; with a host-time window
+        [t0, t1] (datetime.now() values) only the samples taken inside it count."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -115,9 +118,18 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) >= 9:
-                rows.append(f)
+            if len(f) >= 10:
+                try:
+                    ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                except ValueError:
+                    continue
+                rows.append((ts, f[1:]))
         os.unlink(self.path)
+        if t0 is not None and t1 is not None:
+            inside = [r for ts, r in rows if t0 <= ts <= t1]
+            rows = inside if inside else [r for _, r in rows]
+        else:
+            rows = [r for _, r in rows]
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -128,6 +140,16 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
 
+
+def clocks_rejected(clk) -> bool:
+    """A hardware or thermal slowdown, or SM clocks held far below max with no
+    reason given (a leftover clock lock), invalidates a timing."""
+    if not clk:
+        return False
+    if set(clk["reasons"]) & {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}:
+        return True
+    sm, mx = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    return bool(sm and mx and not clk["reasons"] and sm < 0.6 * mx)
 
 
 # ------------------------------------------------------------------ end to end
@@ -602,7 +624,6 @@ def main():
     dev = torch.device("cuda", local)
     pg = None
     if world > 1:
-        import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
@@ -622,29 +643,45 @@ def main():
         raise RuntimeError("a kernel reported a pipeline timeout during warm-up")
 
     # ---- device-timed region: K steps, per-launch events on the launching stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(torch.cuda.current_device())
+    def timed_region():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+               for _ in range(args.steps)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(torch.cuda.current_device())
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        time.sleep(0.3)   # nvidia-smi is sampling before the timed steps start
+        n0 = T.tpl_launch_count()
+        t0 = datetime.datetime.now()
+        start.record(stream)
+        for k in range(args.steps):
+            wl.step(stream, evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        t1 = datetime.datetime.now()
+        launches = T.tpl_launch_count() - n0
+        clk = clocks.stop(t0, t1)
+        if pg is not None:
+            pg.barrier()
+        if T.tpl_get_device_status(stream) != 0:
+            raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
+        part_ms = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1])
+                                   for k in range(args.steps)) for i in range(n_ev - 1)]
+        return start.elapsed_time(stop), part_ms, launches, clk
+
+    ms, part_ms, launches, clk = timed_region()
+    # A run under a hardware or thermal slowdown (or a stale clock lock) is taken
+    # again once; every rank makes the same decision.
+    bad = torch.tensor([1.0 if clocks_rejected(clk) else 0.0], device=dev)
     if pg is not None:
-        pg.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    n0 = T.tpl_launch_count()
-    start.record(stream)
-    for k in range(args.steps):
-        wl.step(stream, evs[k])
-    stop.record(stream)
-    torch.cuda.synchronize()
-    launches = T.tpl_launch_count() - n0
-    clk = clocks.stop()
-    if pg is not None:
-        pg.barrier()
-    ms = start.elapsed_time(stop)
-    if T.tpl_get_device_status(stream) != 0:
-        raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
-    part_ms = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
-               for i in range(n_ev - 1)]
+        dist.all_reduce(bad, op=dist.ReduceOp.MAX)
+    remeasured = bool(bad.item() > 0)
+    if remeasured:
+        ms, part_ms, launches, clk = timed_region()
+    if clk is not None:
+        clk["remeasured"] = remeasured
 
     # ---- the LM head in a decode loop: back-to-back launches, as once per decode step
     decode_ms = None

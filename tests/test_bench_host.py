@@ -1,0 +1,63 @@
+"""Host logic of bench.py that needs no GPU: the clock sampler's parsing and
+time window, and the rule that rejects a timing taken under throttling."""
+import datetime
+import os
+import sys
+import tempfile
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+class _Proc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        pass
+
+
+def _sampler_with(rows, now):
+    """A ClockSampler whose nvidia-smi output is the given (sm_mhz, power_cap) rows,
+    one per second from `now`."""
+    c = bench.ClockSampler(0)
+    fd, c.path = tempfile.mkstemp(suffix=".csv")
+    os.close(fd)
+    with open(c.path, "w") as f:
+        for i, (mhz, cap, hw) in enumerate(rows):
+            ts = (now + datetime.timedelta(seconds=i)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+            f.write(f"{ts}, 0, {mhz}, 1965, 900.00, 0x4, {hw}, Not Active, Not Active, {cap}\n")
+    c.proc = _Proc()
+    c.out = open(os.devnull, "w")
+    return c
+
+
+def test_clock_samples_outside_the_timed_window_are_dropped():
+    now = datetime.datetime.now()
+    rows = [(1965, "Not Active", "Not Active"), (1400, "Active", "Not Active"),
+            (1300, "Active", "Not Active"), (1965, "Not Active", "Not Active")]
+    c = _sampler_with(rows, now)
+    clk = c.stop(now + datetime.timedelta(seconds=0.5), now + datetime.timedelta(seconds=2.5))
+    assert clk == {"sm_mhz": 1350.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 2}
+
+
+def test_clock_window_with_no_samples_keeps_them_all():
+    now = datetime.datetime.now()
+    c = _sampler_with([(1800, "Not Active", "Not Active"), (1700, "Not Active", "Active")], now)
+    far = now + datetime.timedelta(hours=1)
+    clk = c.stop(far, far + datetime.timedelta(seconds=1))
+    assert clk["samples"] == 2 and clk["reasons"] == ["hw_slowdown"]
+
+
+def test_throttled_or_locked_clocks_are_rejected():
+    assert not bench.clocks_rejected(None)
+    assert not bench.clocks_rejected({"reasons": ["sw_power_cap"], "sm_mhz": 1300,
+                                      "sm_max_mhz": 1965})
+    for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clocks_rejected({"reasons": [r], "sm_mhz": 1900, "sm_max_mhz": 1965})
+    # far below max with no reason: a clock lock left by someone else
+    assert bench.clocks_rejected({"reasons": [], "sm_mhz": 900, "sm_max_mhz": 1965})
+    assert not bench.clocks_rejected({"reasons": [], "sm_mhz": 1900, "sm_max_mhz": 1965})
