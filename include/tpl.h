@@ -149,7 +149,11 @@ tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, i
  *             reduction; slower: one extra pass per rank).
  *   M == 0 is a no-op (h, w, y may then be NULL).
  *
- * bf16 needs every k_w[r] % 8 == 0 and 16-byte aligned h and w.
+ * bf16 needs every k_w[r] % 8 == 0 and 16-byte aligned h and w.  The bf16
+ * kernel takes at most two contraction widths, each held by a contiguous run
+ * of ranks (k_w = {a, .., a, b, .., b}, the shape tpl_partition_subparams
+ * gives an uneven split); other patterns return TPL_ERR_UNSUPPORTED.  fp32
+ * takes any widths.
  */
 tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
                                  int64_t N, const void* w, const void* bias,
