@@ -295,6 +295,69 @@ tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t K, const v
                                     int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
                                     int32_t* shard_idx, int32_t* ids, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The TP linears split over GPUs: one process per GPU, rank `rank` of `tp`.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * This rank's shard of a row-parallel linear whose reduction is a
+ * reduce-scatter over the token dimension (google-research: each shard's
+ * "{YZ unreduced}" partial, reduced afterwards; nanotron "MLP Module": the
+ * c_proj output is [batch, seq // tp, hidden] per rank).  The partial
+ *   P = H_rank W_rank^T   (bf16 in, fp32 accumulate, stored bf16)
+ * is written by the GEMM epilogue straight into the receive buffer of the rank
+ * that owns each token, so the exchange overlaps the GEMM tile by tile.
+ *
+ *   h     device bf16 [batch * seq][K], this rank's contraction slice of the
+ *         activations (token b * seq + t in row b * seq + t).
+ *   w     device bf16 [N][K], this rank's columns of the unsharded [N][tp*K]
+ *         weight.
+ *   peer  HOST array of tp device pointers: peer[q] is rank q's receive buffer,
+ *         bf16 [tp][batch][seq / tp][N] (slot s holds rank s's partial of the
+ *         tokens q * seq/tp .. (q+1) * seq/tp - 1 of every sequence).  For
+ *         q != rank it must be a mapping of that GPU's buffer into this process
+ *         (CUDA IPC or equivalent); the kernel writes it with plain stores.
+ *         Token t of sequence b goes to peer[t / (seq/tp)], slot `rank`, row
+ *         b * seq/tp + t % (seq/tp).
+ * Requirements: seq % tp == 0 (else TPL_ERR_INDIVISIBLE), K % 8 == 0, h and w
+ * 16-byte aligned (else TPL_ERR_ALIGN), batch * seq <= INT32_MAX.
+ * Completion: the writes are complete when this call's work on `stream` is;
+ * a rank may read its receive buffer only after every rank's scatter has
+ * completed (a stream-ordered collective, e.g. an all-reduce of one element,
+ * after the scatter on every rank).
+ */
+tpl_status tpl_row_linear_scatter(const void* h, int64_t K, int64_t batch, int64_t seq, int64_t N,
+                                  const void* w, int32_t rank, int32_t tp, void* const* peer,
+                                  void* stream);
+
+/*
+ * The reduction step of the reduce-scatter above, on the rank that owns a
+ * token slice:  y[i][n] = bf16( sum_{s < tp} recv[s][i][n] + bias[n]
+ * + residual[i][n] ), summed in fp32 in rank order (the order of the one-GPU
+ * tpl_row_linear_reduce).
+ *   recv      device bf16 [tp][rows][N] (the receive buffer, rows = batch*seq/tp).
+ *   bias      device bf16 [N] or NULL.   residual  device bf16 [rows][N] or NULL.
+ *   y         device bf16 [rows][N]; may alias residual.
+ * rows == 0 is a no-op.
+ */
+tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t N,
+                            const void* bias, const void* residual, void* y, void* stream);
+
+/*
+ * Global argmax of a vocab split over tp GPUs (Tenstorrent LMHead1D: every
+ * device's candidates combined at the end).  Rank s ran tpl_lmhead_argmax on
+ * its vocab slice (ids local to the slice); after an all-gather of those
+ * outputs:
+ *   shard_max  device fp32 [tp][B];  shard_idx  device int32 [tp][B], local
+ *              ids, -1 for none.  Rank s's global id = s * id_stride + local
+ *              (id_stride = the slice size, ceil(V / tp)).
+ *   ids        device int32 [B]: the largest logit, ties to the lowest global
+ *              id; -1 if no rank has a candidate.
+ * Requirements: tp * id_stride <= INT32_MAX.
+ */
+tpl_status tpl_argmax_merge(const float* shard_max, const int32_t* shard_idx, int32_t tp,
+                            int64_t B, int64_t id_stride, int32_t* ids, void* stream);
+
 /*
  * Self-test of the failure path.  (No counterpart on the pages: a diagnostic
  * of this library.)  Launches one thread that waits, with the bounded wait the

@@ -32,7 +32,8 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_get_device_status", "tpl_status_string", "tpl_launch_count",
             "tpl_lmhead_argmax_static", "tpl_row_linear_reduce_scatter",
             "tpl_column_linear_allgather", "tpl_swiglu_column_linear", "tpl_embedding_lookup",
-            "tpl_selftest_wait_timeout")
+            "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
+            "tpl_argmax_merge")
 
 
 class TplError(RuntimeError):
@@ -91,6 +92,10 @@ def lib():
         L.tpl_swiglu_column_linear.argtypes = [vp, i64, i64, vp, i64, i32, i32, vp, vp]
         L.tpl_embedding_lookup.argtypes = [vp, i64, vp, i64, i64, i32, i32, vp, vp]
         L.tpl_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp]
+        L.tpl_row_linear_scatter.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32,
+                                             ctypes.POINTER(vp), vp]
+        L.tpl_reduce_slots.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+        L.tpl_argmax_merge.argtypes = [vp, vp, i32, i64, i64, vp, vp]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -369,6 +374,77 @@ def tpl_embedding_lookup(ids: torch.Tensor, table: torch.Tensor, tp: int,
                                       DTYPE[table.dtype], _ptr(out), _stream(stream)),
            "tpl_embedding_lookup")
     return out
+
+
+def tpl_row_linear_scatter(h: torch.Tensor, w: torch.Tensor, batch: int, seq: int, rank: int,
+                           tp: int, peers: Sequence, stream=None) -> None:
+    """This rank's row-parallel shard, written into every owner rank's receive buffer.
+
+    ``peers[q]`` is rank q's receive buffer ``[tp][batch][seq // tp][N]`` bf16:
+    a CUDA tensor, or the integer device address of a buffer mapped from
+    another GPU (see include/tpl.h).
+    """
+    _cuda(h, "h", torch.bfloat16)
+    _cuda(w, "w", torch.bfloat16)
+    M, K = int(batch) * int(seq), h.shape[-1]
+    if h.numel() != M * K or w.numel() % K != 0:
+        raise ValueError("h must be [batch * seq, K] and w [N, K]")
+    N = w.numel() // K
+    if len(peers) != tp:
+        raise ValueError("peers must hold one receive buffer per rank")
+    addr = []
+    for q, p in enumerate(peers):
+        if isinstance(p, torch.Tensor):
+            _cuda(p, f"peers[{q}]", torch.bfloat16)
+            if p.numel() < M * N:
+                raise ValueError(f"peers[{q}] is smaller than [tp][batch][seq // tp][N]")
+            addr.append(p.data_ptr())
+        else:
+            addr.append(int(p))
+    arr = (ctypes.c_void_p * tp)(*addr)
+    _check(lib().tpl_row_linear_scatter(_ptr(h), int(K), int(batch), int(seq), int(N), _ptr(w),
+                                        int(rank), int(tp), arr, _stream(stream)),
+           "tpl_row_linear_scatter")
+
+
+def tpl_reduce_slots(recv: torch.Tensor, tp: int, N: int, bias: Optional[torch.Tensor] = None,
+                     residual: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """``y = sum of the tp slots of recv (+ bias) (+ residual)``: this rank's token slice."""
+    _cuda(recv, "recv", torch.bfloat16)
+    if recv.numel() % (tp * N) != 0:
+        raise ValueError("recv must be [tp][rows][N]")
+    rows = recv.numel() // (tp * N)
+    if y is None:
+        y = torch.empty((rows, N), dtype=torch.bfloat16, device=recv.device)
+    _cuda(y, "y", torch.bfloat16)
+    if bias is not None:
+        _cuda(bias, "bias", torch.bfloat16)
+    if residual is not None:
+        _cuda(residual, "residual", torch.bfloat16)
+        if residual.numel() != rows * N:
+            raise ValueError("residual must be [rows][N]")
+    if y.numel() != rows * N:
+        raise ValueError("y must be [rows][N]")
+    _check(lib().tpl_reduce_slots(_ptr(recv), int(tp), int(rows), int(N), _ptr(bias),
+                                  _ptr(residual), _ptr(y), _stream(stream)), "tpl_reduce_slots")
+    return y
+
+
+def tpl_argmax_merge(shard_max: torch.Tensor, shard_idx: torch.Tensor, id_stride: int,
+                     ids: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Global argmax over ranks from the gathered ``[tp][B]`` per-rank LM-head outputs."""
+    _cuda(shard_max, "shard_max", torch.float32)
+    _cuda(shard_idx, "shard_idx", torch.int32)
+    tp, B = shard_max.shape
+    if shard_idx.shape != shard_max.shape:
+        raise ValueError("shard_idx must match shard_max")
+    if ids is None:
+        ids = torch.empty(B, dtype=torch.int32, device=shard_max.device)
+    _cuda(ids, "ids", torch.int32)
+    _check(lib().tpl_argmax_merge(_ptr(shard_max), _ptr(shard_idx), int(tp), int(B),
+                                  int(id_stride), _ptr(ids), _stream(stream)), "tpl_argmax_merge")
+    return ids
 
 
 def tpl_selftest_wait_timeout(limit_ns: int, waited_us: Optional[torch.Tensor] = None,

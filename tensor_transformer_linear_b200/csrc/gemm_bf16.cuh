@@ -61,6 +61,8 @@ struct ColPiece {
   int32_t pad_;
 };
 
+constexpr int kMaxPeers = 64;  // TPL_MAX_TP
+
 struct GemmArgs {
   CUtensorMap tmA;  // column: X {K, M};      row: H  {Kr, M, tp} of ranks 0 .. r_split-1
   CUtensorMap tmB;  // column: W {K, rows};   row: W2 {Kr, N, tp} of ranks 0 .. r_split-1
@@ -90,6 +92,12 @@ struct GemmArgs {
   // Row mode with two contraction widths: ranks below r_split use tmA/tmB and
   // k_iters K blocks, the others tmA2/tmB2 and k_iters2 (r_split = tp if equal).
   int32_t r_split, k_iters2;
+  // Peer scatter (row mode, one rank's shard of a row-parallel linear split
+  // over GPUs): token m = b * sp_seq + t belongs to rank t / sp_seg and lands
+  // in slot src_rank of that rank's receive buffer [tp][sp_batch][sp_seg][N],
+  // at peer[t / sp_seg] (another GPU's memory for every rank but this one).
+  int32_t scatter, src_rank;
+  __nv_bfloat16* peer[kMaxPeers];
 };
 
 // Number of 64-wide K steps of one tile.
@@ -112,6 +120,22 @@ __device__ __forceinline__ int seq_row(const GemmArgs& a, int m) {
 // Physical output row of logical row m (rank-major when the output is scattered).
 __device__ __forceinline__ int out_row(const GemmArgs& a, int m) {
   return a.out_remap ? seq_row(a, m) : m;
+}
+
+// Output base and row of logical row m: this launch's y, or in peer-scatter
+// mode the receive buffer of the rank that owns the token (see GemmArgs).
+__device__ __forceinline__ __nv_bfloat16* out_base(const GemmArgs& a, int m, int& prow) {
+  if (!a.scatter) {
+    prow = out_row(a, m);
+    return a.y;
+  }
+  const unsigned seq = static_cast<unsigned>(a.sp_seq), seg = static_cast<unsigned>(a.sp_seg);
+  const unsigned b = static_cast<unsigned>(m) / seq;
+  const unsigned t = static_cast<unsigned>(m) - b * seq;
+  const unsigned q = t / seg;
+  prow = static_cast<int>((static_cast<unsigned>(a.src_rank) * static_cast<unsigned>(a.sp_batch) +
+                           b) * seg + (t - q * seg));
+  return a.peer[q];
 }
 
 struct HalfInfo {
@@ -191,8 +215,8 @@ __device__ __forceinline__ void load_bias_chunk(const GemmArgs& a, const HalfInf
 
 // Epilogue of 32 accumulator columns of one row; bv holds the chunk's bias.
 __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h, int m, int prow,
-                                            int col0, const uint32_t (&r)[32],
-                                            const float (&bv)[32]) {
+                                            __nv_bfloat16* ybase, int col0,
+                                            const uint32_t (&r)[32], const float (&bv)[32]) {
   const int nvalid = min(32, h.valid - col0);
   float v[32];
 #pragma unroll
@@ -238,7 +262,7 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h
         if (j < nvalid) v[j] += bf16_to_f(res[j]);
     }
   }
-  __nv_bfloat16* dst = a.y + off;
+  __nv_bfloat16* dst = ybase + off;
   if (nvalid == 32 && a.vec_store) {
 #pragma unroll
     for (int j = 0; j < 32; j += 8) {
@@ -510,7 +534,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tmem_base + ((q * 32u) << 16) + acc * kAccCols);
       } else if (active) {
         const int m = mb * kBM + row;
-        const int prow = out_row(a, m);
+        int prow;
+        __nv_bfloat16* const yb = out_base(a, m, prow);
         for (int c = 0; c < kHalfN / 32; ++c) {
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
@@ -519,7 +544,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float bv[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) bv[j] = bias_s[c * 32 + j];
-            store_chunk(a, h, m, prow, c * 32, r, bv);
+            store_chunk(a, h, m, prow, yb, c * 32, r, bv);
           }
         }
       }

@@ -213,14 +213,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         tmem_base + ((q * 32u) << 16) + acc * kAccCols);
       } else if (active) {
         const int m = mb * kPairBM + static_cast<int>(rank) * kBM + row;
-        const int prow = out_row(a, m);
+        int prow;
+        __nv_bfloat16* const yb = out_base(a, m, prow);
         for (int c = 0; c < kHalfN / 32; ++c) {
           float bv[32];
           if (a.bias != nullptr && c * 32 < h.valid) load_bias_chunk(a, h, c * 32, bv);
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
           ptx::tmem_ld_wait();
-          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, prow, c * 32, r, bv);
+          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, prow, yb, c * 32, r, bv);
         }
       }
       ptx::tc_fence_before();

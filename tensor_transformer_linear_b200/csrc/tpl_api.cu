@@ -167,6 +167,14 @@ struct SeqPar {
   int32_t a_remap = 0, out_remap = 0;
 };
 
+// One rank's shard of a row-parallel linear split over GPUs: its output rows go
+// to the receive buffers of the ranks that own the tokens (peer[q], [tp] bases).
+struct PeerScatter {
+  int32_t src_rank = 0;
+  int32_t tp = 0;
+  void* const* peer = nullptr;
+};
+
 template <typename Args>
 void set_seqpar(Args& a, const SeqPar& sp) {
   a.sp_batch = sp.batch;
@@ -291,7 +299,8 @@ tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t
 
 tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_t N, const void* w,
                     const void* bias, const void* residual, void* y, float* partials,
-                    cudaStream_t st, const SeqPar& sp = SeqPar{}) {
+                    cudaStream_t st, const SeqPar& sp = SeqPar{},
+                    const PeerScatter* ps = nullptr) {
   for (int r = 0; r < tp; ++r)
     if (k_w[r] % 8 != 0) return TPL_ERR_ALIGN;
   if (!aligned(h, 16) || !aligned(w, 16) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||
@@ -350,6 +359,16 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   a.residual = static_cast<const __nv_bfloat16*>(residual);
   a.partials = nullptr;
   a.vec_store = (N % 8 == 0 && aligned(y, 16) && (residual == nullptr || aligned(residual, 16)));
+  if (ps != nullptr) {
+    a.scatter = 1;
+    a.src_rank = ps->src_rank;
+    bool vec = (N % 8 == 0);
+    for (int q = 0; q < ps->tp; ++q) {
+      a.peer[q] = static_cast<__nv_bfloat16*>(ps->peer[q]);
+      vec = vec && aligned(ps->peer[q], 16);
+    }
+    a.vec_store = vec ? 1 : 0;
+  }
   if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
 
   if (partials != nullptr) {
@@ -752,3 +771,5 @@ extern "C" tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t
 
 // Entry points of the next rows (same translation unit).
 #include "tpl_next.cuh"
+// The TP linears split over GPUs (same translation unit).
+#include "tpl_ranks.cuh"

@@ -1,0 +1,168 @@
+// tpl_ranks.cuh -- the TP linears split over GPUs, one process per GPU (the
+// google-research row-parallel "{YZ unreduced}" partial and its reduction;
+// nanotron "MLP Module": [batch, seq // tp, hidden] per rank after c_proj;
+// Tenstorrent LMHead1D: every device's argmax candidates combined at the end).
+//
+//   tpl_row_linear_scatter  this rank's shard of the row-parallel linear.  The
+//       GEMM epilogue writes each output row straight into the receive buffer
+//       of the rank that owns the token (a peer pointer for every other rank),
+//       so the exchange of partials overlaps the GEMM tile by tile.
+//   tpl_reduce_slots        once every rank's scatter has completed, a rank sums
+//       its tp slots (in rank order, fp32) plus bias and residual: its token
+//       slice of the reduced output (the reduce-scatter).
+//   tpl_argmax_merge        the per-rank LM-head candidates, gathered, reduced to
+//       the global argmax (ties to the lowest global id).
+//
+// Included at the end of tpl_api.cu (one translation unit with its helpers).
+#pragma once
+
+#include "common.cuh"
+
+namespace tpl {
+
+constexpr int kReduceThreads = 256;
+
+// y[i] = bf16(sum_{s < tp} recv[s][i] + bias[i % N] + residual[i]) over the
+// rows * N elements of one rank's slice; kVec: 8 elements per thread (N % 8 == 0,
+// 16-byte aligned buffers).
+template <bool kVec>
+__global__ void __launch_bounds__(kReduceThreads)
+    reduce_slots_kernel(const __nv_bfloat16* __restrict__ recv, int tp, int64_t total, int N,
+                        const __nv_bfloat16* __restrict__ bias,
+                        const __nv_bfloat16* __restrict__ residual, __nv_bfloat16* y) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x * (kVec ? 8 : 1);
+  for (int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * (kVec ? 8 : 1);
+       i < total; i += stride) {
+    if (kVec) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < tp; ++s) {
+        const uint4 q = __ldcs(reinterpret_cast<const uint4*>(recv + s * total + i));
+        acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
+        acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
+        acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
+        acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
+      }
+      if (bias != nullptr) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(bias + i % N));
+        acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
+        acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
+        acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
+        acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
+      }
+      if (residual != nullptr) {
+        const uint4 q = *reinterpret_cast<const uint4*>(residual + i);
+        acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
+        acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
+        acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
+        acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(y + i) = o;
+    } else {
+      float acc = 0.f;
+      for (int s = 0; s < tp; ++s) acc += bf16_to_f(recv[s * total + i]);
+      if (bias != nullptr) acc += bf16_to_f(bias[i % N]);
+      if (residual != nullptr) acc += bf16_to_f(residual[i]);
+      y[i] = __float2bfloat16_rn(acc);
+    }
+  }
+}
+
+// ids[b] = the global id of the best candidate over ranks: rank s's candidate
+// for row b is (shard_max[s][b], s * id_stride + shard_idx[s][b]); a negative
+// shard_idx is "no candidate".  Larger logit wins, then the lower global id.
+__global__ void argmax_merge_kernel(const float* shard_max, const int32_t* shard_idx, int tp,
+                                    int B, int64_t id_stride, int32_t* ids) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  float best = 0.f;
+  int64_t best_id = -1;
+  for (int s = 0; s < tp; ++s) {
+    const int32_t local = shard_idx[static_cast<int64_t>(s) * B + b];
+    if (local < 0) continue;
+    const float v = shard_max[static_cast<int64_t>(s) * B + b];
+    const int64_t gid = s * id_stride + local;
+    if (best_id < 0 || v > best || (v == best && gid < best_id)) {
+      best = v;
+      best_id = gid;
+    }
+  }
+  ids[b] = static_cast<int32_t>(best_id);
+}
+
+}  // namespace tpl
+
+extern "C" {
+
+tpl_status tpl_row_linear_scatter(const void* h, int64_t K, int64_t batch, int64_t seq, int64_t N,
+                                  const void* w, int32_t rank, int32_t tp, void* const* peer,
+                                  void* stream) {
+  if (peer == nullptr) return TPL_ERR_NULL;
+  SeqPar sp;
+  tpl_status s = seqpar_of(batch, seq, tp, &sp);
+  if (s != TPL_OK) return s;
+  if (rank < 0 || rank >= tp || K < 1 || K > INT32_MAX || N < 1 || N > INT32_MAX)
+    return TPL_ERR_SHAPE;
+  if (h == nullptr || w == nullptr) return TPL_ERR_NULL;
+  for (int q = 0; q < tp; ++q) {
+    if (peer[q] == nullptr) return TPL_ERR_NULL;
+    if (!aligned(peer[q], 2)) return TPL_ERR_ALIGN;
+  }
+  PeerScatter ps;
+  ps.src_rank = rank;
+  ps.tp = tp;
+  ps.peer = peer;
+  const int64_t kw[1] = {K};
+  return row_bf16(h, kw, 1, batch * seq, N, w, nullptr, nullptr, nullptr, nullptr,
+                  static_cast<cudaStream_t>(stream), sp, &ps);
+}
+
+tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t N,
+                            const void* bias, const void* residual, void* y, void* stream) {
+  if (tp < 1 || tp > TPL_MAX_TP || rows < 0 || N < 1 || N > INT32_MAX) return TPL_ERR_SHAPE;
+  if (rows == 0) return TPL_OK;
+  if (recv == nullptr || y == nullptr) return TPL_ERR_NULL;
+  if (!aligned(recv, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||
+      (residual && !aligned(residual, 2)))
+    return TPL_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  tpl_status s = device_info(&dev);
+  if (s != TPL_OK) return s;
+  const int64_t total = rows * N;
+  const bool vec = (N % 8 == 0) && aligned(recv, 16) && aligned(y, 16) &&
+                   (bias == nullptr || aligned(bias, 16)) &&
+                   (residual == nullptr || aligned(residual, 16));
+  const int64_t per_block = static_cast<int64_t>(tpl::kReduceThreads) * (vec ? 8 : 1);
+  const int grid = static_cast<int>(std::min<int64_t>((total + per_block - 1) / per_block,
+                                                      static_cast<int64_t>(dev->sm_count) * 8));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* rv = static_cast<const __nv_bfloat16*>(recv);
+  const auto* bv = static_cast<const __nv_bfloat16*>(bias);
+  const auto* res = static_cast<const __nv_bfloat16*>(residual);
+  auto* yv = static_cast<__nv_bfloat16*>(y);
+  const int Ni = static_cast<int>(N);
+  if (vec)
+    tpl::reduce_slots_kernel<true><<<grid, tpl::kReduceThreads, 0, st>>>(rv, tp, total, Ni, bv, res, yv);
+  else
+    tpl::reduce_slots_kernel<false><<<grid, tpl::kReduceThreads, 0, st>>>(rv, tp, total, Ni, bv, res, yv);
+  return launched();
+}
+
+tpl_status tpl_argmax_merge(const float* shard_max, const int32_t* shard_idx, int32_t tp,
+                            int64_t B, int64_t id_stride, int32_t* ids, void* stream) {
+  if (tp < 1 || tp > TPL_MAX_TP || B < 1 || B > INT32_MAX || id_stride < 1 ||
+      id_stride * tp > INT32_MAX)
+    return TPL_ERR_SHAPE;
+  if (shard_max == nullptr || shard_idx == nullptr || ids == nullptr) return TPL_ERR_NULL;
+  if (!aligned(shard_max, 4) || !aligned(shard_idx, 4) || !aligned(ids, 4)) return TPL_ERR_ALIGN;
+  const int Bi = static_cast<int>(B);
+  tpl::argmax_merge_kernel<<<(Bi + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      shard_max, shard_idx, tp, Bi, id_stride, ids);
+  return launched();
+}
+
+}  // extern "C"

@@ -8,12 +8,13 @@ residual section.  Each step is one call into libtpl.so.
 """
 from __future__ import annotations
 
-from typing import List, Optional, Sequence
+from typing import Callable, List, Optional, Sequence
 
 import torch
 
-from ._tpl import (Partition, tpl_column_linear, tpl_partition_subparams, tpl_rmsnorm,
-                   tpl_row_linear_reduce)
+from ._tpl import (Partition, tpl_argmax_merge, tpl_column_linear, tpl_lmhead_argmax,
+                   tpl_lmhead_workspace_size, tpl_partition_subparams, tpl_reduce_slots,
+                   tpl_rmsnorm, tpl_row_linear_reduce, tpl_row_linear_scatter)
 
 
 def shard_views(y: torch.Tensor, p: Partition, M: int) -> List[torch.Tensor]:
@@ -88,3 +89,177 @@ class TPStack:
         for layer in self.layers:
             layer(x, out=x, stream=stream)
         return x
+
+
+# ---------------------------------------------------------------------------
+# The TP linears split over GPUs: one process per GPU, rank `rank` of `tp`.
+# ---------------------------------------------------------------------------
+
+def sp_rows(batch: int, seq: int, tp: int) -> int:
+    """Token rows a rank owns after the reduce-scatter: ``batch * seq / tp``
+    (nanotron "MLP Module": ``[batch, seq // tp, hidden]`` per rank)."""
+    if seq % tp != 0:
+        raise ValueError(f"seq {seq} is not divisible by tp {tp}")
+    return batch * (seq // tp)
+
+
+def sp_token_owner(t: int, seq: int, tp: int) -> int:
+    """The rank that owns token ``t`` of every sequence."""
+    return t // (seq // tp)
+
+
+def sp_slice(x: torch.Tensor, batch: int, seq: int, tp: int, rank: int) -> torch.Tensor:
+    """Rank ``rank``'s token slice ``[batch, seq/tp, N]`` of a ``[batch*seq, N]``
+    tensor, contiguous (e.g. its share of the residual stream)."""
+    n = x.shape[-1]
+    return x.reshape(batch, tp, seq // tp, n)[:, rank].contiguous()
+
+
+def recv_buffer_numel(tp: int, batch: int, seq: int, N: int) -> int:
+    """Elements of one rank's receive buffer ``[tp][batch][seq/tp][N]``: one slot
+    per source rank, each that source's partial of this rank's tokens."""
+    return tp * sp_rows(batch, seq, tp) * N
+
+
+class PeerBuffers:
+    """This rank's receive buffer and the device address of every rank's receive
+    buffer as mapped into this process (``addrs[rank]`` is the local one)."""
+
+    def __init__(self, local: torch.Tensor, addrs: Sequence[int], keep: Sequence = ()):
+        self.local = local
+        self.addrs = [int(a) for a in addrs]
+        self._keep = list(keep)  # mapped peer storages stay open while in use
+
+
+def local_peer_buffers(bufs: Sequence[torch.Tensor], rank: int) -> PeerBuffers:
+    """Every rank's buffer lives in this process (ranks run one after another)."""
+    return PeerBuffers(bufs[rank], [b.data_ptr() for b in bufs])
+
+
+def exchange_peer_buffers(local: torch.Tensor, group=None) -> PeerBuffers:
+    """Maps every rank's receive buffer into this process.
+
+    One process per GPU on one node with peer access between the GPUs: each rank
+    exports its buffer's storage as a CUDA IPC handle, the handles are
+    all-gathered over the process group, and each peer storage is opened here.
+    Plain peer mappings only: nothing is bound to a multicast object.
+    """
+    import torch.distributed as dist
+    st = local.untyped_storage()
+    handle = st._share_cuda_()
+    offset = local.data_ptr() - st.data_ptr()
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    got = [None] * world
+    dist.all_gather_object(got, (handle, offset), group=group)
+    addrs, keep = [], []
+    for q, (h, off) in enumerate(got):
+        if q == rank:
+            addrs.append(local.data_ptr())
+            continue
+        peer = torch.UntypedStorage._new_shared_cuda(*h)
+        keep.append(peer)
+        addrs.append(peer.data_ptr() + off)
+    return PeerBuffers(local, addrs, keep)
+
+
+def stream_barrier(group=None, device=None) -> Callable:
+    """A barrier ordered on a stream: an all-reduce of one element over the
+    group, enqueued on the stream.  Work after it on that stream starts only when
+    every rank's work before its own barrier has completed, which is what makes
+    the peer writes of every rank's scatter visible to the readers."""
+    import torch.distributed as dist
+    token = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def barrier(stream=None):
+        if stream is None:
+            dist.all_reduce(token, group=group)
+        else:
+            with torch.cuda.stream(stream):
+                dist.all_reduce(token, group=group)
+    return barrier
+
+
+class TPRowParallelRank:
+    """Rank ``rank``'s row-parallel linear over ``tp`` GPUs, reduced by a
+    reduce-scatter along the sequence (google-research: each shard's partial,
+    reduced afterwards; nanotron "MLP Module": ``[batch, seq // tp, hidden]``).
+
+    Each call: scatter (this rank's partial, written by the GEMM epilogue into
+    every owner's receive buffer) -> barrier -> reduce this rank's slots (+ bias,
+    + residual) -> barrier.  The first barrier makes every partial visible before
+    any rank reads its slots; the second keeps the next call's scatter from
+    overwriting slots a slower rank is still reading.
+
+    ``w_shard`` is ``[N, k]``, this rank's columns of the unsharded weight.
+    ``scatter`` and ``reduce`` default to the library's calls.
+    """
+
+    def __init__(self, w_shard: torch.Tensor, rank: int, tp: int, peers: PeerBuffers,
+                 barrier: Callable, scatter: Optional[Callable] = None,
+                 reduce: Optional[Callable] = None):
+        self.w = w_shard.contiguous()
+        self.rank, self.tp, self.peers, self.barrier = rank, tp, peers, barrier
+        self.scatter = scatter or tpl_row_linear_scatter
+        self.reduce = reduce or tpl_reduce_slots
+
+    def __call__(self, h_shard: torch.Tensor, batch: int, seq: int,
+                 bias: Optional[torch.Tensor] = None, residual: Optional[torch.Tensor] = None,
+                 y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """``h_shard`` ``[batch*seq, k]``; ``residual`` this rank's token slice
+        ``[batch*seq/tp, N]`` (see :func:`sp_slice`).  Returns that slice of Y."""
+        N = self.w.shape[0]
+        sp_rows(batch, seq, self.tp)
+        self.scatter(h_shard, self.w, batch, seq, self.rank, self.tp, self.peers.addrs,
+                     stream=stream)
+        self.barrier(stream)
+        out = self.reduce(self.peers.local, self.tp, N, bias, residual, y, stream=stream)
+        self.barrier(stream)
+        return out
+
+
+class TPLMHeadRank:
+    """Rank ``rank``'s share of the decode LM head over ``tp`` GPUs (Tenstorrent
+    LMHead1D: every device computes its vocab slice; the candidates are combined
+    at the end): the argmax candidates of its slice, all-gathered (8 bytes per
+    row per rank), merged into global ids.
+
+    ``w_slice`` is rows ``rank * shard .. (rank+1) * shard`` of W, with
+    ``shard = ceil(V / tp)``.  ``local_argmax``, ``gather`` and ``merge``
+    default to the library's calls and the process group's all-gather.
+    """
+
+    def __init__(self, w_slice: torch.Tensor, rank: int, tp: int, shard: int, group=None,
+                 local_argmax: Optional[Callable] = None, gather: Optional[Callable] = None,
+                 merge: Optional[Callable] = None):
+        self.w = w_slice.contiguous()
+        self.rank, self.tp, self.shard, self.group = rank, tp, shard, group
+        self.local_argmax = local_argmax or self._local_argmax
+        self.gather = gather or self._gather
+        self.merge = merge or (lambda m, i, stride, stream=None:
+                               tpl_argmax_merge(m, i, stride, stream=stream))
+        self._ws = None
+
+    def _local_argmax(self, x, stream=None):
+        B = x.shape[0]
+        need = tpl_lmhead_workspace_size(B, self.w.shape[0], 1, 1)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
+        _, m, i = tpl_lmhead_argmax(x, self.w, 1, 1, self._ws, stream=stream)
+        return m[0], i[0]
+
+    def _gather(self, t: torch.Tensor, stream=None) -> torch.Tensor:
+        """``[tp, ...]``: every rank's ``t``, in rank order."""
+        import torch.distributed as dist
+        parts = [torch.empty_like(t) for _ in range(self.tp)]
+        if stream is None:
+            dist.all_gather(parts, t, group=self.group)
+            return torch.stack(parts)
+        with torch.cuda.stream(stream):
+            dist.all_gather(parts, t, group=self.group)
+            return torch.stack(parts)
+
+    def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        """``x`` ``[B, K]`` (the same on every rank).  Returns global ids ``[B]``."""
+        m, i = self.local_argmax(x, stream=stream)
+        return self.merge(self.gather(m, stream=stream), self.gather(i, stream=stream),
+                          self.shard, stream=stream)

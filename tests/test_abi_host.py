@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 15, names
+    assert len(names) == 18, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -199,6 +199,29 @@ def test_next_rows_rejections():
     assert L.tpl_embedding_lookup(None, 0, None, 10, 8, 2, 1, None, s) == 0
     assert L.tpl_embedding_lookup(FAKE, 4, FAKE, 10, 8, 65, 1, FAKE, s) == 2
     assert L.tpl_embedding_lookup(FAKE, 4, FAKE_ODD, 10, 8, 2, 1, FAKE, s) == 5
+
+
+def test_multi_gpu_rows_rejections():
+    L = T.lib()
+    s = ctypes.c_void_p(0)
+    peers = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert L.tpl_row_linear_scatter(FAKE, 64, 2, 8, 16, FAKE, 0, 2, None, s) == 1
+    assert L.tpl_row_linear_scatter(FAKE, 64, 2, 7, 16, FAKE, 0, 2, peers, s) == 3   # seq % tp
+    assert L.tpl_row_linear_scatter(FAKE, 64, 2, 8, 16, FAKE, 2, 2, peers, s) == 2   # rank
+    assert L.tpl_row_linear_scatter(FAKE, 60, 2, 8, 16, FAKE, 0, 2, peers, s) == 5   # K % 8
+    assert L.tpl_row_linear_scatter(None, 64, 2, 8, 16, FAKE, 0, 2, peers, s) == 1
+    assert L.tpl_row_linear_scatter(FAKE, 64, 2, 8, 16, FAKE, 0, 2,
+                                    (ctypes.c_void_p * 2)(FAKE, None), s) == 1
+    assert L.tpl_row_linear_scatter(FAKE, 64, 2, 8, 16, FAKE, 0, 2,
+                                    (ctypes.c_void_p * 2)(FAKE, FAKE_ODD), s) == 5
+    assert L.tpl_reduce_slots(FAKE, 0, 4, 8, None, None, FAKE, s) == 2
+    assert L.tpl_reduce_slots(None, 2, 0, 8, None, None, None, s) == 0
+    assert L.tpl_reduce_slots(None, 2, 4, 8, None, None, FAKE, s) == 1
+    assert L.tpl_reduce_slots(FAKE, 2, 4, 8, None, None, FAKE_ODD, s) == 5
+    assert L.tpl_argmax_merge(FAKE, FAKE, 2, 0, 10, FAKE, s) == 2
+    assert L.tpl_argmax_merge(FAKE, FAKE, 8, 4, 2**29, FAKE, s) == 2
+    assert L.tpl_argmax_merge(None, FAKE, 2, 4, 10, FAKE, s) == 1
+    assert L.tpl_argmax_merge(FAKE, FAKE, 2, 4, 10, FAKE_ODD, s) == 5
 
 
 def test_selftest_rejections():

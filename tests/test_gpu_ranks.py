@@ -1,0 +1,123 @@
+"""GPU parity of the TP linears split over GPUs, with the ranks run one after
+another on one GPU: every rank's scatter writes into the receive buffers of all
+ranks (here local tensors standing in for its peers'; no kernel waits on
+another), then every rank reduces its slots.  Checked against the fp64 oracle:
+the reduce-scatter result, every slot's partial, and the argmax merged over
+ranks."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import tensor_transformer_linear_b200 as T
+from workloads import gen
+
+from ._parity import TOL_BF16, check_ids, f64, rel
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _t(shape, sigma, tid, seed=5):
+    return gen.normal(shape, sigma, tensor_id=tid, seed=seed)
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    yield
+    assert T.tpl_get_device_status() == 0
+
+
+@pytest.mark.parametrize("tp,batch,seq,inter,N,with_bias,with_res", [
+    (4, 2, 256, 512, 256, True, True),       # M = 512: CTA-pair kernel
+    (2, 1, 64, 128, 130, False, True),       # M = 64: single-CTA kernel; N % 8 != 0
+    (8, 1, 1024, 1792, 512, False, False),   # tp 8, the MLP's contraction split
+    (3, 2, 96, 200, 64, True, False),        # uneven contraction split 72/64/64
+])
+def test_scatter_then_reduce_is_the_reduce_scatter(tp, batch, seq, inter, N, with_bias,
+                                                   with_res):
+    part = O.partition_subparams([inter], tp, 8)
+    k_w = part.shard_width
+    M, seg = batch * seq, seq // tp
+    H = _t((M, inter), 1.0, 0)
+    W2 = _t((N, inter), 0.02, 2)
+    bias = _t((N,), 0.02, 3) if with_bias else None
+    res = _t((M, N), 1.0, 4) if with_res else None
+
+    recv = [torch.full((tp * batch * seg * N,), float("nan"), dtype=torch.bfloat16, device=DEV)
+            for _ in range(tp)]
+    koff = 0
+    for r in range(tp):
+        hr = H[:, koff:koff + k_w[r]].contiguous().to(DEV)
+        wr = W2[:, koff:koff + k_w[r]].contiguous().to(DEV)
+        T.tpl_row_linear_scatter(hr, wr, batch, seq, r, tp, recv)
+        koff += k_w[r]
+    torch.cuda.synchronize()
+
+    bias_d = bias.to(DEV) if bias is not None else None
+    ys = []
+    for q in range(tp):
+        rq = None
+        if res is not None:   # rank q's token slice of the residual stream
+            rq = res.view(batch, tp, seg, N)[:, q].contiguous().to(DEV)
+        ys.append(T.tpl_reduce_slots(recv[q], tp, N, bias_d, rq))
+    torch.cuda.synchronize()
+    got = np.stack([f64(y).reshape(batch, seg, N) for y in ys])
+
+    h_parts, off = [], 0
+    for k in k_w:
+        h_parts.append(f64(H)[:, off:off + k])
+        off += k
+    w_parts = O.row_weight_slices(f64(W2), k_w)
+    res_sp = O.seq_scatter(f64(res), batch, seq, tp) if res is not None else None
+    ref = O.row_linear_reduce_scatter(h_parts, w_parts, batch, seq,
+                                      bias=None if bias is None else f64(bias),
+                                      residual_sp=res_sp)
+    assert rel(got, ref) <= TOL_BF16
+
+    # Slot s of rank q's buffer is rank s's partial of rank q's tokens.
+    parts = O.row_partials(h_parts, w_parts)
+    for q in range(tp):
+        slots = f64(recv[q]).reshape(tp, batch, seg, N)
+        for s in range(tp):
+            assert rel(slots[s], O.seq_scatter(parts[s], batch, seq, tp)[q]) <= TOL_BF16
+
+
+def test_reduce_slots_in_place_on_the_residual():
+    tp, rows, N = 3, 40, 64
+    recv = _t((tp, rows, N), 1.0, 6).to(DEV)
+    res = _t((rows, N), 1.0, 7)
+    y = res.to(DEV)
+    T.tpl_reduce_slots(recv, tp, N, None, y, y=y)
+    torch.cuda.synchronize()
+    ref = f64(recv).sum(axis=0) + f64(res)
+    assert rel(y, ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("B,K,V,tp", [(32, 256, 4999, 4), (5, 64, 37, 8)])
+def test_lmhead_argmax_merged_over_ranks(B, K, V, tp):
+    x = _t((B, K), 1.0, 0)
+    w = _t((V, K), 0.02, 1).clone()
+    shard = -(-V // tp)
+    if V > 3 * shard:
+        # batch row 0's maximum planted twice, on ranks 1 and 3: an exact tie
+        # across ranks, which the lower global id must win
+        w[shard + 7] = (3.0 * x[0].float() / x[0].float().norm()).to(torch.bfloat16)
+        w[3 * shard + 2] = w[shard + 7]
+    smax = torch.empty((tp, B), dtype=torch.float32, device=DEV)
+    sidx = torch.empty((tp, B), dtype=torch.int32, device=DEV)
+    for s in range(tp):
+        lo, hi = s * shard, min(V, (s + 1) * shard)
+        if lo >= hi:                       # a rank whose vocab slice is empty
+            smax[s].fill_(float("-inf"))
+            sidx[s].fill_(-1)
+            continue
+        ws = T.lmhead_workspace(B, hi - lo, 1, 1)
+        _, m, i = T.tpl_lmhead_argmax(x.to(DEV), w[lo:hi].contiguous().to(DEV), 1, 1, ws)
+        smax[s], sidx[s] = m[0], i[0]
+    ids = T.tpl_argmax_merge(smax, sidx, shard)
+    torch.cuda.synchronize()
+    res = O.lmhead_argmax(f64(x), f64(w), tp, 1)
+    check_ids(ids.cpu().numpy(), res)
+    if V > 3 * shard:
+        assert int(ids[0]) == shard + 7
