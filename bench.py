@@ -469,6 +469,39 @@ class NextRows:
                     self.hbuf, self.k_w, b, sq, self.w2, None, self.x, y=self.y, stream=s))]
             self.flops = self.gemm_flops = m.flops()
             self.io_in, self.io_out = ["x"], ["y"]
+        elif kind == "tp_ranks":
+            # The MLP's c_proj as tp rank-local shards, the ranks run one after
+            # another on this GPU: each rank's GEMM scatters its partial into
+            # every rank's receive buffer (local tensors standing in for peer
+            # memory), then every rank sums its slots.
+            tp, b, sq, N, I = m.tp, m.batch, m.seq, m.hidden, m.inter
+            M, kr = m.M, m.inter // m.tp
+            rows = b * (sq // tp)
+            self.name = (f"tp-ranks c_proj x[{b},{sq},{I}] bf16 -> {N}, {tp} ranks in sequence "
+                         f"on one GPU (peer-scatter GEMM + slot reduction)")
+            self.parallelism = (f"{tp} TP ranks emulated in sequence on one GPU: each rank's "
+                                "GEMM writes its partials into every rank's receive buffer, "
+                                "then every rank reduces its slots")
+            self.h = gen.normal((tp * M, kr), 1.0, tensor_id=gen.TID_X, device=dev)
+            self.w2p = T.pack_row_weight(C.mlp_w2(m, 0, dev), [kr] * tp)
+            self.recv = [torch.empty(tp * rows * N, dtype=torch.bfloat16, device=dev)
+                         for _ in range(tp)]
+            self.y = torch.empty(tp * rows * N, dtype=torch.bfloat16, device=dev)
+
+            def scatter_all(s):
+                hs, ws = self.h.view(tp, M, kr), self.w2p.view(tp, N, kr)
+                for r in range(tp):
+                    T.tpl_row_linear_scatter(hs[r], ws[r], b, sq, r, tp, self.recv, stream=s)
+
+            def reduce_all(s):
+                ys = self.y.view(tp, rows, N)
+                for q in range(tp):
+                    T.tpl_reduce_slots(self.recv[q], tp, N, None, None, y=ys[q], stream=s)
+            self.launches += [("rank_scatter_gemms", scatter_all), ("rank_slot_reductions", reduce_all)]
+            self.flops = self.gemm_flops = 2.0 * M * N * I
+            self.gemm_launches = tp            # one scatter GEMM per rank in its part
+            self.reduce_bytes = tp * (tp + 1) * rows * N * 2
+            self.io_in, self.io_out = ["h"], ["y"]
         else:
             raise ValueError(kind)
         self.parts = [n for n, _ in self.launches]
@@ -483,7 +516,8 @@ class NextRows:
 
     def gemm_part_ids(self):
         return [i for i, n in enumerate(self.parts)
-                if n in ("swiglu_column", "sp_column_gelu", "sp_row_scatter")]
+                if n in ("swiglu_column", "sp_column_gelu", "sp_row_scatter",
+                         "rank_scatter_gemms")]
 
     def lmhead_bytes(self):
         return None
@@ -494,6 +528,9 @@ class NextRows:
         if self.kind == "seqpar":
             return [("roofline_rmsnorm", "rmsnorm_cta", "sp_rmsnorm",
                      2 * 2 * self.m.M * self.m.hidden)]
+        if self.kind == "tp_ranks":
+            return [("roofline_reduce", "reduce_slots_kernel", "rank_slot_reductions",
+                     self.reduce_bytes, self.m.tp)]
         return []
 
     def oracle_sample(self, rows=64):
@@ -505,6 +542,13 @@ class NextRows:
             xs, w = f64(self.x[:rows]), f64(self.w)
             return (lambda: O.swiglu_column_linear(xs, w, self.F, m.tp),
                     2.0 * rows * m.hidden * 2 * self.F, f"{rows} token rows")
+        if self.kind == "tp_ranks":
+            rows = 1024
+            tp, kr = m.tp, m.inter // m.tp
+            hs = f64(self.h.view(tp, m.M, kr)[:, :rows])
+            w2 = f64(self.w2p).reshape(tp, m.hidden, kr)
+            return (lambda: O.row_linear_reduce(list(hs), list(w2)),
+                    2.0 * rows * m.hidden * m.inter, f"{rows} token rows of the {tp} ranks")
         if self.kind == "embed":
             sub = 16032
             table = f64(self.table[:sub])
@@ -526,7 +570,8 @@ WORKLOADS = {"block": Block, "stack": Stack,
              "lmhead": lambda dev: Block(dev, ("lmhead",)),
              "swiglu": lambda dev: NextRows(dev, "swiglu"),
              "embed": lambda dev: NextRows(dev, "embed"),
-             "seqpar": lambda dev: NextRows(dev, "seqpar")}
+             "seqpar": lambda dev: NextRows(dev, "seqpar"),
+             "tp_ranks": lambda dev: NextRows(dev, "tp_ranks")}
 
 
 # ------------------------------------------------------------------ timing
@@ -728,7 +773,7 @@ def main():
         e2e_val = replica_rate(world, wl.flops, e_ms / e_steps)
         # dominant kernel: the tcgen05 GEMM (all launches of it in the step)
         gids = wl.gemm_part_ids()
-        n_gemm = len(gids)
+        n_gemm = getattr(wl, "gemm_launches", len(gids)) if gids else 0
         gemm_ms = sum(part_ms[i] for i in gids)
         gemm_launch_flops = wl.gemm_flops / max(1, n_gemm)
         gemm_achieved = wl.gemm_flops / (gemm_ms * 1e-3) / 1e12 if n_gemm else 0.0
@@ -741,8 +786,9 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded SplitMix64 / Irwin-Hall normal, the pages' shapes)",
             "config": {"workload": wl.name,
-                       "parallelism": f"{world} replica(s); tp shards of each linear computed "
-                                      "on one GPU, cross-shard sum in the GEMM epilogue",
+                       "parallelism": f"{world} replica(s); " + getattr(
+                           wl, "parallelism", "tp shards of each linear computed on one GPU, "
+                                              "cross-shard sum in the GEMM epilogue"),
                        "l2": "not flushed: one step streams ~1.5 GB (block) / ~4 GB (stack), "
                              "far above the 126 MB L2"},
             "roofline": {"kernel": "gemm_bf16_tcgen05_pair", "bound": "tensor",
@@ -783,12 +829,14 @@ def main():
                     "frac_of_8000": round(dg / 8000.0, 4), "ms_per_launch": round(decode_ms, 4),
                     "measured": f"{DECODE_LAUNCHES} back-to-back launches (a decode loop), "
                                 "CUDA events on the launching stream"}
-        for key, kern, part, nbytes in wl.hbm_parts():
+        for key, kern, part, nbytes, *n_l in wl.hbm_parts():
             p_ms = part_ms[wl.parts.index(part)]
             gb = nbytes / (p_ms * 1e-3) / 1e9
+            n_l = n_l[0] if n_l else 1
             line[key] = {"kernel": kern, "bound": "hbm", "achieved": round(gb, 1),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gb / pk["hbm_gbs"], 4), "bytes_per_launch": nbytes}
+                         "frac": round(gb / pk["hbm_gbs"], 4), "bytes_per_launch": nbytes // n_l,
+                         "launches_per_step": n_l}
         if not gids:
             first = "roofline_lmhead" if "roofline_lmhead" in line else wl.hbm_parts()[0][0]
             line["roofline"] = line.pop(first)
