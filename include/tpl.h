@@ -2,8 +2,9 @@
  * tpl.h -- C ABI of the tensor-parallel sharded-linear library for B200 (sm_100a).
  *
  * One GPU computes every tensor-parallel (TP) shard of a transformer block's
- * linear layers locally.  The calls follow the shapes of the pages they come
- * from:
+ * linear layers locally; the last group of calls splits the same linears over
+ * GPUs, one process per GPU.  The calls follow the shapes of the pages they
+ * come from:
  *
  *   - nanotron rules, "Tensor-Parallel Component Patterns" (sections
  *     "Attention Module" and "MLP Module"): TP linears take the full logical
@@ -298,6 +299,36 @@ tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t K, const v
 /* ------------------------------------------------------------------------
  * The TP linears split over GPUs: one process per GPU, rank `rank` of `tp`.
  * ------------------------------------------------------------------------ */
+
+#define TPL_MAX_GATHER 16
+
+/*
+ * This rank's shard of a column-parallel linear over the all-gathered tokens
+ * (nanotron "MLP Module": the sequence-parallel activations [batch, seq // tp,
+ * hidden] of every rank are gathered ahead of the column-parallel c_fc; DeepSpeed
+ * "Class SubParamLinearLayer" for the shard's pieces).  Computes, for all
+ * batch * seq tokens,  Y = act(X W^T + b)  with this rank's weight rows, where
+ * the GEMM reads each 128-row tile of X straight from the rank that owns those
+ * tokens, so the all-gather overlaps the GEMM tile by tile.
+ *
+ *   p       partition of this rank's weight (tp_size 1 for a plain shard; the
+ *           shard's fused pieces, e.g. q, k, v, as sub-parameters).
+ *   peer_x  HOST array of tp device pointers: peer_x[q] is rank q's token slice,
+ *           bf16 [batch][seq / tp][K] (tokens q * seq/tp .. of every sequence);
+ *           a mapping of that GPU's buffer for q != this rank.  Read with plain
+ *           TMA loads.
+ *   w, bias, act, y  as tpl_column_linear with M = batch * seq (y holds every
+ *           token's row of this rank's shard).
+ * Requirements: tp <= TPL_MAX_GATHER and (seq / tp) % 128 == 0 (else
+ * TPL_ERR_UNSUPPORTED), seq % tp == 0 (else TPL_ERR_INDIVISIBLE), K % 8 == 0
+ * and 16-byte aligned slices and w (else TPL_ERR_ALIGN).  bf16 only.
+ * Completion: every rank's slice must be complete before this call's work on
+ * `stream` starts (a stream-ordered collective after the producers on every
+ * rank), and must not be overwritten until this call's work has completed.
+ */
+tpl_status tpl_column_linear_gather(const tpl_partition* p, void* const* peer_x, int32_t tp,
+                                    int64_t batch, int64_t seq, int64_t K, const void* w,
+                                    const void* bias, tpl_act act, void* y, void* stream);
 
 /*
  * This rank's shard of a row-parallel linear whose reduction is a

@@ -33,7 +33,7 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_lmhead_argmax_static", "tpl_row_linear_reduce_scatter",
             "tpl_column_linear_allgather", "tpl_swiglu_column_linear", "tpl_embedding_lookup",
             "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
-            "tpl_argmax_merge")
+            "tpl_argmax_merge", "tpl_column_linear_gather")
 
 
 class TplError(RuntimeError):
@@ -96,6 +96,8 @@ def lib():
                                              ctypes.POINTER(vp), vp]
         L.tpl_reduce_slots.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
         L.tpl_argmax_merge.argtypes = [vp, vp, i32, i64, i64, vp, vp]
+        L.tpl_column_linear_gather.argtypes = [ctypes.POINTER(Partition), ctypes.POINTER(vp), i32,
+                                               i64, i64, i64, vp, vp, i32, vp, vp]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -374,6 +376,43 @@ def tpl_embedding_lookup(ids: torch.Tensor, table: torch.Tensor, tp: int,
                                       DTYPE[table.dtype], _ptr(out), _stream(stream)),
            "tpl_embedding_lookup")
     return out
+
+
+def _addresses(bufs: Sequence, name: str, dtype=torch.bfloat16):
+    """Device addresses of CUDA tensors, or integers given as addresses (mapped peer buffers)."""
+    out = []
+    for q, b in enumerate(bufs):
+        if isinstance(b, torch.Tensor):
+            _cuda(b, f"{name}[{q}]", dtype)
+            out.append(b.data_ptr())
+        else:
+            out.append(int(b))
+    return (ctypes.c_void_p * len(out))(*out)
+
+
+def tpl_column_linear_gather(p: Partition, peer_x: Sequence, batch: int, seq: int,
+                             w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                             act: str = "none", y: Optional[torch.Tensor] = None,
+                             stream=None) -> torch.Tensor:
+    """This rank's column shard over every rank's token slice ``peer_x[q]``
+    (``[batch, seq // tp, K]`` bf16, a CUDA tensor or a mapped peer address)."""
+    _cuda(w, "w", torch.bfloat16)
+    if bias is not None:
+        _cuda(bias, "bias", torch.bfloat16)
+    tp = len(peer_x)
+    K = w.shape[-1]
+    M = int(batch) * int(seq)
+    for q, b in enumerate(peer_x):
+        if isinstance(b, torch.Tensor) and b.numel() != M // tp * K:
+            raise ValueError(f"peer_x[{q}] must be [batch, seq // tp, K]")
+    if y is None:
+        y = torch.empty(M * p.logical_out, dtype=torch.bfloat16, device=w.device)
+    _cuda(y, "y", torch.bfloat16)
+    _check(lib().tpl_column_linear_gather(ctypes.byref(p), _addresses(peer_x, "peer_x"), int(tp),
+                                          int(batch), int(seq), int(K), _ptr(w), _ptr(bias),
+                                          ACT[act], _ptr(y), _stream(stream)),
+           "tpl_column_linear_gather")
+    return y
 
 
 def tpl_row_linear_scatter(h: torch.Tensor, w: torch.Tensor, batch: int, seq: int, rank: int,

@@ -61,7 +61,8 @@ struct ColPiece {
   int32_t pad_;
 };
 
-constexpr int kMaxPeers = 64;  // TPL_MAX_TP
+constexpr int kMaxPeers = 64;   // TPL_MAX_TP
+constexpr int kMaxGather = 16;  // ranks a column GEMM can read A from (TPL_MAX_GATHER)
 
 struct GemmArgs {
   CUtensorMap tmA;  // column: X {K, M};      row: H  {Kr, M, tp} of ranks 0 .. r_split-1
@@ -98,6 +99,13 @@ struct GemmArgs {
   // at peer[t / sp_seg] (another GPU's memory for every rank but this one).
   int32_t scatter, src_rank;
   __nv_bfloat16* peer[kMaxPeers];
+  // Peer gather (column mode, one rank's column shard of a linear split over
+  // GPUs, fed by every rank's token slice): the A row of token
+  // m = b * sp_seq + t is row b * sp_seg + t % sp_seg of rank t / sp_seg's slice
+  // [sp_batch][sp_seg][K], loaded through tmGather[t / sp_seg] (a map of another
+  // GPU's memory for every rank but this one; plain TMA loads, no multicast).
+  int32_t a_gather;
+  CUtensorMap tmGather[kMaxGather];
 };
 
 // Number of 64-wide K steps of one tile.
@@ -120,6 +128,20 @@ __device__ __forceinline__ int seq_row(const GemmArgs& a, int m) {
 // Physical output row of logical row m (rank-major when the output is scattered).
 __device__ __forceinline__ int out_row(const GemmArgs& a, int m) {
   return a.out_remap ? seq_row(a, m) : m;
+}
+
+// Tensor map and row holding the A row of logical row m (column mode).
+__device__ __forceinline__ const CUtensorMap* a_source(const GemmArgs& a, int m, int& arow) {
+  if (!a.a_gather) {
+    arow = a.a_remap ? seq_row(a, m) : m;
+    return &a.tmA;
+  }
+  const unsigned seq = static_cast<unsigned>(a.sp_seq), seg = static_cast<unsigned>(a.sp_seg);
+  const unsigned b = static_cast<unsigned>(m) / seq;
+  const unsigned t = static_cast<unsigned>(m) - b * seq;
+  const unsigned q = t / seg;
+  arow = static_cast<int>(b * seg + (t - q * seg));
+  return &a.tmGather[q];
 }
 
 // Output base and row of logical row m: this launch's y, or in peer-scatter
@@ -387,7 +409,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const HalfInfo h0 = decode_half(a, 2 * nt);
         const HalfInfo h1 = has1 ? decode_half(a, 2 * nt + 1) : h0;
         const uint32_t bytes = kABytes + (has1 ? 2 : 1) * kBHalfBytes;
-        const int arow = a.a_remap ? seq_row(a, mb * kBM) : mb * kBM;
+        int arow;
+        const CUtensorMap* mAcol = a_source(a, mb * kBM, arow);
         int rr = a.r0, kb = 0;  // row mode: rank and K block of the next step
         for (int ki = 0; ki < k_total; ++ki) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -399,7 +422,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ptx::mbar_arrive_expect_tx(&full[stage], bytes);
           if (a.mode != kModeRow) {
             const int kc = ki * kBK;
-            ptx::tma_load_2d_nohint(sA, &a.tmA, &full[stage], kc, arow);
+            ptx::tma_load_2d_nohint(sA, mAcol, &full[stage], kc, arow);
             ptx::tma_load_2d_nohint(sB, &a.tmB, &full[stage], kc, h0.brow);
             if (has1) ptx::tma_load_2d_nohint(sB + kBHalfBytes, &a.tmB, &full[stage], kc, h1.brow);
           } else {

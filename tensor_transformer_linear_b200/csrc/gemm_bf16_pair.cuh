@@ -94,7 +94,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // This CTA's half of B; an odd last half is padded with the even one.
         const HalfInfo h = decode_half(a, (rank == 1 && has1) ? 2 * nt + 1 : 2 * nt);
         const int m_row = mb * kPairBM + static_cast<int>(rank) * kBM;
-        const int arow = a.a_remap ? seq_row(a, m_row) : m_row;
+        int arow;
+        const CUtensorMap* mAcol = a_source(a, m_row, arow);
         int rr = a.r0, kb = 0;  // row mode: rank and K block of the next step
         for (int ki = 0; ki < k_total; ++ki) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -107,7 +108,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t bar = full_lead + 8u * stage;
           if (a.mode != kModeRow) {
             const int kc = ki * kBK;
-            ptx::tma_load_2d_pair(sA, &a.tmA, bar, kc, arow);
+            ptx::tma_load_2d_pair(sA, mAcol, bar, kc, arow);
             ptx::tma_load_2d_pair(sB, &a.tmB, bar, kc, h.brow);
           } else {
             const bool g2 = rr >= a.r_split;  // second contraction width

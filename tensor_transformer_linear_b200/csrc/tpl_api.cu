@@ -186,22 +186,41 @@ void set_seqpar(Args& a, const SeqPar& sp) {
 
 // ------------------------------------------------------------------ column
 
+// Token slices of the A operand held by several ranks (peer gather): rank q's
+// slice [batch][seq/tp][K] at gather[q], q < tp.
+struct GatherA {
+  int32_t tp = 0;
+  void* const* gather = nullptr;
+};
+
 tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
                        const void* bias, int act, void* y, cudaStream_t st,
-                       const SeqPar& sp = SeqPar{}) {
+                       const SeqPar& sp = SeqPar{}, const GatherA* ga = nullptr) {
   if ((K % 8) != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 2) ||
       (bias != nullptr && !aligned(bias, 2)))
     return TPL_ERR_ALIGN;
+  if (ga != nullptr)
+    for (int q = 0; q < ga->tp; ++q)
+      if (!aligned(ga->gather[q], 16)) return TPL_ERR_ALIGN;
   DeviceInfo* dev = nullptr;
   tpl_status s = device_info(&dev);
   if (s != TPL_OK) return s;
 
   tpl::GemmArgs a;
   std::memset(&a, 0, sizeof(a));
-  {
+  if (ga == nullptr) {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
     if ((s = encode_bf16(&a.tmA, x, 2, dims, str, tpl::kBM)) != TPL_OK) return s;
+  } else {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K),
+                              static_cast<uint64_t>(sp.batch) * static_cast<uint64_t>(sp.seg)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    for (int q = 0; q < ga->tp; ++q)
+      if ((s = encode_bf16(&a.tmGather[q], ga->gather[q], 2, dims, str, tpl::kBM)) != TPL_OK)
+        return s;
+    a.tmA = a.tmGather[0];
+    a.a_gather = 1;
   }
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(p->logical_out)};

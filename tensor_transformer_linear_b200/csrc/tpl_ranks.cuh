@@ -3,6 +3,10 @@
 // nanotron "MLP Module": [batch, seq // tp, hidden] per rank after c_proj;
 // Tenstorrent LMHead1D: every device's argmax candidates combined at the end).
 //
+//   tpl_column_linear_gather  this rank's shard of a column-parallel linear over
+//       the all-gathered tokens: the GEMM's A tiles are TMA-loaded straight
+//       from the rank that owns the tokens (peer memory), so the all-gather
+//       overlaps the GEMM tile by tile.
 //   tpl_row_linear_scatter  this rank's shard of the row-parallel linear.  The
 //       GEMM epilogue writes each output row straight into the receive buffer
 //       of the rank that owns the token (a peer pointer for every other rank),
@@ -97,6 +101,29 @@ __global__ void argmax_merge_kernel(const float* shard_max, const int32_t* shard
 }  // namespace tpl
 
 extern "C" {
+
+tpl_status tpl_column_linear_gather(const tpl_partition* p, void* const* peer_x, int32_t tp,
+                                    int64_t batch, int64_t seq, int64_t K, const void* w,
+                                    const void* bias, tpl_act act, void* y, void* stream) {
+  if (p == nullptr || peer_x == nullptr) return TPL_ERR_NULL;
+  if (!act_ok(act)) return TPL_ERR_DTYPE;
+  tpl_status s = check_partition(p);
+  if (s != TPL_OK) return s;
+  if (tp > TPL_MAX_GATHER) return TPL_ERR_UNSUPPORTED;
+  SeqPar sp;
+  if ((s = seqpar_of(batch, seq, tp, &sp)) != TPL_OK) return s;
+  if (K < 1 || K > INT32_MAX) return TPL_ERR_SHAPE;
+  // A tiles are 128-row TMA boxes that must each come from one rank's slice.
+  if (sp.seg % tpl::kBM != 0) return TPL_ERR_UNSUPPORTED;
+  if (w == nullptr || y == nullptr) return TPL_ERR_NULL;
+  for (int q = 0; q < tp; ++q)
+    if (peer_x[q] == nullptr) return TPL_ERR_NULL;
+  GatherA ga;
+  ga.tp = tp;
+  ga.gather = peer_x;
+  return column_bf16(p, peer_x[0], batch * seq, K, w, bias, act, y,
+                     static_cast<cudaStream_t>(stream), sp, &ga);
+}
 
 tpl_status tpl_row_linear_scatter(const void* h, int64_t K, int64_t batch, int64_t seq, int64_t N,
                                   const void* w, int32_t rank, int32_t tp, void* const* peer,

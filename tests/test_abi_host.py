@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 18, names
+    assert len(names) == 19, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -214,6 +214,17 @@ def test_multi_gpu_rows_rejections():
                                     (ctypes.c_void_p * 2)(FAKE, None), s) == 1
     assert L.tpl_row_linear_scatter(FAKE, 64, 2, 8, 16, FAKE, 0, 2,
                                     (ctypes.c_void_p * 2)(FAKE, FAKE_ODD), s) == 5
+    pr = T.tpl_partition_subparams([256], 1, 1)
+    xs = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    gather = L.tpl_column_linear_gather
+    assert gather(ctypes.byref(pr), None, 2, 2, 256, 64, FAKE, None, 0, FAKE, s) == 1
+    assert gather(ctypes.byref(pr), xs, 2, 2, 255, 64, FAKE, None, 0, FAKE, s) == 3   # seq % tp
+    assert gather(ctypes.byref(pr), xs, 2, 2, 128, 64, FAKE, None, 0, FAKE, s) == 8   # seg % 128
+    assert gather(ctypes.byref(pr), xs, 17, 2, 17 * 128, 64, FAKE, None, 0, FAKE, s) == 8
+    assert gather(ctypes.byref(pr), xs, 2, 2, 256, 60, FAKE, None, 0, FAKE, s) == 5  # K % 8
+    assert gather(ctypes.byref(pr), (ctypes.c_void_p * 2)(FAKE, FAKE_ODD), 2, 2, 256, 64, FAKE,
+                  None, 0, FAKE, s) == 5
+    assert gather(ctypes.byref(pr), xs, 2, 2, 256, 64, FAKE, None, 7, FAKE, s) == 4  # act
     assert L.tpl_reduce_slots(FAKE, 0, 4, 8, None, None, FAKE, s) == 2
     assert L.tpl_reduce_slots(None, 2, 0, 8, None, None, None, s) == 0
     assert L.tpl_reduce_slots(None, 2, 4, 8, None, None, FAKE, s) == 1

@@ -121,3 +121,31 @@ def test_lmhead_argmax_merged_over_ranks(B, K, V, tp):
     check_ids(ids.cpu().numpy(), res)
     if V > 3 * shard:
         assert int(ids[0]) == shard + 7
+
+
+@pytest.mark.parametrize("tp,batch,seq,K,subs,align,with_bias,act", [
+    (4, 2, 512, 256, [1024], 1, True, "gelu_erf"),            # c_fc shard, CTA-pair kernel
+    (2, 1, 256, 128, [512, 256, 256], 128, True, "none"),      # fused QKV pieces per rank
+    (8, 1, 1024, 64, [256], 1, False, "gelu_tanh"),            # tp 8, 128-token slices
+    (1, 1, 128, 64, [256], 1, True, "none"),                   # M = 128: single-CTA kernel
+])
+def test_gather_column_is_the_column_linear_of_the_gathered_tokens(tp, batch, seq, K, subs, align,
+                                                                   with_bias, act):
+    M, seg = batch * seq, seq // tp
+    x = _t((M, K), 1.0, 0)
+    W = _t((sum(subs), K), 0.02, 1)
+    b = _t((sum(subs),), 0.02, 3) if with_bias else None
+    part = O.partition_subparams(subs, tp, align)
+    ref = O.column_linear(f64(x), f64(W), None if b is None else f64(b), part, act)
+    # rank q's token slice: tokens q * seg .. of every sequence
+    slices = [x.view(batch, tp, seg, K)[:, q].contiguous().to(DEV) for q in range(tp)]
+    for r in range(tp):
+        widths = [part.width[r][j] for j in range(len(subs))]
+        rows = [slice(part.src_off[r][j], part.src_off[r][j] + widths[j])
+                for j in range(len(subs))]
+        w_r = torch.cat([W[s] for s in rows]).contiguous().to(DEV)
+        b_r = torch.cat([b[s] for s in rows]).contiguous().to(DEV) if b is not None else None
+        p_r = T.tpl_partition_subparams(widths, 1, 1)
+        y_r = T.tpl_column_linear_gather(p_r, slices, batch, seq, w_r, b_r, act)
+        torch.cuda.synchronize()
+        assert rel(f64(y_r).reshape(M, part.shard_width[r]), ref[r]) <= TOL_BF16
