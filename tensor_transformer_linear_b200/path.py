@@ -12,9 +12,9 @@ from typing import Callable, List, Optional, Sequence
 
 import torch
 
-from ._tpl import (Partition, tpl_argmax_merge, tpl_column_linear, tpl_lmhead_argmax,
-                   tpl_lmhead_workspace_size, tpl_partition_subparams, tpl_reduce_slots,
-                   tpl_rmsnorm, tpl_row_linear_reduce, tpl_row_linear_scatter)
+from ._tpl import (Partition, tpl_argmax_merge, tpl_column_linear, tpl_column_linear_gather,
+                   tpl_lmhead_argmax, tpl_lmhead_workspace_size, tpl_partition_subparams,
+                   tpl_reduce_slots, tpl_rmsnorm, tpl_row_linear_reduce, tpl_row_linear_scatter)
 
 
 def shard_views(y: torch.Tensor, p: Partition, M: int) -> List[torch.Tensor]:
@@ -215,6 +215,64 @@ class TPRowParallelRank:
         out = self.reduce(self.peers.local, self.tp, N, bias, residual, y, stream=stream)
         self.barrier(stream)
         return out
+
+
+class TPRankMLP:
+    """Rank ``rank``'s share of the sequence-parallel TP MLP block over ``tp``
+    GPUs (nanotron "MLP Module": activations ``[batch, seq // tp, hidden]`` per
+    rank, gathered ahead of the column-parallel c_fc and reduce-scattered after
+    the row-parallel c_proj; google-research residual section):
+
+      RMSNorm of its token slice -> barrier -> c_fc + act over all tokens, each
+      token tile read from the rank that owns it -> c_proj, partials scattered
+      to the owner ranks -> barrier -> its slots summed with the residual, in
+      place on its slice -> barrier.
+
+    The first barrier makes every normalised slice visible before any rank
+    reads it; the second every partial before any rank sums; the third keeps
+    the next call from overwriting normalised slices or slots a slower rank
+    still reads.  ``xn`` and ``recv`` are the peer-visible buffers
+    (``[batch*seq/tp, hidden]`` and :func:`recv_buffer_numel` elements).
+    ``w1_shard`` is ``[inter/tp, hidden]``, ``w2_shard`` ``[hidden, inter/tp]``.
+    The ops default to the library's calls.
+    """
+
+    def __init__(self, w1_shard: torch.Tensor, w2_shard: torch.Tensor, rank: int, tp: int,
+                 act: str, xn: PeerBuffers, recv: PeerBuffers, barrier: Callable,
+                 scale: Optional[torch.Tensor] = None, centered: bool = False,
+                 eps: float = 1e-6, ops: Optional[dict] = None):
+        self.w1, self.w2 = w1_shard.contiguous(), w2_shard.contiguous()
+        self.rank, self.tp, self.act = rank, tp, act
+        self.xn, self.recv, self.barrier = xn, recv, barrier
+        self.scale, self.centered, self.eps = scale, centered, eps
+        self.part = tpl_partition_subparams([self.w1.shape[0]], 1, 1)
+        ops = ops or {}
+        self.rmsnorm = ops.get("rmsnorm", tpl_rmsnorm)
+        self.column = ops.get("column", tpl_column_linear_gather)
+        self.scatter = ops.get("scatter", tpl_row_linear_scatter)
+        self.reduce = ops.get("reduce", tpl_reduce_slots)
+        self._h = None
+
+    def __call__(self, x_slice: torch.Tensor, batch: int, seq: int, stream=None) -> torch.Tensor:
+        """``x_slice`` ``[batch*seq/tp, hidden]``: this rank's tokens of the residual
+        stream, updated in place to ``x + MLP(RMSNorm(x))``."""
+        H, tp = self.w2.shape[0], self.tp
+        M = batch * seq
+        sp_rows(batch, seq, tp)
+        if self._h is None or self._h.numel() < M * self.w1.shape[0]:
+            self._h = torch.empty(M * self.w1.shape[0], dtype=x_slice.dtype,
+                                  device=x_slice.device)
+        self.rmsnorm(x_slice, self.scale, self.centered, self.eps, y=self.xn.local,
+                     stream=stream)
+        self.barrier(stream)
+        h = self.column(self.part, self.xn.addrs, batch, seq, self.w1, None, self.act,
+                        y=self._h, stream=stream)
+        self.scatter(h.view(M, -1), self.w2, batch, seq, self.rank, tp, self.recv.addrs,
+                     stream=stream)
+        self.barrier(stream)
+        self.reduce(self.recv.local, tp, H, None, x_slice, x_slice, stream=stream)
+        self.barrier(stream)
+        return x_slice
 
 
 class TPLMHeadRank:

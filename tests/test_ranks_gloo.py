@@ -1,8 +1,8 @@
 """Host logic of the TP linears split over GPUs, run as two real processes with
 gloo on CPU: the rank orchestration of path.py (the row-parallel
 scatter -> barrier -> reduce -> barrier sequence with its token-slice helpers,
-and the LM head's gather of per-rank candidates), its stream barrier and its
-gather.  The per-rank GPU kernels are replaced by CPU stand-ins that do what
+the whole sequence-parallel MLP block of TPRankMLP over two layers, and the LM
+head's gather of per-rank candidates), its stream barrier and its gather.  The per-rank GPU kernels are replaced by CPU stand-ins that do what
 include/tpl.h says they do; the kernels themselves are tested on the GPU in
 test_gpu_ranks.py.  The results are checked against the fp64 oracle."""
 import datetime
@@ -30,6 +30,9 @@ def _free_port():
 def _problem(batch=2, seq=8, inter=24, N=6, V=23, B=3, K=5):
     rng = np.random.default_rng(7)
     return dict(batch=batch, seq=seq, inter=inter, N=N,
+                X=rng.standard_normal((batch * seq, N)),
+                W1=rng.standard_normal((inter, N)) * 0.3,
+                scale=rng.standard_normal(N) * 0.1,
                 H=rng.standard_normal((batch * seq, inter)),
                 W2=rng.standard_normal((N, inter)) * 0.1,
                 bias=rng.standard_normal(N) * 0.1,
@@ -87,6 +90,51 @@ def _row_parallel(rank, P):
     return y.numpy()
 
 
+def _mlp_block(rank, P):
+    from tensor_transformer_linear_b200 import path
+    tp, batch, seq, N, I = WORLD, P["batch"], P["seq"], P["N"], P["inter"]
+    kr = I // tp
+    w1 = torch.from_numpy(P["W1"][rank * kr:(rank + 1) * kr].copy())
+    w2 = torch.from_numpy(P["W2"][:, rank * kr:(rank + 1) * kr].copy())
+    rows = path.sp_rows(batch, seq, tp)
+    xn = torch.full((rows, N), float("nan"), dtype=torch.float64)
+    recv = torch.full((path.recv_buffer_numel(tp, batch, seq, N),), float("nan"),
+                      dtype=torch.float64)
+
+    def rmsnorm(x_, scale_, centered_, eps_, y=None, stream=None):
+        y.copy_(torch.from_numpy(O.rmsnorm(x_.numpy(), scale_.numpy(), centered_, eps_)))
+        return y
+
+    def column(part_, addrs, b_, s_, w_, bias_, act_, y=None, stream=None):
+        # what tpl_column_linear_gather computes from every rank's normalised slice
+        parts = [torch.empty_like(xn) for _ in range(tp)]
+        dist.all_gather(parts, xn)
+        x_full = O.seq_gather(torch.stack(parts).numpy(), b_, s_, tp)
+        return torch.from_numpy(O.activation(x_full @ w_.numpy().T, act_))
+
+    def scatter(h_, w_, b_, s_, r_, tp_, addrs, stream=None):
+        full = h_ @ w_.T
+        parts = [torch.empty_like(full) for _ in range(tp_)]
+        dist.all_gather(parts, full)
+        slots = recv.view(tp_, -1, N)
+        for src in range(tp_):
+            slots[src] = path.sp_slice(parts[src], b_, s_, tp_, rank).reshape(-1, N)
+
+    def reduce(recv_, tp_, N_, bias_, res_, y_, stream=None):
+        y_.copy_(recv_.view(tp_, -1, N_).sum(0) + res_)
+        return y_
+
+    block = path.TPRankMLP(w1, w2, rank, tp, "gelu_erf", path.PeerBuffers(xn, [0] * tp),
+                           path.PeerBuffers(recv, [0] * tp), path.stream_barrier(),
+                           scale=torch.from_numpy(P["scale"]), centered=True,
+                           ops=dict(rmsnorm=rmsnorm, column=column, scatter=scatter,
+                                    reduce=reduce))
+    x = path.sp_slice(torch.from_numpy(P["X"]), batch, seq, tp, rank).reshape(rows, N)
+    for _ in range(2):                       # two layers sharing the weights
+        block(x, batch, seq)
+    return x.numpy()
+
+
 def _lmhead(rank, P):
     from tensor_transformer_linear_b200 import path
     tp, V = WORLD, P["W"].shape[0]
@@ -122,6 +170,7 @@ def _worker(rank, port, P, out):
                             timeout=datetime.timedelta(seconds=60))
     try:
         out[(rank, "row")] = _row_parallel(rank, P)
+        out[(rank, "mlp")] = _mlp_block(rank, P)
         out[(rank, "lm")] = _lmhead(rank, P)
     finally:
         dist.destroy_process_group()
@@ -154,6 +203,15 @@ def test_rank_orchestration_over_two_processes():
     for r in range(tp):
         got = out[(r, "row")].reshape(batch, seq // tp, -1)
         assert np.allclose(got, ref[r], rtol=1e-12, atol=1e-12)
+
+    x = P["X"]
+    for _ in range(2):
+        x = O.tp_mlp(x, P["W1"], P["W2"], tp, "gelu_erf", scale=P["scale"], centered=True,
+                     norm=True, residual=True)
+    ref_mlp = O.seq_scatter(x, batch, seq, tp)
+    for r in range(tp):
+        got = out[(r, "mlp")].reshape(batch, seq // tp, -1)
+        assert np.allclose(got, ref_mlp[r], rtol=1e-12, atol=1e-12)
 
     lm = O.lmhead_argmax(P["x"], P["W"], tp, 1)
     for r in range(tp):
