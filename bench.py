@@ -470,38 +470,59 @@ class NextRows:
             self.flops = self.gemm_flops = m.flops()
             self.io_in, self.io_out = ["x"], ["y"]
         elif kind == "tp_ranks":
-            # The MLP's c_proj as tp rank-local shards, the ranks run one after
-            # another on this GPU: each rank's GEMM scatters its partial into
-            # every rank's receive buffer (local tensors standing in for peer
-            # memory), then every rank sums its slots.
+            # The RMSNorm + MLP block as tp rank-local shares, the ranks run one
+            # after another on this GPU, their peers' buffers standing in as
+            # local tensors: each rank normalises its token slice, runs c_fc +
+            # GELU over all tokens reading every rank's slice (peer gather),
+            # scatters its c_proj partials into every rank's receive buffer,
+            # and sums its slots into its slice of the residual stream.
             tp, b, sq, N, I = m.tp, m.batch, m.seq, m.hidden, m.inter
             M, kr = m.M, m.inter // m.tp
             rows = b * (sq // tp)
-            self.name = (f"tp-ranks c_proj x[{b},{sq},{I}] bf16 -> {N}, {tp} ranks in sequence "
-                         f"on one GPU (peer-scatter GEMM + slot reduction)")
+            self.name = (f"tp-ranks rmsnorm-tp-mlp x[{b},{sq},{N}] bf16 {N}->{I}->{N} "
+                         f"gelu-erf, {tp} ranks in sequence on one GPU (peer-gather c_fc, "
+                         "peer-scatter c_proj, slot reduction)")
             self.parallelism = (f"{tp} TP ranks emulated in sequence on one GPU: each rank's "
-                                "GEMM writes its partials into every rank's receive buffer, "
-                                "then every rank reduces its slots")
-            self.h = gen.normal((tp * M, kr), 1.0, tensor_id=gen.TID_X, device=dev)
+                                "c_fc reads every rank's token slice, its c_proj writes into "
+                                "every rank's receive buffer, then every rank reduces its slots")
+            self.xs = C.mlp_x(m, dev).view(b, tp, sq // tp, N).transpose(0, 1).contiguous()
+            self.scale = C.mlp_scale(m, 0, dev)
+            self.xn = torch.empty_like(self.xs)
+            self.w1 = C.mlp_w1(m, 0, dev)
             self.w2p = T.pack_row_weight(C.mlp_w2(m, 0, dev), [kr] * tp)
+            self.p_rank = T.tpl_partition_subparams([kr], 1, 1)
+            self.hbuf = torch.empty(tp * M * kr, dtype=torch.bfloat16, device=dev)
             self.recv = [torch.empty(tp * rows * N, dtype=torch.bfloat16, device=dev)
                          for _ in range(tp)]
-            self.y = torch.empty(tp * rows * N, dtype=torch.bfloat16, device=dev)
+
+            def norm_all(s):
+                for q in range(tp):
+                    T.tpl_rmsnorm(self.xs[q], self.scale, True, 1e-6, y=self.xn[q], stream=s)
+
+            def gather_all(s):
+                hs = self.hbuf.view(tp, M * kr)
+                slices = [self.xn[q] for q in range(tp)]
+                for r in range(tp):
+                    T.tpl_column_linear_gather(self.p_rank, slices, b, sq,
+                                               self.w1[r * kr:(r + 1) * kr], None, m.act,
+                                               y=hs[r], stream=s)
 
             def scatter_all(s):
-                hs, ws = self.h.view(tp, M, kr), self.w2p.view(tp, N, kr)
+                hs, ws = self.hbuf.view(tp, M, kr), self.w2p.view(tp, N, kr)
                 for r in range(tp):
                     T.tpl_row_linear_scatter(hs[r], ws[r], b, sq, r, tp, self.recv, stream=s)
 
             def reduce_all(s):
-                ys = self.y.view(tp, rows, N)
                 for q in range(tp):
-                    T.tpl_reduce_slots(self.recv[q], tp, N, None, None, y=ys[q], stream=s)
-            self.launches += [("rank_scatter_gemms", scatter_all), ("rank_slot_reductions", reduce_all)]
-            self.flops = self.gemm_flops = 2.0 * M * N * I
-            self.gemm_launches = tp            # one scatter GEMM per rank in its part
-            self.reduce_bytes = tp * (tp + 1) * rows * N * 2
-            self.io_in, self.io_out = ["h"], ["y"]
+                    x_q = self.xs[q].view(rows, N)
+                    T.tpl_reduce_slots(self.recv[q], tp, N, None, x_q, y=x_q, stream=s)
+            self.launches += [("rank_rmsnorm", norm_all), ("rank_gather_gemms", gather_all),
+                              ("rank_scatter_gemms", scatter_all),
+                              ("rank_slot_reductions", reduce_all)]
+            self.flops = self.gemm_flops = m.flops()
+            self.gemm_launches = 2 * tp         # one gather and one scatter GEMM per rank
+            self.reduce_bytes = tp * (tp + 2) * rows * N * 2
+            self.io_in, self.io_out = ["xs"], ["xs"]   # the residual stream, in place
         else:
             raise ValueError(kind)
         self.parts = [n for n, _ in self.launches]
@@ -517,7 +538,7 @@ class NextRows:
     def gemm_part_ids(self):
         return [i for i, n in enumerate(self.parts)
                 if n in ("swiglu_column", "sp_column_gelu", "sp_row_scatter",
-                         "rank_scatter_gemms")]
+                         "rank_gather_gemms", "rank_scatter_gemms")]
 
     def lmhead_bytes(self):
         return None
@@ -529,7 +550,9 @@ class NextRows:
             return [("roofline_rmsnorm", "rmsnorm_cta", "sp_rmsnorm",
                      2 * 2 * self.m.M * self.m.hidden)]
         if self.kind == "tp_ranks":
-            return [("roofline_reduce", "reduce_slots_kernel", "rank_slot_reductions",
+            return [("roofline_rmsnorm", "rmsnorm_cta", "rank_rmsnorm",
+                     2 * 2 * self.m.M * self.m.hidden, self.m.tp),
+                    ("roofline_reduce", "reduce_slots_kernel", "rank_slot_reductions",
                      self.reduce_bytes, self.m.tp)]
         return []
 
@@ -543,12 +566,13 @@ class NextRows:
             return (lambda: O.swiglu_column_linear(xs, w, self.F, m.tp),
                     2.0 * rows * m.hidden * 2 * self.F, f"{rows} token rows")
         if self.kind == "tp_ranks":
-            rows = 1024
-            tp, kr = m.tp, m.inter // m.tp
-            hs = f64(self.h.view(tp, m.M, kr)[:, :rows])
-            w2 = f64(self.w2p).reshape(tp, m.hidden, kr)
-            return (lambda: O.row_linear_reduce(list(hs), list(w2)),
-                    2.0 * rows * m.hidden * m.inter, f"{rows} token rows of the {tp} ranks")
+            rows = 128
+            tp = m.tp
+            xs = f64(self.xs.transpose(0, 1).reshape(m.M, m.hidden)[:rows])
+            w1, w2, sc = f64(self.w1), f64(C.mlp_w2(m, 0, self.xs.device)), f64(self.scale)
+            return (lambda: O.tp_mlp(xs, w1, w2, tp, m.act, scale=sc, centered=True, norm=True,
+                                     residual=True),
+                    4.0 * rows * m.hidden * m.inter, f"{rows} tokens through the block")
         if self.kind == "embed":
             sub = 16032
             table = f64(self.table[:sub])
