@@ -61,3 +61,13 @@ def test_throttled_or_locked_clocks_are_rejected():
     # far below max with no reason: a clock lock left by someone else
     assert bench.clocks_rejected({"reasons": [], "sm_mhz": 900, "sm_max_mhz": 1965})
     assert not bench.clocks_rejected({"reasons": [], "sm_mhz": 1900, "sm_max_mhz": 1965})
+
+
+def test_gemm_peak_follows_the_clock_regime():
+    pk = {"bf16_tflops": 1659.1, "bf16_tflops_sustained": 1400.6}
+    capped = {"reasons": ["sw_power_cap"], "sm_mhz": 1383, "sm_max_mhz": 1965}
+    full = {"reasons": [], "sm_mhz": 1965, "sm_max_mhz": 1965}
+    assert bench.tensor_peak(pk, "measured", capped)[0] == 1400.6
+    assert "sustained" in bench.tensor_peak(pk, "measured", capped)[1]
+    assert bench.tensor_peak(pk, "measured", full) == (1659.1, "measured bf16 burst")
+    assert bench.tensor_peak(pk, "fallback", None) == (1659.1, "fallback bf16 burst")
