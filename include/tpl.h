@@ -369,7 +369,8 @@ tpl_status tpl_row_linear_scatter(const void* h, int64_t K, int64_t batch, int64
  *   recv      device bf16 [tp][rows][N] (the receive buffer, rows = batch*seq/tp).
  *   bias      device bf16 [N] or NULL.   residual  device bf16 [rows][N] or NULL.
  *   y         device bf16 [rows][N]; may alias residual.
- * rows == 0 is a no-op.
+ * rows == 0 is a no-op.  TPL_ERR_SHAPE if tp is outside [1, TPL_MAX_TP], N is
+ * outside [1, INT32_MAX], rows < 0, or tp * rows * N overflows int64_t.
  */
 tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t N,
                             const void* bias, const void* residual, void* y, void* stream);

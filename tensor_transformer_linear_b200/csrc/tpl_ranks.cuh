@@ -151,6 +151,8 @@ tpl_status tpl_row_linear_scatter(const void* h, int64_t K, int64_t batch, int64
 tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t N,
                             const void* bias, const void* residual, void* y, void* stream) {
   if (tp < 1 || tp > TPL_MAX_TP || rows < 0 || N < 1 || N > INT32_MAX) return TPL_ERR_SHAPE;
+  // every element index of recv, tp * rows * N, must fit an int64_t
+  if (rows > INT64_MAX / (N * tp)) return TPL_ERR_SHAPE;
   if (rows == 0) return TPL_OK;
   if (recv == nullptr || y == nullptr) return TPL_ERR_NULL;
   if (!aligned(recv, 2) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||

@@ -229,6 +229,7 @@ def test_multi_gpu_rows_rejections():
     assert L.tpl_reduce_slots(None, 2, 0, 8, None, None, None, s) == 0
     assert L.tpl_reduce_slots(None, 2, 4, 8, None, None, FAKE, s) == 1
     assert L.tpl_reduce_slots(FAKE, 2, 4, 8, None, None, FAKE_ODD, s) == 5
+    assert L.tpl_reduce_slots(FAKE, 8, 2**60, 2**10, None, None, FAKE, s) == 2   # overflow
     assert L.tpl_argmax_merge(FAKE, FAKE, 2, 0, 10, FAKE, s) == 2
     assert L.tpl_argmax_merge(FAKE, FAKE, 8, 4, 2**29, FAKE, s) == 2
     assert L.tpl_argmax_merge(None, FAKE, 2, 4, 10, FAKE, s) == 1
