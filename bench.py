@@ -44,6 +44,7 @@ from workloads import gen  # noqa: E402
 
 METRIC = "sharded-linear TFLOP/s (% bf16 peak); LM-head decode GB/s (% HBM) at 1 B200"
 DECODE_LAUNCHES = 50
+ALONE_LAUNCHES = 30
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -777,6 +778,31 @@ def main():
         if pg is not None:
             decode_ms = max_over_ranks([decode_ms], dev)[0]
 
+    # ---- the HBM-bound parts alone: each launch after a read-only L2 flush (a
+    # 256 MiB sum, which evicts earlier kernels' dirty lines and leaves L2
+    # clean), timed with events around that launch alone; median of ALONE_LAUNCHES
+    alone_ms = {}
+    launch_of = dict(getattr(wl, "launches", []))
+    parts_alone = [h for h in wl.hbm_parts() if h[2] in launch_of]
+    if parts_alone:
+        flush = torch.ones(256 * 2**20 // 4, dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            for key, _, part, *_ in parts_alone:
+                fn = launch_of[part]
+                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(ALONE_LAUNCHES)]
+                for _ in range(3):
+                    fn(stream)
+                for e0, e1 in evs:
+                    flush.sum()
+                    e0.record(stream)
+                    fn(stream)
+                    e1.record(stream)
+                torch.cuda.synchronize()
+                t = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+                alone_ms[key] = max_over_ranks([t], dev)[0] if pg is not None else t
+        del flush
+
     # ---- end to end through pinned host buffers, copies inside the timed region
     e2e = E2EPipeline(wl, stream)
     b_in, b_out = e2e.bytes_in, e2e.bytes_out
@@ -870,7 +896,16 @@ def main():
             line[key] = {"kernel": kern, "bound": "hbm", "achieved": round(gb, 1),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gb / pk["hbm_gbs"], 4), "bytes_per_launch": nbytes // n_l,
-                         "launches_per_step": n_l}
+                         "launches_per_step": n_l,
+                         "measured": "inside the timed steps, after the kernel before it, whose "
+                                     "dirty output lines in L2 it evicts"}
+            if key in alone_ms:
+                ga = nbytes / (alone_ms[key] * 1e-3) / 1e9
+                line[key]["alone"] = {
+                    "achieved": round(ga, 1), "frac": round(ga / pk["hbm_gbs"], 4),
+                    "ms": round(alone_ms[key], 4),
+                    "measured": f"median of {ALONE_LAUNCHES} launches, each after a read-only "
+                                "256 MiB L2 flush, CUDA events around the launch alone"}
         if not gids:
             first = "roofline_lmhead" if "roofline_lmhead" in line else wl.hbm_parts()[0][0]
             line["roofline"] = line.pop(first)
