@@ -468,8 +468,9 @@ tpl_status rmsnorm_launch(const void* x, int64_t M, int64_t H, const float* scal
   const int t = tpl::kNormWarps * 32;
   const int Hi = static_cast<int>(H);
   if (vec && H / P >= 2 * tpl::kNormCtaThreads && cta_vec <= 16) {
-    // Wide rows: a CTA per row, up to 16 CTAs resident per SM.
-    const int gc = static_cast<int>(std::min<int64_t>(M, static_cast<int64_t>(dev->sm_count) * 16));
+    // Wide rows: a CTA per row (the block scheduler balances rows over SMs as
+    // CTAs finish), up to 16 CTAs resident per SM.
+    const int gc = static_cast<int>(std::min<int64_t>(M, INT32_MAX));
     const int tc = tpl::kNormCtaThreads;
     if (cta_vec <= 2)
       tpl::rmsnorm_cta<T, 2><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
