@@ -14,6 +14,7 @@
 namespace tpl {
 
 constexpr int kEmbedWarps = 8;
+constexpr int kEmbedBatch = 8;  // 16-byte vectors per lane in flight
 
 template <typename T, bool kVec>
 __global__ void __launch_bounds__(kEmbedWarps * 32)
@@ -35,19 +36,28 @@ __global__ void __launch_bounds__(kEmbedWarps * 32)
     }
     T* dst = out + i * H;
     if (kVec) {
+      // kEmbedBatch vectors per lane are loaded before any is stored, so a warp
+      // keeps kEmbedBatch * 512 bytes of the row in flight.
       const int64_t nv = H / P;
       const uint4* src = reinterpret_cast<const uint4*>(table + (row < 0 ? 0 : row) * H);
-      for (int64_t v = lane; v < nv; v += 32) {
-        float acc[P];
+      for (int64_t v0 = lane; v0 < nv; v0 += 32 * kEmbedBatch) {
+        uint4 q[kEmbedBatch];
 #pragma unroll
-        for (int e = 0; e < P; ++e) acc[e] = 0.0f;
-        if (row >= 0) {
-          float f[P];
-          VT::unpack(__ldcs(src + v), f);
-#pragma unroll
-          for (int e = 0; e < P; ++e) acc[e] += f[e];
+        for (int u = 0; u < kEmbedBatch; ++u) {
+          const int64_t v = v0 + 32 * u;
+          q[u] = (row >= 0 && v < nv) ? __ldcs(src + v) : make_uint4(0u, 0u, 0u, 0u);
         }
-        __stcs(reinterpret_cast<uint4*>(dst) + v, VT::pack(acc));
+#pragma unroll
+        for (int u = 0; u < kEmbedBatch; ++u) {
+          const int64_t v = v0 + 32 * u;
+          if (v < nv) {
+            float f[P], acc[P];
+            VT::unpack(q[u], f);
+#pragma unroll
+            for (int e = 0; e < P; ++e) acc[e] = 0.0f + f[e];
+            __stcs(reinterpret_cast<uint4*>(dst) + v, VT::pack(acc));
+          }
+        }
       }
     } else {
       for (int64_t c = lane; c < H; c += 32) {
