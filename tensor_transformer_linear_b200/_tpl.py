@@ -405,9 +405,15 @@ def tpl_column_linear_gather(p: Partition, peer_x: Sequence, batch: int, seq: in
     for q, b in enumerate(peer_x):
         if isinstance(b, torch.Tensor) and b.numel() != M // tp * K:
             raise ValueError(f"peer_x[{q}] must be [batch, seq // tp, K]")
+    if w.numel() != p.logical_out * K:
+        raise ValueError("w must be [logical_out, K]")
+    if bias is not None and bias.numel() != p.logical_out:
+        raise ValueError("bias must be [logical_out]")
     if y is None:
         y = torch.empty(M * p.logical_out, dtype=torch.bfloat16, device=w.device)
     _cuda(y, "y", torch.bfloat16)
+    if y.numel() < M * p.logical_out:
+        raise ValueError("y must hold batch * seq * logical_out elements")
     _check(lib().tpl_column_linear_gather(ctypes.byref(p), _addresses(peer_x, "peer_x"), int(tp),
                                           int(batch), int(seq), int(K), _ptr(w), _ptr(bias),
                                           ACT[act], _ptr(y), _stream(stream)),
@@ -459,6 +465,8 @@ def tpl_reduce_slots(recv: torch.Tensor, tp: int, N: int, bias: Optional[torch.T
     _cuda(y, "y", torch.bfloat16)
     if bias is not None:
         _cuda(bias, "bias", torch.bfloat16)
+        if bias.numel() != N:
+            raise ValueError("bias must be [N]")
     if residual is not None:
         _cuda(residual, "residual", torch.bfloat16)
         if residual.numel() != rows * N:
@@ -481,6 +489,8 @@ def tpl_argmax_merge(shard_max: torch.Tensor, shard_idx: torch.Tensor, id_stride
     if ids is None:
         ids = torch.empty(B, dtype=torch.int32, device=shard_max.device)
     _cuda(ids, "ids", torch.int32)
+    if ids.numel() < B:
+        raise ValueError("ids must hold B elements")
     _check(lib().tpl_argmax_merge(_ptr(shard_max), _ptr(shard_idx), int(tp), int(B),
                                   int(id_stride), _ptr(ids), _stream(stream)), "tpl_argmax_merge")
     return ids
