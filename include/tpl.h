@@ -376,6 +376,39 @@ tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t 
                             const void* bias, const void* residual, void* y, void* stream);
 
 /*
+ * The same reduction, with the slice stored into EVERY rank's full output
+ * (google-research: the row-parallel partials reduced over the sharded
+ * contraction axis; nanotron "MLP Module" without sequence parallelism, where
+ * each rank keeps the whole [batch, seq, hidden] output).  Rank `rank` owns
+ * tokens rank * seq/tp .. (rank + 1) * seq/tp of every sequence; it computes
+ *   S[b][t][n] = bf16( sum_{s < tp} recv[s][b][t][n] + bias[n]
+ *                      + residual[b * seq + rank * seq/tp + t][n] )
+ * and stores S at row b * seq + rank * seq/tp + t of peer_y[q] for every q.
+ * After tpl_row_linear_scatter, a barrier and this call on every rank, and a
+ * second barrier, every rank's output holds the full
+ *   Y = sum_r H_r W2_r^T (+ bias) (+ residual):
+ * an all-reduce whose data moves only in the GEMM epilogue's and this
+ * kernel's peer stores.
+ *   recv      device bf16 [tp][batch][seq/tp][N], this rank's receive buffer.
+ *   bias      device bf16 [N] or NULL.
+ *   residual  device bf16 [batch * seq][N] or NULL: this rank's own copy of
+ *             the residual stream (identical on every rank); it may alias
+ *             peer_y[rank] (in place), as each element of this rank's token
+ *             rows is read and then stored by one thread, and no other rank
+ *             writes those rows.
+ *   peer_y    array of tp pointers: rank q's output [batch * seq][N] bf16 (a
+ *             mapped peer address for q != rank).  The caller keeps the
+ *             mappings valid until the stream has passed this call.
+ * Requirements: seq % tp == 0 (else TPL_ERR_INDIVISIBLE), 0 <= rank < tp,
+ * 1 <= N <= INT32_MAX, batch * seq <= INT32_MAX (else TPL_ERR_SHAPE); every
+ * pointer 2-byte aligned (else TPL_ERR_ALIGN).  16-byte alignment of every
+ * buffer and N % 8 == 0 select the vectorised kernel.
+ */
+tpl_status tpl_reduce_slots_allgather(const void* recv, int32_t tp, int64_t batch, int64_t seq,
+                                      int64_t N, const void* bias, const void* residual,
+                                      int32_t rank, void* const* peer_y, void* stream);
+
+/*
  * Global argmax of a vocab split over tp GPUs (Tenstorrent LMHead1D: every
  * device's candidates combined at the end).  Rank s ran tpl_lmhead_argmax on
  * its vocab slice (ids local to the slice); after an all-gather of those

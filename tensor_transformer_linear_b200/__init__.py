@@ -11,8 +11,9 @@ from ._tpl import (EXPORTED, Partition, TplError, lib, lmhead_workspace,  # noqa
                    tpl_row_linear_reduce_scatter, tpl_column_linear_allgather,
                    tpl_swiglu_column_linear, tpl_embedding_lookup, tpl_selftest_wait_timeout,
                    tpl_row_linear_scatter, tpl_reduce_slots, tpl_argmax_merge,
-                   tpl_column_linear_gather)
-from .path import (TPMLP, TPLMHeadRank, TPRankMLP, TPRowParallelRank, TPStack,  # noqa: F401
+                   tpl_column_linear_gather, tpl_reduce_slots_allgather)
+from .path import (TPMLP, TPLMHeadRank, TPRankMLP, TPRowParallelAllReduceRank,  # noqa: F401
+                   TPRowParallelRank, TPStack,
                    PeerBuffers,
                    exchange_peer_buffers, local_peer_buffers, pack_row_weight, recv_buffer_numel,
                    shard_views, sp_rows, sp_slice, sp_token_owner, stream_barrier)

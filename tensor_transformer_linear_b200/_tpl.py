@@ -33,7 +33,7 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_lmhead_argmax_static", "tpl_row_linear_reduce_scatter",
             "tpl_column_linear_allgather", "tpl_swiglu_column_linear", "tpl_embedding_lookup",
             "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
-            "tpl_argmax_merge", "tpl_column_linear_gather")
+            "tpl_argmax_merge", "tpl_column_linear_gather", "tpl_reduce_slots_allgather")
 
 
 class TplError(RuntimeError):
@@ -95,6 +95,8 @@ def lib():
         L.tpl_row_linear_scatter.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32,
                                              ctypes.POINTER(vp), vp]
         L.tpl_reduce_slots.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+        L.tpl_reduce_slots_allgather.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32,
+                                                 ctypes.POINTER(vp), vp]
         L.tpl_argmax_merge.argtypes = [vp, vp, i32, i64, i64, vp, vp]
         L.tpl_column_linear_gather.argtypes = [ctypes.POINTER(Partition), ctypes.POINTER(vp), i32,
                                                i64, i64, i64, vp, vp, i32, vp, vp]
@@ -476,6 +478,38 @@ def tpl_reduce_slots(recv: torch.Tensor, tp: int, N: int, bias: Optional[torch.T
     _check(lib().tpl_reduce_slots(_ptr(recv), int(tp), int(rows), int(N), _ptr(bias),
                                   _ptr(residual), _ptr(y), _stream(stream)), "tpl_reduce_slots")
     return y
+
+
+def tpl_reduce_slots_allgather(recv: torch.Tensor, tp: int, batch: int, seq: int, N: int,
+                               rank: int, peers_y: Sequence,
+                               bias: Optional[torch.Tensor] = None,
+                               residual: Optional[torch.Tensor] = None, stream=None) -> None:
+    """This rank's token slice of ``sum of the tp slots of recv (+ bias)
+    (+ residual)``, stored at its rows of every rank's full ``[batch * seq, N]``
+    output ``peers_y[q]`` (a CUDA tensor, or a mapped peer address); see
+    include/tpl.h.  ``residual`` is this rank's full ``[batch * seq, N]``
+    residual stream and may be ``peers_y[rank]`` itself."""
+    _cuda(recv, "recv", torch.bfloat16)
+    M = int(batch) * int(seq)
+    if len(peers_y) != tp:
+        raise ValueError("peers_y must hold one output buffer per rank")
+    if recv.numel() != M * N:
+        raise ValueError("recv must be [tp][batch][seq // tp][N]")
+    if bias is not None:
+        _cuda(bias, "bias", torch.bfloat16)
+        if bias.numel() != N:
+            raise ValueError("bias must be [N]")
+    if residual is not None:
+        _cuda(residual, "residual", torch.bfloat16)
+        if residual.numel() != M * N:
+            raise ValueError("residual must be [batch * seq][N]")
+    for q, t in enumerate(peers_y):
+        if isinstance(t, torch.Tensor) and t.numel() < M * N:
+            raise ValueError(f"peers_y[{q}] is smaller than [batch * seq][N]")
+    _check(lib().tpl_reduce_slots_allgather(_ptr(recv), int(tp), int(batch), int(seq), int(N),
+                                            _ptr(bias), _ptr(residual), int(rank),
+                                            _addresses(peers_y, "peers_y"), _stream(stream)),
+           "tpl_reduce_slots_allgather")
 
 
 def tpl_argmax_merge(shard_max: torch.Tensor, shard_idx: torch.Tensor, id_stride: int,

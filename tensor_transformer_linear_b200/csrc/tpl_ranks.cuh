@@ -14,6 +14,10 @@
 //   tpl_reduce_slots        once every rank's scatter has completed, a rank sums
 //       its tp slots (in rank order, fp32) plus bias and residual: its token
 //       slice of the reduced output (the reduce-scatter).
+//   tpl_reduce_slots_allgather  the same sum, stored into every rank's full
+//       [batch * seq][N] output at the rank's token rows (peer stores), so that
+//       once every rank has run it, every rank holds the whole reduced output:
+//       with the scatter before it, an all-reduce of the partials.
 //   tpl_argmax_merge        the per-rank LM-head candidates, gathered, reduced to
 //       the global argmax (ties to the lowest global id).
 //
@@ -72,6 +76,68 @@ __global__ void __launch_bounds__(kReduceThreads)
       if (bias != nullptr) acc += bf16_to_f(bias[i % N]);
       if (residual != nullptr) acc += bf16_to_f(residual[i]);
       y[i] = __float2bfloat16_rn(acc);
+    }
+  }
+}
+
+struct PeerOut {
+  __nv_bfloat16* y[kMaxPeers];
+};
+
+// The slice sum of reduce_slots_kernel, stored into every rank's full output:
+// slice element i (row i / N = b * seg + t, column i % N) goes to full row
+// b * seq + rank * seg + t of out.y[0 .. tp).  residual, if given, is the
+// rank's own full [batch * seq][N] residual stream, read at that full row, and
+// may alias out.y[rank].  kVec as in reduce_slots_kernel.
+template <bool kVec>
+__global__ void __launch_bounds__(kReduceThreads)
+    reduce_slots_allgather_kernel(const __nv_bfloat16* __restrict__ recv, int tp, int64_t total,
+                                  int N, int seg, int seq, int rank,
+                                  const __nv_bfloat16* __restrict__ bias,
+                                  const __nv_bfloat16* residual, const PeerOut out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x * (kVec ? 8 : 1);
+  for (int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * (kVec ? 8 : 1);
+       i < total; i += stride) {
+    const int64_t row = i / N;
+    const int64_t col = i - row * N;
+    const int64_t b = row / seg;
+    const int64_t dst = (b * seq + static_cast<int64_t>(rank) * seg + (row - b * seg)) * N + col;
+    if (kVec) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < tp; ++s) {
+        const uint4 q = __ldcs(reinterpret_cast<const uint4*>(recv + s * total + i));
+        acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
+        acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
+        acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
+        acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
+      }
+      if (bias != nullptr) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(bias + col));
+        acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
+        acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
+        acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
+        acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
+      }
+      if (residual != nullptr) {
+        const uint4 q = *reinterpret_cast<const uint4*>(residual + dst);
+        acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
+        acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
+        acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
+        acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      for (int q = 0; q < tp; ++q) *reinterpret_cast<uint4*>(out.y[q] + dst) = o;
+    } else {
+      float acc = 0.f;
+      for (int s = 0; s < tp; ++s) acc += bf16_to_f(recv[s * total + i]);
+      if (bias != nullptr) acc += bf16_to_f(bias[col]);
+      if (residual != nullptr) acc += bf16_to_f(residual[dst]);
+      const __nv_bfloat16 o = __float2bfloat16_rn(acc);
+      for (int q = 0; q < tp; ++q) out.y[q][dst] = o;
     }
   }
 }
@@ -178,6 +244,47 @@ tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t 
     tpl::reduce_slots_kernel<true><<<grid, tpl::kReduceThreads, 0, st>>>(rv, tp, total, Ni, bv, res, yv);
   else
     tpl::reduce_slots_kernel<false><<<grid, tpl::kReduceThreads, 0, st>>>(rv, tp, total, Ni, bv, res, yv);
+  return launched();
+}
+
+tpl_status tpl_reduce_slots_allgather(const void* recv, int32_t tp, int64_t batch, int64_t seq,
+                                      int64_t N, const void* bias, const void* residual,
+                                      int32_t rank, void* const* peer_y, void* stream) {
+  SeqPar sp;
+  tpl_status s = seqpar_of(batch, seq, tp, &sp);
+  if (s != TPL_OK) return s;
+  if (rank < 0 || rank >= tp || N < 1 || N > INT32_MAX) return TPL_ERR_SHAPE;
+  // every element index of the full output, batch * seq * N, must fit an int64_t
+  if (static_cast<int64_t>(sp.batch) * sp.seq > INT64_MAX / N) return TPL_ERR_SHAPE;
+  if (recv == nullptr || peer_y == nullptr) return TPL_ERR_NULL;
+  bool vec = (N % 8 == 0) && aligned(recv, 16) && (bias == nullptr || aligned(bias, 16)) &&
+             (residual == nullptr || aligned(residual, 16));
+  tpl::PeerOut out{};
+  for (int q = 0; q < tp; ++q) {
+    if (peer_y[q] == nullptr) return TPL_ERR_NULL;
+    if (!aligned(peer_y[q], 2)) return TPL_ERR_ALIGN;
+    vec = vec && aligned(peer_y[q], 16);
+    out.y[q] = static_cast<__nv_bfloat16*>(peer_y[q]);
+  }
+  if (!aligned(recv, 2) || (bias && !aligned(bias, 2)) || (residual && !aligned(residual, 2)))
+    return TPL_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  if ((s = device_info(&dev)) != TPL_OK) return s;
+  const int64_t total = static_cast<int64_t>(sp.batch) * sp.seg * N;  // this rank's slice
+  const int64_t per_block = static_cast<int64_t>(tpl::kReduceThreads) * (vec ? 8 : 1);
+  const int grid = static_cast<int>(std::min<int64_t>((total + per_block - 1) / per_block,
+                                                      static_cast<int64_t>(dev->sm_count) * 8));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* rv = static_cast<const __nv_bfloat16*>(recv);
+  const auto* bv = static_cast<const __nv_bfloat16*>(bias);
+  const auto* res = static_cast<const __nv_bfloat16*>(residual);
+  const int Ni = static_cast<int>(N);
+  if (vec)
+    tpl::reduce_slots_allgather_kernel<true><<<grid, tpl::kReduceThreads, 0, st>>>(
+        rv, tp, total, Ni, sp.seg, sp.seq, rank, bv, res, out);
+  else
+    tpl::reduce_slots_allgather_kernel<false><<<grid, tpl::kReduceThreads, 0, st>>>(
+        rv, tp, total, Ni, sp.seg, sp.seq, rank, bv, res, out);
   return launched();
 }
 

@@ -14,7 +14,8 @@ import torch
 
 from ._tpl import (Partition, tpl_argmax_merge, tpl_column_linear, tpl_column_linear_gather,
                    tpl_lmhead_argmax, tpl_lmhead_workspace_size, tpl_partition_subparams,
-                   tpl_reduce_slots, tpl_rmsnorm, tpl_row_linear_reduce, tpl_row_linear_scatter)
+                   tpl_reduce_slots, tpl_reduce_slots_allgather, tpl_rmsnorm,
+                   tpl_row_linear_reduce, tpl_row_linear_scatter)
 
 
 def shard_views(y: torch.Tensor, p: Partition, M: int) -> List[torch.Tensor]:
@@ -215,6 +216,51 @@ class TPRowParallelRank:
         out = self.reduce(self.peers.local, self.tp, N, bias, residual, y, stream=stream)
         self.barrier(stream)
         return out
+
+
+class TPRowParallelAllReduceRank:
+    """Rank ``rank``'s row-parallel linear over ``tp`` GPUs with the full output
+    on every rank (google-research: the partials reduced over the sharded
+    contraction axis; nanotron "MLP Module" without sequence parallelism).
+
+    Each call: scatter (this rank's partial into every owner's receive buffer)
+    -> barrier -> sum this rank's slots (+ bias, + residual) and store the
+    token slice into every rank's output -> barrier.  Together an all-reduce;
+    the data moves only in the library's peer stores.  The first barrier makes
+    every partial visible before any rank sums; the second makes every slice
+    visible before any rank reads its output, and keeps the next call from
+    overwriting slots or outputs a slower rank still uses.
+
+    ``recv`` holds the receive buffers (:func:`recv_buffer_numel` elements),
+    ``out`` the ``[batch*seq, N]`` outputs.  ``w_shard`` is ``[N, k]``, this
+    rank's columns of the unsharded weight.  ``scatter`` and ``reduce``
+    default to the library's calls.
+    """
+
+    def __init__(self, w_shard: torch.Tensor, rank: int, tp: int, recv: PeerBuffers,
+                 out: PeerBuffers, barrier: Callable, scatter: Optional[Callable] = None,
+                 reduce: Optional[Callable] = None):
+        self.w = w_shard.contiguous()
+        self.rank, self.tp, self.recv, self.out = rank, tp, recv, out
+        self.barrier = barrier
+        self.scatter = scatter or tpl_row_linear_scatter
+        self.reduce = reduce or tpl_reduce_slots_allgather
+
+    def __call__(self, h_shard: torch.Tensor, batch: int, seq: int,
+                 bias: Optional[torch.Tensor] = None, residual: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        """``h_shard`` ``[batch*seq, k]``; ``residual`` this rank's full
+        ``[batch*seq, N]`` residual stream (it may be ``out.local``).  Returns
+        ``out.local`` as ``[batch*seq, N]``, the full Y."""
+        N = self.w.shape[0]
+        sp_rows(batch, seq, self.tp)
+        self.scatter(h_shard, self.w, batch, seq, self.rank, self.tp, self.recv.addrs,
+                     stream=stream)
+        self.barrier(stream)
+        self.reduce(self.recv.local, self.tp, batch, seq, N, self.rank, self.out.addrs,
+                    bias=bias, residual=residual, stream=stream)
+        self.barrier(stream)
+        return self.out.local.view(batch * seq, N)
 
 
 class TPRankMLP:

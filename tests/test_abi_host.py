@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 19, names
+    assert len(names) == 20, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -230,6 +230,17 @@ def test_multi_gpu_rows_rejections():
     assert L.tpl_reduce_slots(None, 2, 4, 8, None, None, FAKE, s) == 1
     assert L.tpl_reduce_slots(FAKE, 2, 4, 8, None, None, FAKE_ODD, s) == 5
     assert L.tpl_reduce_slots(FAKE, 8, 2**60, 2**10, None, None, FAKE, s) == 2   # overflow
+    ag = L.tpl_reduce_slots_allgather
+    ys = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert ag(FAKE, 0, 2, 8, 16, None, None, 0, ys, s) == 2                 # tp
+    assert ag(FAKE, 2, 2, 7, 16, None, None, 0, ys, s) == 3                 # seq % tp
+    assert ag(FAKE, 2, 2, 8, 16, None, None, 2, ys, s) == 2                 # rank
+    assert ag(FAKE, 2, 2, 8, 0, None, None, 0, ys, s) == 2                  # N
+    assert ag(None, 2, 2, 8, 16, None, None, 0, ys, s) == 1
+    assert ag(FAKE, 2, 2, 8, 16, None, None, 0, None, s) == 1
+    assert ag(FAKE, 2, 2, 8, 16, None, None, 0, (ctypes.c_void_p * 2)(FAKE, None), s) == 1
+    assert ag(FAKE, 2, 2, 8, 16, None, None, 1, (ctypes.c_void_p * 2)(FAKE_ODD, FAKE), s) == 5
+    assert ag(FAKE, 2, 2, 8, 16, None, FAKE_ODD, 0, ys, s) == 5
     assert L.tpl_argmax_merge(FAKE, FAKE, 2, 0, 10, FAKE, s) == 2
     assert L.tpl_argmax_merge(FAKE, FAKE, 8, 4, 2**29, FAKE, s) == 2
     assert L.tpl_argmax_merge(None, FAKE, 2, 4, 10, FAKE, s) == 1

@@ -2,7 +2,8 @@
 another on one GPU: every rank's scatter writes into the receive buffers of all
 ranks (here local tensors standing in for its peers'; no kernel waits on
 another), then every rank reduces its slots.  Checked against the fp64 oracle:
-the reduce-scatter result, every slot's partial, and the argmax merged over
+the reduce-scatter result, every slot's partial, the all-reduce form (every
+rank's slice stored into every rank's full output), and the argmax merged over
 ranks."""
 import numpy as np
 import pytest
@@ -81,6 +82,58 @@ def test_scatter_then_reduce_is_the_reduce_scatter(tp, batch, seq, inter, N, wit
         slots = f64(recv[q]).reshape(tp, batch, seg, N)
         for s in range(tp):
             assert rel(slots[s], O.seq_scatter(parts[s], batch, seq, tp)[q]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("tp,batch,seq,inter,N,with_bias,res_mode", [
+    (4, 2, 256, 512, 256, True, "in_place"),    # vector kernel, residual = the output
+    (2, 1, 64, 128, 130, False, "separate"),    # N % 8 != 0: scalar kernel
+    (8, 1, 1024, 1792, 512, False, "none"),     # tp 8, the MLP's contraction split
+    (3, 2, 96, 200, 64, True, "separate"),      # uneven contraction split 72/64/64
+])
+def test_scatter_then_reduce_allgather_is_the_full_row_linear_on_every_rank(
+        tp, batch, seq, inter, N, with_bias, res_mode):
+    part = O.partition_subparams([inter], tp, 8)
+    k_w = part.shard_width
+    M = batch * seq
+    H = _t((M, inter), 1.0, 0)
+    W2 = _t((N, inter), 0.02, 2)
+    bias = _t((N,), 0.02, 3) if with_bias else None
+    res = _t((M, N), 1.0, 4) if res_mode != "none" else None
+
+    recv = [torch.full((M * N,), float("nan"), dtype=torch.bfloat16, device=DEV)
+            for _ in range(tp)]
+    if res_mode == "in_place":      # every rank's output starts as its residual stream
+        outs = [res.to(DEV) for _ in range(tp)]
+    else:
+        outs = [torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+                for _ in range(tp)]
+    koff = 0
+    for r in range(tp):
+        hr = H[:, koff:koff + k_w[r]].contiguous().to(DEV)
+        wr = W2[:, koff:koff + k_w[r]].contiguous().to(DEV)
+        T.tpl_row_linear_scatter(hr, wr, batch, seq, r, tp, recv)
+        koff += k_w[r]
+    bias_d = bias.to(DEV) if bias is not None else None
+    for q in range(tp):
+        res_q = None
+        if res_mode == "in_place":
+            res_q = outs[q]
+        elif res_mode == "separate":
+            res_q = res.to(DEV)
+        T.tpl_reduce_slots_allgather(recv[q], tp, batch, seq, N, q, outs, bias=bias_d,
+                                     residual=res_q)
+    torch.cuda.synchronize()
+
+    h_parts, off = [], 0
+    for k in k_w:
+        h_parts.append(f64(H)[:, off:off + k])
+        off += k
+    ref = O.row_linear_reduce(h_parts, O.row_weight_slices(f64(W2), k_w),
+                              None if bias is None else f64(bias),
+                              None if res is None else f64(res))
+    for q in range(tp):
+        assert rel(outs[q], ref) <= TOL_BF16, q
+        assert torch.equal(outs[q], outs[0]), q      # every rank holds the same Y
 
 
 def test_reduce_slots_in_place_on_the_residual():

@@ -1,9 +1,11 @@
 """Host logic of the TP linears split over GPUs, run as two real processes with
-gloo on CPU: the rank orchestration of path.py (the row-parallel
+gloo on CPU.  Covered: the rank orchestration of path.py -- the row-parallel
 scatter -> barrier -> reduce -> barrier sequence with its token-slice helpers,
-the whole sequence-parallel MLP block of TPRankMLP over two layers, and the LM
-head's gather of per-rank candidates), its stream barrier and its gather.  The per-rank GPU kernels are replaced by CPU stand-ins that do what
-include/tpl.h says they do; the kernels themselves are tested on the GPU in
+in its reduce-scatter form and in its all-reduce form (the full output on
+every rank); the whole sequence-parallel MLP block of TPRankMLP over two
+layers; the LM head's gather of per-rank candidates -- with its stream barrier
+and its gather.  The per-rank GPU kernels are replaced by CPU stand-ins that
+do what include/tpl.h says they do; the kernels themselves are tested on the GPU in
 test_gpu_ranks.py.  The results are checked against the fp64 oracle."""
 import datetime
 import os
@@ -90,6 +92,58 @@ def _row_parallel(rank, P):
     return y.numpy()
 
 
+def _row_allreduce(rank, P):
+    from tensor_transformer_linear_b200 import path
+    tp, batch, seq, N = WORLD, P["batch"], P["seq"], P["N"]
+    part = O.partition_subparams([P["inter"]], tp, 1)
+    off = sum(part.shard_width[:rank])
+    k = part.shard_width[rank]
+    h = torch.from_numpy(P["H"][:, off:off + k].copy())
+    w = torch.from_numpy(P["W2"][:, off:off + k].copy())
+    recv = torch.full((path.recv_buffer_numel(tp, batch, seq, N),), float("nan"),
+                      dtype=torch.float64)
+    out = torch.from_numpy(P["res"].copy())          # in place on the residual stream
+    calls = []
+
+    def scatter(h_, w_, b_, s_, r_, tp_, addrs, stream=None):
+        calls.append("scatter")
+        full = h_ @ w_.T
+        parts = [torch.empty_like(full) for _ in range(tp_)]
+        dist.all_gather(parts, full)
+        slots = recv.view(tp_, -1, N)
+        for src in range(tp_):
+            slots[src] = path.sp_slice(parts[src], b_, s_, tp_, rank).reshape(-1, N)
+
+    def reduce(recv_, tp_, b_, s_, N_, r_, addrs, bias=None, residual=None, stream=None):
+        # what tpl_reduce_slots_allgather leaves in every rank's output: rank r_'s
+        # token rows hold the sum of its slots + bias + its residual rows
+        calls.append("reduce")
+        rows = path.sp_slice(residual, b_, s_, tp_, r_).reshape(-1, N_)
+        mine = recv_.view(tp_, -1, N_).sum(0) + rows
+        if bias is not None:
+            mine = mine + bias
+        slices = [torch.empty_like(mine) for _ in range(tp_)]
+        dist.all_gather(slices, mine)
+        seg = s_ // tp_
+        full = out.view(b_, s_, N_)
+        for src in range(tp_):
+            full[:, src * seg:(src + 1) * seg] = slices[src].view(b_, seg, N_)
+
+    barrier = path.stream_barrier()
+
+    def counted_barrier(stream=None):
+        calls.append("barrier")
+        barrier(stream)
+
+    layer = path.TPRowParallelAllReduceRank(w, rank, tp, path.PeerBuffers(recv, [0] * tp),
+                                            path.PeerBuffers(out, [0] * tp), counted_barrier,
+                                            scatter=scatter, reduce=reduce)
+    y = layer(h, batch, seq, bias=torch.from_numpy(P["bias"]), residual=out)
+    assert calls == ["scatter", "barrier", "reduce", "barrier"]
+    assert y.shape == (batch * seq, N)
+    return y.numpy().copy()
+
+
 def _mlp_block(rank, P):
     from tensor_transformer_linear_b200 import path
     tp, batch, seq, N, I = WORLD, P["batch"], P["seq"], P["N"], P["inter"]
@@ -170,6 +224,7 @@ def _worker(rank, port, P, out):
                             timeout=datetime.timedelta(seconds=60))
     try:
         out[(rank, "row")] = _row_parallel(rank, P)
+        out[(rank, "allreduce")] = _row_allreduce(rank, P)
         out[(rank, "mlp")] = _mlp_block(rank, P)
         out[(rank, "lm")] = _lmhead(rank, P)
     finally:
@@ -203,6 +258,11 @@ def test_rank_orchestration_over_two_processes():
     for r in range(tp):
         got = out[(r, "row")].reshape(batch, seq // tp, -1)
         assert np.allclose(got, ref[r], rtol=1e-12, atol=1e-12)
+
+    ref_full = O.row_linear_reduce(h_parts, O.row_weight_slices(P["W2"], part.shard_width),
+                                   P["bias"], P["res"])
+    for r in range(tp):
+        assert np.allclose(out[(r, "allreduce")], ref_full, rtol=1e-12, atol=1e-12)
 
     x = P["X"]
     for _ in range(2):
