@@ -39,7 +39,10 @@
  *   - A kernel that gives up waiting on its own pipeline records
  *     TPL_ERR_TIMEOUT in a per-device status word; tpl_get_device_status reads
  *     and clears it.
- *   - The library allocates no device memory.  The calls are thread-safe.
+ *   - The library allocates no device memory.  Its only device state is two
+ *     module-level variables per device, loaded with the library: the status
+ *     word and the fixed scratch of tpl_lmhead_argmax_static.  The calls are
+ *     thread-safe.
  */
 #ifndef TPL_H
 #define TPL_H
