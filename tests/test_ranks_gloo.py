@@ -277,3 +277,59 @@ def test_rank_orchestration_over_two_processes():
     for r in range(tp):
         assert list(out[(r, "lm")]) == [int(v) for v in lm.ids]
     assert int(lm.ids[1]) == 4          # the tie went to the lower global id
+
+
+def _leaver_worker(rank, port, step1_done, out):
+    """Both ranks run one row-parallel step; then rank 1 leaves (between steps,
+    nothing in flight) and rank 0 runs the next step, whose barrier must end with
+    an error within the process-group timeout instead of waiting for good."""
+    import time
+    from tensor_transformer_linear_b200 import path
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD,
+                            timeout=datetime.timedelta(seconds=5))
+    batch, seq, N, k = 1, 4, 3, 2
+    recv = torch.zeros(path.recv_buffer_numel(WORLD, batch, seq, N), dtype=torch.float64)
+
+    def scatter(h_, w_, b_, s_, r_, tp_, addrs, stream=None):
+        pass                                    # the exchange itself is not under test
+
+    def reduce(recv_, tp_, N_, bias_, res_, y_, stream=None):
+        return recv_.view(tp_, -1, N_).sum(0)
+
+    layer = path.TPRowParallelRank(torch.ones(N, k, dtype=torch.float64), rank, WORLD,
+                                   path.PeerBuffers(recv, [0] * WORLD), path.stream_barrier(),
+                                   scatter=scatter, reduce=reduce)
+    h = torch.ones(batch * seq, k, dtype=torch.float64)
+    layer(h, batch, seq)
+    if rank == 1:
+        step1_done.wait(30)
+        os._exit(0)                             # leaves without a word to rank 0
+    step1_done.set()
+    time.sleep(0.5)
+    t0 = time.monotonic()
+    try:
+        layer(h, batch, seq)
+        out["result"] = "returned"
+    except Exception as e:                      # gloo reports the lost peer or the timeout
+        out["result"] = "error"
+        out["kind"] = type(e).__name__
+    out["seconds"] = time.monotonic() - t0
+    os._exit(0)                                 # the group cannot be torn down cleanly
+
+
+def test_a_rank_that_leaves_ends_the_next_barrier_with_an_error():
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    step1_done = ctx.Event()
+    port = _free_port()
+    procs = [ctx.Process(target=_leaver_worker, args=(r, port, step1_done, out))
+             for r in range(WORLD)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert out.get("result") == "error", dict(out)
+    assert out["seconds"] < 30, dict(out)
