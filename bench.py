@@ -311,37 +311,6 @@ class Block:
             return []
         return [("roofline_rmsnorm", "rmsnorm_cta", "rmsnorm", 2 * 2 * self.m.M * self.m.hidden)]
 
-    # --- the oracle on a bounded sample (CPU baseline / reference arm)
-    def oracle_sample(self, rows_qkv=256, rows_mlp=96, lm_rows=16032):
-        import numpy as np
-        import oracle as O
-        f64 = lambda t: t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
-        q, m, l = self.q, self.m, self.l
-        jobs, flops, desc = [], 0.0, []
-        if "qkv" in self.sel:
-            xq, wq, bq = f64(self.qx[:rows_qkv]), f64(self.qw), f64(self.qb)
-            part = O.partition_subparams(list(q.sub_sizes), q.tp, q.align)
-            jobs.append(lambda: O.column_linear(xq, wq, bq, part))
-            flops += 2.0 * rows_qkv * q.hidden * q.out
-            desc.append(f"{rows_qkv} token rows of the fused QKV")
-        if "mlp" in self.sel:
-            xm, w1 = f64(self.mx[:rows_mlp]), f64(self.mlp.w1)
-            w2, sc = f64(C.mlp_w2(m, 0, self.mx.device)), f64(self.mlp.scale)
-            jobs.append(lambda: O.tp_mlp(xm, w1, w2, m.tp, m.act, scale=sc, centered=True,
-                                         norm=True))
-            flops += 4.0 * rows_mlp * m.hidden * m.inter
-            desc.append(f"{rows_mlp} token rows of the RMSNorm+MLP")
-        if "lmhead" in self.sel:
-            xl, wl = f64(self.lx), f64(self.lw[:lm_rows])
-            jobs.append(lambda: O.lmhead_argmax(xl, wl, 1, 1))
-            flops += 2.0 * l.batch * l.hidden * lm_rows
-            desc.append(f"{lm_rows} vocab rows x {l.batch} batch rows of the LM head")
-
-        def run():
-            for j in jobs:
-                j()
-        return run, flops, ", ".join(desc)
-
 
 class Stack:
     """The 4-layer residual TP stack."""
@@ -398,20 +367,6 @@ class Stack:
     def gemm_part_ids(self):
         return [i for i in range(len(self.parts)) if i % 3 != 0]
 
-    def oracle_sample(self, rows=8):
-        import numpy as np
-        import oracle as O
-        f64 = lambda t: t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
-        w = self.w
-        xs = f64(self.x0[:rows])
-        layers = [(f64(l.w1), f64(C.mlp_w2(w, i, self.x0.device)), None)
-                  for i, l in enumerate(self.layers)]
-
-        def run():
-            O.tp_stack(xs, layers, w.tp, w.act)
-        return run, w.layers * 4.0 * rows * w.hidden * w.inter, \
-            f"{rows} token rows through all {w.layers} layers"
-
 
 class NextRows:
     """Workloads of the path's next rows, one at a time (measured like the block).
@@ -435,7 +390,7 @@ class NextRows:
         self.launches = []
         if kind == "swiglu":
             self.F = m.inter
-            self.name = (f"fused-swiglu-column x[8,1024,4096] bf16 4096->2x{self.F} tp{m.tp}")
+            self.name = WORKLOAD_NAMES["swiglu"]
             self.x = C.mlp_x(m, dev)
             self.w = gen.normal((2 * self.F, m.hidden), m.w_sigma, tensor_id=gen.TID_W1,
                                 device=dev)
@@ -445,8 +400,7 @@ class NextRows:
             self.flops = self.gemm_flops = 2.0 * m.M * m.hidden * 2 * self.F
             self.io_in, self.io_out = ["x"], ["h"]
         elif kind == "embed":
-            self.name = (f"vocab-sharded-embedding ids[8,1024] W[{l.vocab},{l.hidden}] bf16 "
-                         f"tp{l.tp}")
+            self.name = WORKLOAD_NAMES["embed"]
             g = torch.Generator(device=dev)
             g.manual_seed(0)
             self.ids = torch.randint(0, l.vocab, (m.M,), generator=g, device=dev,
@@ -459,8 +413,7 @@ class NextRows:
             self.io_in, self.io_out = ["ids"], ["out"]
         elif kind == "seqpar":
             b, sq = m.batch, m.seq
-            self.name = (f"sequence-parallel rmsnorm-tp-mlp x[{b},{sq},{m.hidden}] bf16 "
-                         f"{m.hidden}->{m.inter}->{m.hidden} tp{m.tp}")
+            self.name = WORKLOAD_NAMES["seqpar"]
             self.x = C.mlp_x(m, dev)      # read as the rank-major [tp][b][s/tp][H] layout
             self.scale = C.mlp_scale(m, 0, dev)
             self.w1 = C.mlp_w1(m, 0, dev)
@@ -489,12 +442,7 @@ class NextRows:
             tp, b, sq, N, I = m.tp, m.batch, m.seq, m.hidden, m.inter
             M, kr = m.M, m.inter // m.tp
             rows = b * (sq // tp)
-            self.name = (f"tp-ranks rmsnorm-tp-mlp x[{b},{sq},{N}] bf16 {N}->{I}->{N} "
-                         f"gelu-erf, {tp} ranks in sequence on one GPU (peer-gather c_fc, "
-                         "peer-scatter c_proj, slot reduction)")
-            self.parallelism = (f"{tp} TP ranks emulated in sequence on one GPU: each rank's "
-                                "c_fc reads every rank's token slice, its c_proj writes into "
-                                "every rank's receive buffer, then every rank reduces its slots")
+            self.name = WORKLOAD_NAMES["tp_ranks"]
             self.xs = C.mlp_x(m, dev).view(b, tp, sq // tp, N).transpose(0, 1).contiguous()
             self.scale = C.mlp_scale(m, 0, dev)
             self.xn = torch.empty_like(self.xs)
@@ -566,36 +514,139 @@ class NextRows:
                      self.reduce_bytes, self.m.tp)]
         return []
 
-    def oracle_sample(self, rows=64):
-        import numpy as np
-        import oracle as O
-        f64 = lambda t: t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
-        m, l = self.m, self.l
-        if self.kind == "swiglu":
-            xs, w = f64(self.x[:rows]), f64(self.w)
-            return (lambda: O.swiglu_column_linear(xs, w, self.F, m.tp),
-                    2.0 * rows * m.hidden * 2 * self.F, f"{rows} token rows")
-        if self.kind == "tp_ranks":
-            rows = 128
-            tp = m.tp
-            xs = f64(self.xs.transpose(0, 1).reshape(m.M, m.hidden)[:rows])
-            w1, w2, sc = f64(self.w1), f64(C.mlp_w2(m, 0, self.xs.device)), f64(self.scale)
-            return (lambda: O.tp_mlp(xs, w1, w2, tp, m.act, scale=sc, centered=True, norm=True,
-                                     residual=True),
-                    4.0 * rows * m.hidden * m.inter, f"{rows} tokens through the block")
-        if self.kind == "embed":
-            sub = 16032
-            table = f64(self.table[:sub])
-            ids = (self.ids[:4096] % sub).cpu().numpy()
-            return (lambda: O.embedding_lookup(ids, table, l.tp),
-                    ids.size * l.hidden * 2 * 2 + ids.size * 4,
-                    f"{ids.size} ids over a {sub}-row slice of the table")
-        xs = f64(self.x[:rows])
-        w1, w2 = f64(self.w1), f64(C.mlp_w2(m, 0, self.x.device))
-        sc = f64(self.scale)
-        return (lambda: O.tp_mlp(xs, w1, w2, m.tp, m.act, scale=sc, centered=True, norm=True,
-                                 residual=True),
-                4.0 * rows * m.hidden * m.inter, f"{rows} tokens through the block")
+
+# ------------------------------------------------------------------ the oracle
+#
+# The CPU baseline and the reference arm time the fp64 oracle on a bounded
+# sample of a workload.  The sample's tensors are generated on the host by the
+# seeded generator (bit-identical to the device copies); nothing here imports
+# the library or touches CUDA.  Each job returns (run, work, description) with
+# work in FLOP (or bytes, for the embedding).
+
+def _f64(t):
+    import numpy as np
+    return t.to(torch.float32).numpy().astype(np.float64)
+
+
+def _sample_rows(M, n):
+    """n token rows spread evenly over [0, M)."""
+    return [int(i * M // n) for i in range(n)]
+
+
+def oracle_job_block(parts=("qkv", "mlp", "lmhead"), rows_qkv=256, rows_mlp=96,
+                     lm_rows=16032):
+    import oracle as O
+    q, m, l = C.GQA_QKV, C.TP_MLP, C.LM_HEAD
+    jobs, flops, desc = [], 0.0, []
+    if "qkv" in parts:
+        xq = _f64(gen.rows((q.M, q.hidden), _sample_rows(q.M, rows_qkv), 1.0,
+                           tensor_id=gen.TID_X))
+        wq, bq = _f64(C.qkv_w(q)), _f64(C.qkv_bias(q))
+        part = O.partition_subparams(list(q.sub_sizes), q.tp, q.align)
+        jobs.append(lambda: O.column_linear(xq, wq, bq, part))
+        flops += 2.0 * rows_qkv * q.hidden * q.out
+        desc.append(f"{rows_qkv} token rows of the fused QKV")
+    if "mlp" in parts:
+        xm = _f64(gen.rows((m.M, m.hidden), _sample_rows(m.M, rows_mlp), 1.0,
+                           tensor_id=gen.TID_X))
+        w1, w2, sc = _f64(C.mlp_w1(m)), _f64(C.mlp_w2(m)), _f64(C.mlp_scale(m))
+        jobs.append(lambda: O.tp_mlp(xm, w1, w2, m.tp, m.act, scale=sc, centered=True,
+                                     norm=True))
+        flops += 4.0 * rows_mlp * m.hidden * m.inter
+        desc.append(f"{rows_mlp} token rows of the RMSNorm+MLP")
+    if "lmhead" in parts:
+        xl = _f64(C.lm_x(l))
+        wl = _f64(gen.normal((lm_rows, l.hidden), l.w_sigma, tensor_id=gen.TID_W1))
+        jobs.append(lambda: O.lmhead_argmax(xl, wl, 1, 1))
+        flops += 2.0 * l.batch * l.hidden * lm_rows
+        desc.append(f"{lm_rows} vocab rows x {l.batch} batch rows of the LM head")
+
+    def run():
+        for j in jobs:
+            j()
+    return run, flops, ", ".join(desc)
+
+
+def oracle_job_stack(rows=8):
+    import oracle as O
+    w = C.STACK4
+    xs = _f64(gen.rows((w.M, w.hidden), _sample_rows(w.M, rows), 1.0, tensor_id=gen.TID_X))
+    layers = [(C.mlp_w1(w, i).to(torch.float32).numpy(),
+               C.mlp_w2(w, i).to(torch.float32).numpy()) for i in range(w.layers)]
+
+    def run():
+        # fp32 holds the bf16 weights exactly; each layer is widened to fp64 as it is used
+        x = xs
+        for w1, w2 in layers:
+            x = O.tp_mlp(x, w1.astype("float64"), w2.astype("float64"), w.tp, w.act,
+                         norm=True, residual=True)
+    return run, w.layers * 4.0 * rows * w.hidden * w.inter, \
+        f"{rows} token rows through all {w.layers} layers"
+
+
+def oracle_job_next(kind, rows=64):
+    import oracle as O
+    m, l = C.TP_MLP, C.LM_HEAD
+    if kind == "swiglu":
+        F = m.inter
+        xs = _f64(gen.rows((m.M, m.hidden), _sample_rows(m.M, rows), 1.0, tensor_id=gen.TID_X))
+        w = _f64(gen.normal((2 * F, m.hidden), m.w_sigma, tensor_id=gen.TID_W1))
+        return (lambda: O.swiglu_column_linear(xs, w, F, m.tp),
+                2.0 * rows * m.hidden * 2 * F, f"{rows} token rows")
+    if kind == "embed":
+        sub = 16032
+        table = _f64(gen.normal((sub, l.hidden), l.w_sigma, tensor_id=gen.TID_W1))
+        g = torch.Generator()
+        g.manual_seed(0)
+        ids = torch.randint(0, sub, (4096,), generator=g).numpy()
+        return (lambda: O.embedding_lookup(ids, table, l.tp),
+                ids.size * l.hidden * 2 * 2 + ids.size * 4,
+                f"{ids.size} ids over a {sub}-row slice of the table")
+    # seqpar / tp_ranks: the RMSNorm + MLP block with the residual, per token
+    rows = 128 if kind == "tp_ranks" else rows
+    xs = _f64(gen.rows((m.M, m.hidden), _sample_rows(m.M, rows), 1.0, tensor_id=gen.TID_X))
+    w1, w2, sc = _f64(C.mlp_w1(m)), _f64(C.mlp_w2(m)), _f64(C.mlp_scale(m))
+    return (lambda: O.tp_mlp(xs, w1, w2, m.tp, m.act, scale=sc, centered=True, norm=True,
+                             residual=True),
+            4.0 * rows * m.hidden * m.inter, f"{rows} tokens through the block")
+
+
+ORACLE_JOBS = {"block": oracle_job_block, "stack": oracle_job_stack,
+               "qkv": lambda: oracle_job_block(("qkv",)),
+               "mlp": lambda: oracle_job_block(("mlp",)),
+               "lmhead": lambda: oracle_job_block(("lmhead",)),
+               "swiglu": lambda: oracle_job_next("swiglu"),
+               "embed": lambda: oracle_job_next("embed"),
+               "seqpar": lambda: oracle_job_next("seqpar"),
+               "tp_ranks": lambda: oracle_job_next("tp_ranks")}
+
+# Workload names for the reference arm's line, without building the workload.
+WORKLOAD_NAMES = {
+    "block": "tp-block: " + " + ".join((C.GQA_QKV.name, C.TP_MLP.name, C.LM_HEAD.name)),
+    "stack": C.STACK4.name, "qkv": C.GQA_QKV.name, "mlp": C.TP_MLP.name,
+    "lmhead": C.LM_HEAD.name,
+    "swiglu": "fused-swiglu-column x[8,1024,4096] bf16 4096->2x14336 tp8",
+    "embed": "vocab-sharded-embedding ids[8,1024] W[128256,4096] bf16 tp8",
+    "seqpar": "sequence-parallel rmsnorm-tp-mlp x[8,1024,4096] bf16 4096->14336->4096 tp8",
+    "tp_ranks": "tp-ranks rmsnorm-tp-mlp x[8,1024,4096] bf16 4096->14336->4096 gelu-erf, 8 ranks "
+                "(peer-gather c_fc, peer-scatter c_proj, slot reduction)",
+}
+
+
+PARALLELISM = {
+    "tp_ranks": "8 TP ranks emulated in sequence on one GPU: each rank's c_fc reads every "
+                "rank's token slice, its c_proj writes into every rank's receive buffer, then "
+                "every rank reduces its slots"}
+L2_NOTE = ("not flushed: one step streams ~1.5 GB (block) / ~4 GB (stack), far above the "
+           "126 MB L2")
+
+
+def workload_config(kind, world):
+    """The ``config`` of a line: the same for both arms of one workload and N."""
+    par = PARALLELISM.get(kind, "tp shards of each linear computed on one GPU, cross-shard sum "
+                                "in the GEMM epilogue")
+    return {"workload": WORKLOAD_NAMES[kind], "parallelism": f"{world} replica(s); " + par,
+            "l2": L2_NOTE}
 
 
 WORKLOADS = {"block": Block, "stack": Stack,
@@ -652,30 +703,161 @@ def time_oracle(run, flops, target_s=15.0, max_reps=50):
     return flops * reps / dt / 1e12, reps, dt
 
 
-def run_reference(args, wl_cls, rank, world):
-    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+def oracle_rate(workload, work, seconds):
+    """(value, unit) of the oracle's work over the given time: TFLOP/s, or GB/s
+    for the bandwidth-only embedding."""
+    if workload == "embed":
+        return work / seconds / 1e9, "GB/s"
+    return work / seconds / 1e12, "TFLOP/s"
+
+
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle as the reference arm (rank 0 only).
+
+    Its inputs come from the host generator; it neither loads the library nor
+    initialises CUDA."""
     if rank != 0:
         return
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    wl = wl_cls(dev)
-    run, flops, desc = wl.oracle_sample()
+    run, work, desc = ORACLE_JOBS[args.workload]()
     for _ in range(max(1, args.warmup)):
         run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         run()
     dt = time.perf_counter() - t0
-    v = flops * args.steps / dt / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+    v, unit = oracle_rate(args.workload, work * args.steps, dt)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "parallelism": "oracle on host cores"},
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas_threads(),
+            "config": workload_config(args.workload, world),
+            "runs_on": "host cores: the fp64 oracle on a bounded sample of the workload",
+            "cpu_baseline": {"value": v, "unit": unit, "cores": blas_threads(),
                              "kind": "oracle", "sample": desc},
-            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def timed_steps(wl, stream, steps, pg, dev):
+    """Times ``steps`` steps of ``wl`` on ``stream`` with CUDA events (whole region
+    and per launch), sampling the SM clock meanwhile.  A run under a hardware or
+    thermal slowdown (or a stale clock lock) is taken again once; every rank
+    makes the same decision.  Returns (region ms, mean ms per part, library
+    launches in the region, clock record)."""
+    import tensor_transformer_linear_b200 as T
+    n_ev = len(wl.parts) + 1
+
+    def region():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+               for _ in range(steps)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(torch.cuda.current_device())
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        time.sleep(0.3)   # nvidia-smi is sampling before the timed steps start
+        n0 = T.tpl_launch_count()
+        t0 = datetime.datetime.now()
+        start.record(stream)
+        for k in range(steps):
+            wl.step(stream, evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        t1 = datetime.datetime.now()
+        launches = T.tpl_launch_count() - n0
+        clk = clocks.stop(t0, t1)
+        if pg is not None:
+            pg.barrier()
+        if T.tpl_get_device_status(stream) != 0:
+            raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
+        part_ms = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1])
+                                   for k in range(steps)) for i in range(n_ev - 1)]
+        return start.elapsed_time(stop), part_ms, launches, clk
+
+    ms, part_ms, launches, clk = region()
+    bad = torch.tensor([1.0 if clocks_rejected(clk) else 0.0], device=dev)
+    if pg is not None:
+        pg.all_reduce(bad, op=pg.ReduceOp.MAX)
+    remeasured = bool(bad.item() > 0)
+    if remeasured:
+        ms, part_ms, launches, clk = region()
+    if clk is not None:
+        clk["remeasured"] = remeasured
+    return ms, part_ms, launches, clk
+
+
+def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
+    """The 4-layer residual stack x[4,4096,8192] at full size, timed in the same
+    process: long enough (about a second) to run in the power-capped regime."""
+    wl = Stack(dev)
+    steps = max(20, min(args.steps, 40))
+    for _ in range(3):
+        wl.step(stream)
+    torch.cuda.synchronize()
+    ms, part_ms, launches, clk = timed_steps(wl, stream, steps, pg, dev)
+    if pg is not None:
+        ms = max_over_ranks([ms], dev)[0]
+        part_ms = max_over_ranks(part_ms, dev)
+    step_ms = ms / steps
+    gids = wl.gemm_part_ids()
+    gemm_ms = sum(part_ms[i] for i in gids)
+    achieved = wl.gemm_flops / (gemm_ms * 1e-3) / 1e12
+    peak_t, peak_label = tensor_peak(pk, pk_kind, clk)
+    norm_ms = sum(part_ms[i] for i in range(len(part_ms)) if i not in gids)
+    norm_bytes = wl.w.layers * 2 * 2 * wl.w.M * wl.w.hidden
+    rec = {
+        "workload": wl.name, "steps": steps, "warmup": 3, "ms_per_step": round(step_ms, 4),
+        "value": round(replica_rate(world, wl.flops, step_ms), 2), "unit": "TFLOP/s",
+        "flops_per_step": wl.flops,
+        "kernel": "gemm_bf16_tcgen05_pair", "bound": "tensor",
+        "gemm_launches_per_step": len(gids), "gemm_flops_per_launch": wl.flops / len(gids),
+        "gemm_ms_per_step": round(gemm_ms, 4), "achieved": round(achieved, 2),
+        "peak": peak_t, "peak_kind": peak_label, "frac": round(achieved / peak_t, 4),
+        "frac_of_burst": round(achieved / pk["bf16_tflops"], 4),
+        "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
+        "rmsnorm": {"kernel": "rmsnorm_cta", "bytes_per_step": norm_bytes,
+                    "ms_per_step": round(norm_ms, 4),
+                    "achieved_gbs": round(norm_bytes / (norm_ms * 1e-3) / 1e9, 1)},
+        "parts_ms": {n: round(v, 4) for n, v in zip(wl.parts, part_ms)},
+        "gpu_launches": int(launches), "clocks": clk,
+        "l2": "not flushed: one step streams ~4 GB of weights and activations, far above "
+              "the 126 MB L2",
+        "measured": "CUDA events around every launch on the launching stream, mean over "
+                    "the timed steps; the GEMM rate is the step's GEMM FLOPs over the sum "
+                    "of its GEMM launch times"}
+    del wl
+    torch.cuda.empty_cache()
+    return rec
+
+
+def measure_tiny(dev, stream, reps=200):
+    """The tiny fp32 TP MLP (x[2,16,256], 256->1024->256, tp 4, GELU tanh): the
+    latency of one block (c_fc + c_proj), median over ``reps`` timed launches."""
+    import tensor_transformer_linear_b200 as T
+    w = C.TINY_MLP
+    x = C.mlp_x(w, dev)
+    blk = T.TPMLP(C.mlp_w1(w, 0, dev), C.mlp_w2(w, 0, dev), w.tp, w.act, norm=False)
+    y = torch.empty((w.M, w.hidden), dtype=w.dtype, device=dev)
+    for _ in range(10):
+        blk(x, out=y, stream=stream)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for e0, e1 in evs:
+        e0.record(stream)
+        blk(x, out=y, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
+    us = statistics.median(t)
+    return {"workload": w.name, "dtype": "f32", "us_per_block": round(us, 2),
+            "p10_us": round(t[len(t) // 10], 2), "p90_us": round(t[9 * len(t) // 10], 2),
+            "launches_per_block": 2, "flops_per_block": w.flops(),
+            "gflops": round(w.flops() / (us * 1e-6) / 1e9, 1), "bound": "latency",
+            "measured": f"median of {reps} blocks, CUDA events around each block "
+                        "(c_fc + GELU, c_proj + reduce) on the launching stream"}
 
 
 def main():
@@ -686,6 +868,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="block", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="block workload: skip the 4-layer stack and tiny-MLP records")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -696,7 +880,7 @@ def main():
     wl_cls = WORKLOADS[args.workload]
 
     if args.impl == "reference":
-        run_reference(args, wl_cls, rank, world)
+        run_reference(args, rank, world)
         return
 
     torch.cuda.set_device(local)
@@ -713,7 +897,6 @@ def main():
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
-    n_ev = len(wl.parts) + 1
     for _ in range(args.warmup):
         with torch.cuda.stream(stream):
             wl.step(stream)
@@ -722,45 +905,7 @@ def main():
         raise RuntimeError("a kernel reported a pipeline timeout during warm-up")
 
     # ---- device-timed region: K steps, per-launch events on the launching stream
-    def timed_region():
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-               for _ in range(args.steps)]
-        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        clocks = ClockSampler(torch.cuda.current_device())
-        if pg is not None:
-            pg.barrier()
-        torch.cuda.synchronize()
-        clocks.start()
-        time.sleep(0.3)   # nvidia-smi is sampling before the timed steps start
-        n0 = T.tpl_launch_count()
-        t0 = datetime.datetime.now()
-        start.record(stream)
-        for k in range(args.steps):
-            wl.step(stream, evs[k])
-        stop.record(stream)
-        torch.cuda.synchronize()
-        t1 = datetime.datetime.now()
-        launches = T.tpl_launch_count() - n0
-        clk = clocks.stop(t0, t1)
-        if pg is not None:
-            pg.barrier()
-        if T.tpl_get_device_status(stream) != 0:
-            raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
-        part_ms = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1])
-                                   for k in range(args.steps)) for i in range(n_ev - 1)]
-        return start.elapsed_time(stop), part_ms, launches, clk
-
-    ms, part_ms, launches, clk = timed_region()
-    # A run under a hardware or thermal slowdown (or a stale clock lock) is taken
-    # again once; every rank makes the same decision.
-    bad = torch.tensor([1.0 if clocks_rejected(clk) else 0.0], device=dev)
-    if pg is not None:
-        dist.all_reduce(bad, op=dist.ReduceOp.MAX)
-    remeasured = bool(bad.item() > 0)
-    if remeasured:
-        ms, part_ms, launches, clk = timed_region()
-    if clk is not None:
-        clk["remeasured"] = remeasured
+    ms, part_ms, launches, clk = timed_steps(wl, stream, args.steps, pg, dev)
 
     # ---- the LM head in a decode loop: back-to-back launches, as once per decode step
     decode_ms = None
@@ -825,6 +970,17 @@ def main():
     if pg is not None:
         ms, e_ms = max_over_ranks([ms, e_ms], dev)
 
+    # ---- the other single-GPU configurations, in the same process: the 4-layer
+    # stack (the largest, seconds-long, power-capped) and the tiny fp32 MLP (latency)
+    extra = {}
+    if args.workload == "block" and not args.no_extra:
+        pk, pk_kind = peaks()
+        extra["roofline_stack"] = measure_stack(args, dev, stream, pg, world, pk, pk_kind)
+        extra["tiny_mlp_us"] = measure_tiny(dev, stream)
+        if pg is not None:
+            extra["tiny_mlp_us"]["us_per_block"] = max_over_ranks(
+                [extra["tiny_mlp_us"]["us_per_block"]], dev)[0]
+
     if rank == 0:
         pk, pk_kind = peaks()
         step_ms = ms / args.steps
@@ -844,12 +1000,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded SplitMix64 / Irwin-Hall normal, the pages' shapes)",
-            "config": {"workload": wl.name,
-                       "parallelism": f"{world} replica(s); " + getattr(
-                           wl, "parallelism", "tp shards of each linear computed on one GPU, "
-                                              "cross-shard sum in the GEMM epilogue"),
-                       "l2": "not flushed: one step streams ~1.5 GB (block) / ~4 GB (stack), "
-                             "far above the 126 MB L2"},
+            "config": workload_config(args.workload, world),
             "roofline": {"kernel": "gemm_bf16_tcgen05_pair", "bound": "tensor",
                          "achieved": round(gemm_achieved, 2), "peak": peak_t,
                          "unit": "TFLOP/s", "frac": round(gemm_achieved / peak_t, 4),
@@ -916,11 +1067,13 @@ def main():
             line["e2e"]["value"] = round(wl.hbm_bytes / (e_ms / e_steps * 1e-3) / 1e9 * world, 1)
             line["e2e"]["unit"] = "GB/s"
         if world == 1 and not args.no_cpu_baseline:
-            run, flops, desc = wl.oracle_sample()
-            v, reps, dt = time_oracle(run, flops)
-            line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s",
+            run, work, desc = ORACLE_JOBS[args.workload]()
+            _, reps, dt = time_oracle(run, work)
+            v, unit = oracle_rate(args.workload, work * reps, dt)
+            line["cpu_baseline"] = {"value": round(v, 6), "unit": unit,
                                     "cores": blas_threads(), "kind": "oracle",
                                     "sample": f"{desc}; {reps} reps in {dt:.1f} s"}
+        line.update(extra)
         print(json.dumps(line), flush=True)
 
     if pg is not None:

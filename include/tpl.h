@@ -287,7 +287,12 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
  *     TPL_LMHEAD_STATIC_SCRATCH_BYTES are rejected with TPL_ERR_SHAPE.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture on the device.
+ *     before any stream capture on the device.  The address is kept for the
+ *     device's CUDA context: after cudaDeviceReset the next call looks it up
+ *     again in the new context (so again outside any stream capture), and
+ *     the array starts over at zero.
+ *   - Every check of tpl_lmhead_argmax runs before anything is enqueued: a
+ *     rejected call enqueues nothing, not even the clear below.
  *   - Every call on a device shares the one array and clears the part it uses
  *     (cudaMemsetAsync on `stream`) before the kernel.  Calls whose work
  *     overlaps on the GPU (different streams, or different host threads)

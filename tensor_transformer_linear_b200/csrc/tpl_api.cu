@@ -641,12 +641,19 @@ tpl_status tpl_lmhead_workspace_size(int64_t B, int64_t V, int32_t tp, int32_t n
   return TPL_OK;
 }
 
-tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
-                             int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
-                             int32_t* shard_idx, int32_t* ids, void* workspace, size_t ws_bytes,
-                             void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Every check of an LM-head call and the kernel's arguments (tensor maps
+// included), with nothing enqueued; `scratch` is the keys + counter area of
+// `ws_bytes` bytes (the caller's workspace or the library's fixed array).
+tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
+                          int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
+                          int32_t* shard_idx, int32_t* ids, void* scratch, size_t ws_bytes,
+                          tpl::LmArgs* a, int* smem, int* grid) {
   if (x == nullptr || w == nullptr || shard_max == nullptr || shard_idx == nullptr ||
-      ids == nullptr || workspace == nullptr)
+      ids == nullptr || scratch == nullptr)
     return TPL_ERR_NULL;
   int64_t shard = 0;
   tpl_status s = lm_layout(B, V, tp, n_chunks, &shard);
@@ -655,62 +662,81 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
   size_t need = 0;
   tpl_lmhead_workspace_size(B, V, tp, n_chunks, &need);
   if (ws_bytes < need) return TPL_ERR_SHAPE;
-  if (K % 8 != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(workspace, 16) ||
+  if (K % 8 != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(scratch, 16) ||
       (logits && !aligned(logits, 4)) || !aligned(shard_max, 4) || !aligned(shard_idx, 4) ||
       !aligned(ids, 4))
     return TPL_ERR_ALIGN;
   DeviceInfo* dev = nullptr;
   if ((s = device_info(&dev)) != TPL_OK) return s;
 
-  tpl::LmArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.B = static_cast<int32_t>(B);
-  a.Npad = static_cast<int32_t>((B + 15) / 16 * 16);
+  std::memset(a, 0, sizeof(*a));
+  a->B = static_cast<int32_t>(B);
+  a->Npad = static_cast<int32_t>((B + 15) / 16 * 16);
   // Slab height: the fewest rounds of at most 128-row slabs over the SMs, then
   // the shortest slab that still covers V in that many rounds, so every CTA
   // streams (nearly) the same number of rows.
   {
     const int64_t sms = dev->sm_count;
     const int64_t rounds = (V + sms * tpl::kLmRows - 1) / (sms * tpl::kLmRows);
-    a.slab_rows = static_cast<int32_t>((V + sms * rounds - 1) / (sms * rounds));
+    a->slab_rows = static_cast<int32_t>((V + sms * rounds - 1) / (sms * rounds));
   }
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(V)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
-    if ((s = encode_bf16(&a.tmW, w, 2, dims, str, static_cast<uint32_t>(a.slab_rows))) != TPL_OK)
+    if ((s = encode_bf16(&a->tmW, w, 2, dims, str, static_cast<uint32_t>(a->slab_rows))) !=
+        TPL_OK)
       return s;
   }
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(B)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
-    if ((s = encode_bf16(&a.tmX, x, 2, dims, str, static_cast<uint32_t>(a.Npad))) != TPL_OK)
+    if ((s = encode_bf16(&a->tmX, x, 2, dims, str, static_cast<uint32_t>(a->Npad))) != TPL_OK)
       return s;
   }
-  a.K = static_cast<int32_t>(K);
-  a.k_iters = static_cast<int32_t>((K + tpl::kLmBK - 1) / tpl::kLmBK);
-  a.V = static_cast<int32_t>(V);
-  a.tp = tp;
-  a.shard = static_cast<int32_t>(shard);
-  a.n_slabs = static_cast<int32_t>((V + a.slab_rows - 1) / a.slab_rows);
-  a.stage_bytes = tpl::kLmABytes + a.Npad * tpl::kLmBK * 2;
+  a->K = static_cast<int32_t>(K);
+  a->k_iters = static_cast<int32_t>((K + tpl::kLmBK - 1) / tpl::kLmBK);
+  a->V = static_cast<int32_t>(V);
+  a->tp = tp;
+  a->shard = static_cast<int32_t>(shard);
+  a->n_slabs = static_cast<int32_t>((V + a->slab_rows - 1) / a->slab_rows);
+  a->stage_bytes = tpl::kLmABytes + a->Npad * tpl::kLmBK * 2;
   const int budget = 227 * 1024 - 1024 - 256 - tpl::kLmTbufBytes;
-  a.stages = std::min(tpl::kLmMaxStages, budget / a.stage_bytes);
-  if (a.stages < 2) return TPL_ERR_UNSUPPORTED;
+  a->stages = std::min(tpl::kLmMaxStages, budget / a->stage_bytes);
+  if (a->stages < 2) return TPL_ERR_UNSUPPORTED;
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(2 * a.Npad)) cols <<= 1;
-  a.tmem_cols = cols;
-  a.logits = logits;
-  a.shard_max = shard_max;
-  a.shard_idx = shard_idx;
-  a.ids = ids;
-  a.keys = static_cast<unsigned long long*>(workspace);
-  a.counter = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
-                                              static_cast<size_t>(tp) * B * 8);
-  const int smem = a.stages * a.stage_bytes + 1024 + 256 + tpl::kLmTbufBytes;
-  const int grid = std::min(a.n_slabs, dev->sm_count);
-  tpl::lmhead_argmax_tcgen05<<<grid, tpl::kLmThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-      a);
+  while (cols < static_cast<uint32_t>(2 * a->Npad)) cols <<= 1;
+  a->tmem_cols = cols;
+  a->logits = logits;
+  a->shard_max = shard_max;
+  a->shard_idx = shard_idx;
+  a->ids = ids;
+  a->keys = static_cast<unsigned long long*>(scratch);
+  a->counter = reinterpret_cast<unsigned int*>(static_cast<char*>(scratch) +
+                                               static_cast<size_t>(tp) * B * 8);
+  *smem = a->stages * a->stage_bytes + 1024 + 256 + tpl::kLmTbufBytes;
+  *grid = std::min(a->n_slabs, dev->sm_count);
+  return TPL_OK;
+}
+
+tpl_status lmhead_launch(const tpl::LmArgs& a, int smem, int grid, cudaStream_t st) {
+  tpl::lmhead_argmax_tcgen05<<<grid, tpl::kLmThreads, smem, st>>>(a);
   return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
+                             int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
+                             int32_t* shard_idx, int32_t* ids, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  tpl::LmArgs a;
+  int smem = 0, grid = 0;
+  tpl_status s = lmhead_prepare(x, B, K, w, V, tp, n_chunks, logits, shard_max, shard_idx, ids,
+                                workspace, ws_bytes, &a, &smem, &grid);
+  if (s != TPL_OK) return s;
+  return lmhead_launch(a, smem, grid, static_cast<cudaStream_t>(stream));
 }
 
 tpl_status tpl_get_device_status(void* stream) {
@@ -743,19 +769,51 @@ namespace {
 
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];
 
-// Device address of g_lmhead_scratch on the current device, looked up once per
-// device.  In host code the array's name is only a host-side stand-in, so the
-// kernel must be given this address instead.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id (never reused within the process) of the CUDA context current on
+// this thread; false if there is none yet.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr)
+    return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_lmhead_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the kernel must be given this
+// address instead.  It is looked up once per device and looked up again when
+// the device's context has changed since (after cudaDeviceReset, the next
+// call maps the array in the new context).
 tpl_status lmhead_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TPL_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (g_scratch_addr[dev] == nullptr || !have_ctx || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_lmhead_scratch) != cudaSuccess || p == nullptr)
       return TPL_ERR_CUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id(&ctx) ? ctx : 0ull;
   }
   *out = g_scratch_addr[dev];
   return TPL_OK;
@@ -767,8 +825,6 @@ extern "C" tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t
                                                int64_t V, int32_t tp, int32_t n_chunks,
                                                float* logits, float* shard_max,
                                                int32_t* shard_idx, int32_t* ids, void* stream) {
-  // The checks tpl_lmhead_argmax makes, repeated here so that a rejected call
-  // enqueues nothing (not even the scratch clear).
   if (x == nullptr || w == nullptr || shard_max == nullptr || shard_idx == nullptr ||
       ids == nullptr)
     return TPL_ERR_NULL;
@@ -776,17 +832,19 @@ extern "C" tpl_status tpl_lmhead_argmax_static(const void* x, int64_t B, int64_t
   tpl_status s = tpl_lmhead_workspace_size(B, V, tp, n_chunks, &need);
   if (s != TPL_OK) return s;
   if (need > static_cast<size_t>(TPL_LMHEAD_STATIC_SCRATCH_BYTES)) return TPL_ERR_SHAPE;
-  if (K < 1 || K > INT32_MAX) return TPL_ERR_SHAPE;
-  if (K % 8 != 0 || !aligned(x, 16) || !aligned(w, 16) || (logits && !aligned(logits, 4)) ||
-      !aligned(shard_max, 4) || !aligned(shard_idx, 4) || !aligned(ids, 4))
-    return TPL_ERR_ALIGN;
   void* scratch = nullptr;
   if ((s = lmhead_scratch_address(&scratch)) != TPL_OK) return s;
+  // Every check of tpl_lmhead_argmax, and the kernel's arguments, before
+  // anything is enqueued: a rejected call enqueues nothing, not even the clear.
+  tpl::LmArgs a;
+  int smem = 0, grid = 0;
+  s = lmhead_prepare(x, B, K, w, V, tp, n_chunks, logits, shard_max, shard_idx, ids, scratch,
+                     static_cast<size_t>(TPL_LMHEAD_STATIC_SCRATCH_BYTES), &a, &smem, &grid);
+  if (s != TPL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   // The array keeps the previous call's contents: start this call from zero.
-  if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return TPL_ERR_CUDA;
-  return tpl_lmhead_argmax(x, B, K, w, V, tp, n_chunks, logits, shard_max, shard_idx, ids, scratch,
-                           static_cast<size_t>(TPL_LMHEAD_STATIC_SCRATCH_BYTES), stream);
+  if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return TPL_ERR_CUDA;
+  return lmhead_launch(a, smem, grid, st);
 }
 
 // Entry points of the next rows (same translation unit).

@@ -12,10 +12,11 @@ from typing import Callable, List, Optional, Sequence
 
 import torch
 
-from ._tpl import (Partition, tpl_argmax_merge, tpl_column_linear, tpl_column_linear_gather,
-                   tpl_lmhead_argmax, tpl_lmhead_workspace_size, tpl_partition_subparams,
-                   tpl_reduce_slots, tpl_reduce_slots_allgather, tpl_rmsnorm,
-                   tpl_row_linear_reduce, tpl_row_linear_scatter)
+from ._tpl import (Partition, TplError, tpl_argmax_merge, tpl_column_linear,
+                   tpl_column_linear_gather, tpl_get_device_status, tpl_lmhead_argmax,
+                   tpl_lmhead_workspace_size, tpl_partition_subparams, tpl_reduce_slots,
+                   tpl_reduce_slots_allgather, tpl_rmsnorm, tpl_row_linear_reduce,
+                   tpl_row_linear_scatter)
 
 
 def shard_views(y: torch.Tensor, p: Partition, M: int) -> List[torch.Tensor]:
@@ -337,6 +338,7 @@ class TPLMHeadRank:
                  merge: Optional[Callable] = None):
         self.w = w_slice.contiguous()
         self.rank, self.tp, self.shard, self.group = rank, tp, shard, group
+        self._own_argmax = local_argmax is None
         self.local_argmax = local_argmax or self._local_argmax
         self.gather = gather or self._gather
         self.merge = merge or (lambda m, i, stride, stream=None:
@@ -363,7 +365,20 @@ class TPLMHeadRank:
             return torch.stack(parts)
 
     def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
-        """``x`` ``[B, K]`` (the same on every rank).  Returns global ids ``[B]``."""
+        """``x`` ``[B, K]`` (the same on every rank).  Returns global ids ``[B]``.
+
+        With the library's local argmax, the call ends by reading the device
+        status (which waits for the stream: a decode step needs its ids on the
+        host anyway).  A kernel that gave up waiting leaves its workspace
+        stale, so the workspace is cleared and the call raises TplError; the
+        next call starts clean."""
         m, i = self.local_argmax(x, stream=stream)
-        return self.merge(self.gather(m, stream=stream), self.gather(i, stream=stream),
-                          self.shard, stream=stream)
+        ids = self.merge(self.gather(m, stream=stream), self.gather(i, stream=stream),
+                         self.shard, stream=stream)
+        if self._own_argmax:
+            code = tpl_get_device_status(stream)
+            if code != 0:
+                if self._ws is not None:
+                    self._ws.zero_()
+                raise TplError(code, "TPLMHeadRank")
+        return ids

@@ -71,3 +71,28 @@ def test_gemm_peak_follows_the_clock_regime():
     assert "sustained" in bench.tensor_peak(pk, "measured", capped)[1]
     assert bench.tensor_peak(pk, "measured", full) == (1659.1, "measured bf16 burst")
     assert bench.tensor_peak(pk, "fallback", None) == (1659.1, "fallback bf16 burst")
+
+
+def test_reference_arm_runs_the_oracle_alone():
+    """``--impl reference`` builds its sample on the host and runs only the
+    oracle: the library is never imported, CUDA never initialised, and its
+    ``config`` is the one the library's line prints for the same workload."""
+    import json
+    import subprocess
+    code = (
+        "import sys, runpy, json\n"
+        "sys.argv = ['bench.py', '--impl', 'reference', '--workload', 'qkv',\n"
+        "            '--steps', '1', '--warmup', '1']\n"
+        "runpy.run_path('bench.py', run_name='__main__')\n"
+        "import torch\n"
+        "mods = [m for m in sys.modules if m.startswith('tensor_transformer_linear_b200')]\n"
+        "print(json.dumps({'mods': mods, 'cuda': torch.cuda.is_initialized()}))\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    line, probe = lines[0], lines[-1]
+    assert probe == {"mods": [], "cuda": False}
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"] == bench.workload_config("qkv", 1)
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"

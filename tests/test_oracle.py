@@ -129,6 +129,17 @@ def test_gelu_erf_textbook_phi():
         assert O.gelu_erf(np.array([y]))[0] == pytest.approx(y * phi, rel=1e-14, abs=1e-16)
 
 
+def test_gelu_tanh_worked_values():
+    # 40-digit values of the published tanh form, written by
+    # tests/golden/make_gelu_tanh.py with the standard library's decimal module
+    # only (a wrong cubic coefficient such as 0.0447 moves y = 1 by ~3e-6)
+    rows = _golden_rows("gelu_tanh.txt")
+    assert len(rows) == 8
+    for y, v in rows:
+        y, v = float(y), float(v)
+        assert abs(O.gelu_tanh(np.array([y]))[0] - v) <= 1e-13 * abs(v) + 1e-16, y
+
+
 def test_gelu_identities():
     y = np.linspace(-7.0, 7.0, 2801)
     for f in (O.gelu_erf, O.gelu_tanh):
