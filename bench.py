@@ -834,30 +834,48 @@ def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
 
 def measure_tiny(dev, stream, reps=200):
     """The tiny fp32 TP MLP (x[2,16,256], 256->1024->256, tp 4, GELU tanh): the
-    latency of one block (c_fc + c_proj), median over ``reps`` timed launches."""
+    latency of one block (c_fc + c_proj).  Median over ``reps`` blocks, each
+    bracketed by CUDA events, two ways: replays of the block captured once in a
+    CUDA graph (device latency: the two kernels back to back, no host work in
+    between) and eager calls through the Python binding (each launch also waits
+    for its host-side argument marshalling)."""
     import tensor_transformer_linear_b200 as T
     w = C.TINY_MLP
     x = C.mlp_x(w, dev)
     blk = T.TPMLP(C.mlp_w1(w, 0, dev), C.mlp_w2(w, 0, dev), w.tp, w.act, norm=False)
     y = torch.empty((w.M, w.hidden), dtype=w.dtype, device=dev)
-    for _ in range(10):
-        blk(x, out=y, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(10):
+            blk(x, out=y)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(reps)]
-    for e0, e1 in evs:
-        e0.record(stream)
-        blk(x, out=y, stream=stream)
-        e1.record(stream)
+
+    def timed(run):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for e0, e1 in evs:
+                e0.record(stream)
+                run()
+                e1.record(stream)
+        torch.cuda.synchronize()
+        return sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        blk(x, out=y)
     torch.cuda.synchronize()
-    t = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
-    us = statistics.median(t)
+    tg = timed(graph.replay)
+    te = timed(lambda: blk(x, out=y))
+    del graph
+    us = statistics.median(tg)
     return {"workload": w.name, "dtype": "f32", "us_per_block": round(us, 2),
-            "p10_us": round(t[len(t) // 10], 2), "p90_us": round(t[9 * len(t) // 10], 2),
-            "launches_per_block": 2, "flops_per_block": w.flops(),
+            "p10_us": round(tg[len(tg) // 10], 2), "p90_us": round(tg[9 * len(tg) // 10], 2),
+            "eager_us_per_block": round(statistics.median(te), 2),
+            "launches_per_block": 2, "kernel": "gemm_fp32_simt", "flops_per_block": w.flops(),
             "gflops": round(w.flops() / (us * 1e-6) / 1e9, 1), "bound": "latency",
-            "measured": f"median of {reps} blocks, CUDA events around each block "
-                        "(c_fc + GELU, c_proj + reduce) on the launching stream"}
+            "measured": f"median of {reps} blocks, CUDA events around each block on the "
+                        "launching stream; us_per_block replays the block captured in a CUDA "
+                        "graph, eager_us_per_block calls it through the Python binding"}
 
 
 def main():

@@ -77,6 +77,10 @@ struct GemmArgs {
   int32_t m_blocks, n_tiles, num_tiles, group_m;
   int32_t n_halves;
   int32_t vec_store;  // every output row start is 16-byte aligned
+  // K order of a tile: with k_serp set, a CTA pair walks K backwards on its
+  // odd tiles, so a tile wave starts on the K slices the wave before it read
+  // last (still in L2) when the two waves share operand blocks.
+  int32_t k_serp;
   int32_t n_pieces;
   ColPiece pieces[kMaxPieces];
   const __nv_bfloat16* bias;

@@ -87,7 +87,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = pair; ok && t < a.num_tiles; t += npairs) {
+      int it = 0;
+      for (int t = pair; ok && t < a.num_tiles; t += npairs, ++it) {
         int mb, nt;
         tile_coords(a, t, mb, nt);
         const bool has1 = 2 * nt + 1 < a.n_halves;
@@ -96,8 +97,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int m_row = mb * kPairBM + static_cast<int>(rank) * kBM;
         int arow;
         const CUtensorMap* mAcol = a_source(a, m_row, arow);
-        int rr = a.r0, kb = 0;  // row mode: rank and K block of the next step
-        for (int ki = 0; ki < k_total; ++ki) {
+        const bool rev = a.k_serp && (it & 1);
+        // row mode: rank and K block of the next step (walking backwards when rev)
+        int rr = rev ? a.r1 - 1 : a.r0;
+        int kb = rev ? (rr >= a.r_split ? a.k_iters2 : a.k_iters) - 1 : 0;
+        for (int kstep = 0; kstep < k_total; ++kstep) {
+          const int ki = rev ? k_total - 1 - kstep : kstep;
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -117,9 +122,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const int rc = g2 ? rr - a.r_split : rr;
             ptx::tma_load_3d_pair(sA, mA, bar, kb * kBK, m_row, rc);
             ptx::tma_load_3d_pair(sB, mB, bar, kb * kBK, h.brow, rc);
-            if (++kb == (g2 ? a.k_iters2 : a.k_iters)) {
-              kb = 0;
-              ++rr;
+            if (!rev) {
+              if (++kb == (g2 ? a.k_iters2 : a.k_iters)) {
+                kb = 0;
+                ++rr;
+              }
+            } else if (--kb < 0) {
+              --rr;
+              kb = (rr >= a.r_split ? a.k_iters2 : a.k_iters) - 1;
             }
           }
           if (++stage == kPairStages) {

@@ -15,6 +15,7 @@ import oracle as O
 import tensor_transformer_linear_b200 as T
 from workloads import gen
 
+from . import _bounds as Bd
 from ._parity import TOL_BF16, TOL_FP32, check_ids, check_shard_ids, f64, rel
 
 pytestmark = pytest.mark.gpu
@@ -52,15 +53,18 @@ def test_rmsnorm(dtype, M, H, mode):
     s = _t((H,), 0.1, 4, torch.float32) if mode != "none" else None
     y = T.tpl_rmsnorm(x.to(DEV), s.to(DEV) if s is not None else None, mode == "centered")
     torch.cuda.synchronize()
-    ref = O.rmsnorm(f64(x), None if s is None else f64(s), mode == "centered", 1e-6)
-    assert rel(y, ref) <= (TOL_BF16 if dtype == torch.bfloat16 else TOL_FP32)
+    ref, own = Bd.rmsnorm(f64(x), None if s is None else f64(s), mode == "centered", 1e-6)
+    bf16 = dtype == torch.bfloat16
+    assert rel(y, ref) <= (TOL_BF16 if bf16 else TOL_FP32)
+    Bd.check(f64(y), ref, own, u_out=Bd.U_BF16 if bf16 else Bd.U_FP32)
 
 
 def test_rmsnorm_in_place_and_empty():
     x = _t((64, 4096), 1.0, 0).to(DEV)
-    ref = O.rmsnorm(f64(x))
+    ref, own = Bd.rmsnorm(f64(x))
     T.tpl_rmsnorm(x, None, False, 1e-6, y=x)
     assert rel(x, ref) <= TOL_BF16
+    Bd.check(f64(x), ref, own)
     e = torch.empty((0, 4096), dtype=torch.bfloat16, device=DEV)
     T.tpl_rmsnorm(e)
 
@@ -89,13 +93,14 @@ def test_column_linear_bf16(case):
     p = T.tpl_partition_subparams(subs, tp, align)
     y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), b.to(DEV) if b is not None else None, act)
     torch.cuda.synchronize()
-    ref = O.column_linear(f64(x), f64(w), None if b is None else f64(b), part, act)
+    ref, own, _ = Bd.column(f64(x), f64(w), None if b is None else f64(b), part, act)
     got = [f64(v) for v in T.shard_views(y, p, M)]
     err = O.rel_frobenius(np.concatenate([g.ravel() for g in got]),
                           np.concatenate([r.ravel() for r in ref]))
     assert err <= TOL_BF16, err
-    for g, r in zip(got, ref):
+    for r_, (g, r, e) in enumerate(zip(got, ref, own)):
         assert O.rel_frobenius(g, r) <= TOL_BF16
+        Bd.check(g, r, e, what=f"rank {r_}")
 
 
 def test_column_linear_fp32_tiny_mlp_shapes():
@@ -105,9 +110,10 @@ def test_column_linear_fp32_tiny_mlp_shapes():
     p = T.tpl_partition_subparams([1024], 4, 1)
     y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), None, "gelu_tanh")
     torch.cuda.synchronize()
-    ref = O.column_linear(f64(x), f64(w), None, part, "gelu_tanh")
-    for g, r in zip(T.shard_views(y, p, 32), ref):
+    ref, own, _ = Bd.column(f64(x), f64(w), None, part, "gelu_tanh", simt=True)
+    for g, r, e in zip(T.shard_views(y, p, 32), ref, own):
         assert rel(g, r) <= TOL_FP32
+        Bd.check(f64(g), r, e, u_out=Bd.U_FP32)
 
 
 def test_column_linear_fp32_ragged_with_bias():
@@ -119,9 +125,10 @@ def test_column_linear_fp32_ragged_with_bias():
     p = T.tpl_partition_subparams(subs, tp, 10)
     y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), b.to(DEV), "gelu_erf")
     torch.cuda.synchronize()
-    ref = O.column_linear(f64(x), f64(w), f64(b), part, "gelu_erf")
-    for g, r in zip(T.shard_views(y, p, 67), ref):
+    ref, own, _ = Bd.column(f64(x), f64(w), f64(b), part, "gelu_erf", simt=True)
+    for g, r, e in zip(T.shard_views(y, p, 67), ref, own):
         assert rel(g, r) <= TOL_FP32
+        Bd.check(f64(g), r, e, u_out=Bd.U_FP32)
 
 
 def test_column_linear_many_pieces_two_launches():
@@ -134,9 +141,10 @@ def test_column_linear_many_pieces_two_launches():
     p = T.tpl_partition_subparams(subs, tp, 8)
     y = T.tpl_column_linear(p, x.to(DEV), w.to(DEV), b.to(DEV), "none")
     torch.cuda.synchronize()
-    ref = O.column_linear(f64(x), f64(w), f64(b), part)
-    for g, r in zip(T.shard_views(y, p, 150), ref):
+    ref, own, _ = Bd.column(f64(x), f64(w), f64(b), part)
+    for g, r, e in zip(T.shard_views(y, p, 150), ref, own):
         assert rel(g, r) <= TOL_BF16
+        Bd.check(f64(g), r, e)
 
 
 def test_column_linear_empty_rows():
@@ -177,12 +185,14 @@ def test_row_linear_reduce_bf16(case):
     torch.cuda.synchronize()
     hs = O.row_weight_slices(f64(h), k_w)
     ws = O.row_weight_slices(f64(w2), k_w)
-    ref = O.row_linear_reduce(hs, ws, None if b is None else f64(b), None if res is None else f64(res))
+    ref, own, _ = Bd.row(hs, ws, None if b is None else f64(b), None if res is None else f64(res))
     assert rel(y, ref) <= TOL_BF16
-    pref = O.row_partials(hs, ws)
+    Bd.check(f64(y), ref, own)
+    pref, pown = Bd.partials(hs, ws)
     pg = f64(parts).reshape(tp, M, N)
     for r in range(tp):
         assert O.rel_frobenius(pg[r], pref[r]) <= 1e-5   # fp32 partials of bf16 inputs
+        Bd.check(pg[r], pref[r], pown[r], u_out=Bd.U_FP32, what=f"partial {r}")
 
 
 def test_row_linear_residual_aliases_output():
@@ -195,9 +205,10 @@ def test_row_linear_residual_aliases_output():
     T.tpl_row_linear_reduce(T.pack_row_weight(h, k_w).to(DEV), k_w, M,
                             T.pack_row_weight(w2, k_w).to(DEV), None, xd, y=xd)
     torch.cuda.synchronize()
-    ref = O.row_linear_reduce(O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w),
-                              None, f64(x))
+    ref, own, _ = Bd.row(O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w),
+                         None, f64(x))
     assert rel(xd, ref) <= TOL_BF16
+    Bd.check(f64(xd), ref, own)
 
 
 def test_row_linear_fp32_uneven_ranks():
@@ -213,10 +224,14 @@ def test_row_linear_fp32_uneven_ranks():
                                 partials=parts)
     torch.cuda.synchronize()
     hs, ws = O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w)
-    assert rel(y, O.row_linear_reduce(hs, ws, f64(b), f64(res))) <= TOL_FP32
+    ref, own, _ = Bd.row(hs, ws, f64(b), f64(res), simt=True)
+    assert rel(y, ref) <= TOL_FP32
+    Bd.check(f64(y), ref, own, u_out=Bd.U_FP32)
     pg = f64(parts).reshape(4, M, N)
-    for r, pr in enumerate(O.row_partials(hs, ws)):
+    pref, pown = Bd.partials(hs, ws, simt=True)
+    for r, pr in enumerate(pref):
         assert O.rel_frobenius(pg[r], pr) <= TOL_FP32
+        Bd.check(pg[r], pr, pown[r], u_out=Bd.U_FP32)
 
 
 @pytest.mark.parametrize("k_w,M,N", [([16, 16, 8], 200, 136), ([72, 64, 64, 64], 300, 256),
@@ -231,10 +246,14 @@ def test_row_linear_bf16_two_rank_widths(k_w, M, N):
                                 T.pack_row_weight(w2, k_w).to(DEV), partials=parts)
     torch.cuda.synchronize()
     hs, ws = O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w)
-    assert rel(y, O.row_linear_reduce(hs, ws)) <= TOL_BF16
+    ref, own, _ = Bd.row(hs, ws)
+    assert rel(y, ref) <= TOL_BF16
+    Bd.check(f64(y), ref, own)
     pg = f64(parts).reshape(tp, M, N)
-    for r, pr in enumerate(O.row_partials(hs, ws)):
+    pref, pown = Bd.partials(hs, ws)
+    for r, pr in enumerate(pref):
         assert O.rel_frobenius(pg[r], pr) <= 1e-5
+        Bd.check(pg[r], pr, pown[r], u_out=Bd.U_FP32)
 
 
 def test_row_linear_bf16_three_rank_widths_rejected():
@@ -260,6 +279,8 @@ def test_tp_mlp_uneven_partition_end_to_end():
                               O.row_weight_slices(f64(w2), part.shard_width))
     assert part.shard_width == [336, 336, 328]
     assert rel(y, ref) <= TOL_BF16
+    bref, own, car = Bd.mlp(f64(x), f64(w1), f64(w2), tp, "gelu_erf", align=8)
+    Bd.check(f64(y), bref, own, car)
 
 
 # ---------------------------------------------------------------- LM head
@@ -292,6 +313,8 @@ def test_lmhead_argmax(case):
         check_shard_ids(sidx.cpu().numpy(), smax.cpu().numpy(), res)
         if with_logits:
             assert rel(logits.view(B, V), res.logits) <= 1e-5
+            Bd.check(f64(logits.view(B, V)), res.logits, Bd.logits(f64(x), f64(w)),
+                     u_out=Bd.U_FP32)
         assert int(ws.abs().sum()) == 0
 
 

@@ -9,6 +9,7 @@ import oracle as O
 import tensor_transformer_linear_b200 as T
 from workloads import gen
 
+from . import _bounds as Bd
 from ._parity import TOL_BF16, TOL_FP32, f64, rel
 
 pytestmark = pytest.mark.gpu
@@ -47,7 +48,14 @@ def test_row_linear_reduce_scatter(dtype, tp, batch, seq, kr, N, with_bias, with
                                       O.row_weight_slices(f64(w2), k_w), batch, seq,
                                       None if b is None else f64(b),
                                       None if res is None else f64(res))
-    assert rel(y, ref) <= (TOL_BF16 if dtype == torch.bfloat16 else TOL_FP32)
+    bf16 = dtype == torch.bfloat16
+    assert rel(y, ref) <= (TOL_BF16 if bf16 else TOL_FP32)
+    # element-wise, with the bound laid out like the output (rank-major slices)
+    res_full = None if res is None else O.seq_gather(f64(res), batch, seq, tp)
+    full, own, _ = Bd.row(O.row_weight_slices(f64(h), k_w), O.row_weight_slices(f64(w2), k_w),
+                          None if b is None else f64(b), res_full, simt=not bf16)
+    Bd.check(f64(y), O.seq_scatter(full, batch, seq, tp), O.seq_scatter(own, batch, seq, tp),
+             u_out=Bd.U_BF16 if bf16 else Bd.U_FP32)
 
 
 @pytest.mark.parametrize("dtype,subs,tp,batch,seq,K,act", [
@@ -66,9 +74,13 @@ def test_column_linear_allgather(dtype, subs, tp, batch, seq, K, act):
                                       act)
     torch.cuda.synchronize()
     ref = O.column_linear_allgather(f64(x_sp), batch, seq, f64(w), None, part, act)
-    tol = TOL_BF16 if dtype == torch.bfloat16 else TOL_FP32
-    for g, r in zip(T.shard_views(y, p, M), ref):
+    bf16 = dtype == torch.bfloat16
+    tol = TOL_BF16 if bf16 else TOL_FP32
+    bref, own, _ = Bd.column(O.seq_gather(f64(x_sp), batch, seq, tp), f64(w), None, part, act,
+                             simt=not bf16)
+    for g, r, br, e in zip(T.shard_views(y, p, M), ref, bref, own):
         assert rel(g, r) <= tol
+        Bd.check(f64(g), br, e, u_out=Bd.U_BF16 if bf16 else Bd.U_FP32)
 
 
 def test_column_linear_allgather_needs_whole_tma_boxes_for_bf16():
@@ -102,6 +114,9 @@ def test_sequence_parallel_block_round_trip():
     ref = O.row_linear_reduce_scatter(h_ref, O.row_weight_slices(f64(w2), k_w), batch, seq,
                                       None, xs)
     assert rel(y, ref) <= TOL_BF16
+    full, own, car = Bd.mlp(xg, f64(w1), f64(w2), tp, "gelu_erf", norm=True, residual=True)
+    Bd.check(f64(y), O.seq_scatter(full, batch, seq, tp), O.seq_scatter(own, batch, seq, tp),
+             O.seq_scatter(car, batch, seq, tp))
 
 
 @pytest.mark.parametrize("M,K,F,tp", [
@@ -115,10 +130,11 @@ def test_swiglu_column_linear(M, K, F, tp):
     w = _t((2 * F, K), 0.05, 1)
     h = T.tpl_swiglu_column_linear(x.to(DEV), w.to(DEV), F, tp)
     torch.cuda.synchronize()
-    ref = O.swiglu_column_linear(f64(x), f64(w), F, tp)
+    ref, own = Bd.swiglu(f64(x), f64(w), F, tp)
     p = T.tpl_partition_subparams([F], tp, 1)
-    for g, r in zip(T.shard_views(h, p, M), ref):
+    for g, r, e in zip(T.shard_views(h, p, M), ref, own):
         assert rel(g, r) <= TOL_BF16
+        Bd.check(f64(g), r, e)
 
 
 def test_swiglu_rejects_fp32_and_indivisible():

@@ -13,6 +13,7 @@ import oracle as O
 import tensor_transformer_linear_b200 as T
 from workloads import gen
 
+from . import _bounds as Bd
 from ._parity import TOL_BF16, check_ids, f64, rel
 
 pytestmark = pytest.mark.gpu
@@ -75,13 +76,18 @@ def test_scatter_then_reduce_is_the_reduce_scatter(tp, batch, seq, inter, N, wit
                                       bias=None if bias is None else f64(bias),
                                       residual_sp=res_sp)
     assert rel(got, ref) <= TOL_BF16
+    full, own, car = Bd.scatter_reduce(h_parts, w_parts, None if bias is None else f64(bias),
+                                       None if res is None else f64(res))
+    sp = lambda a: O.seq_scatter(a, batch, seq, tp)
+    Bd.check(got, sp(full), sp(own), sp(car))
 
     # Slot s of rank q's buffer is rank s's partial of rank q's tokens.
-    parts = O.row_partials(h_parts, w_parts)
+    parts, pown = Bd.partials(h_parts, w_parts)
     for q in range(tp):
         slots = f64(recv[q]).reshape(tp, batch, seg, N)
         for s in range(tp):
-            assert rel(slots[s], O.seq_scatter(parts[s], batch, seq, tp)[q]) <= TOL_BF16
+            assert rel(slots[s], sp(parts[s])[q]) <= TOL_BF16
+            Bd.check(slots[s], sp(parts[s])[q], sp(pown[s])[q], what=f"slot {s} of rank {q}")
 
 
 @pytest.mark.parametrize("tp,batch,seq,inter,N,with_bias,res_mode", [
@@ -131,9 +137,13 @@ def test_scatter_then_reduce_allgather_is_the_full_row_linear_on_every_rank(
     ref = O.row_linear_reduce(h_parts, O.row_weight_slices(f64(W2), k_w),
                               None if bias is None else f64(bias),
                               None if res is None else f64(res))
+    full, own, car = Bd.scatter_reduce(h_parts, O.row_weight_slices(f64(W2), k_w),
+                                       None if bias is None else f64(bias),
+                                       None if res is None else f64(res))
     for q in range(tp):
         assert rel(outs[q], ref) <= TOL_BF16, q
         assert torch.equal(outs[q], outs[0]), q      # every rank holds the same Y
+    Bd.check(f64(outs[0]), full, own, car)
 
 
 def test_reduce_slots_in_place_on_the_residual():
@@ -145,6 +155,8 @@ def test_reduce_slots_in_place_on_the_residual():
     torch.cuda.synchronize()
     ref = f64(recv).sum(axis=0) + f64(res)
     assert rel(y, ref) <= TOL_BF16
+    sref, own = Bd.slot_sum(list(f64(recv)), f64(res))
+    Bd.check(f64(y), sref, own)
 
 
 @pytest.mark.parametrize("B,K,V,tp", [(32, 256, 4999, 4), (5, 64, 37, 8)])
@@ -189,7 +201,7 @@ def test_gather_column_is_the_column_linear_of_the_gathered_tokens(tp, batch, se
     W = _t((sum(subs), K), 0.02, 1)
     b = _t((sum(subs),), 0.02, 3) if with_bias else None
     part = O.partition_subparams(subs, tp, align)
-    ref = O.column_linear(f64(x), f64(W), None if b is None else f64(b), part, act)
+    ref, own, _ = Bd.column(f64(x), f64(W), None if b is None else f64(b), part, act)
     # rank q's token slice: tokens q * seg .. of every sequence
     slices = [x.view(batch, tp, seg, K)[:, q].contiguous().to(DEV) for q in range(tp)]
     for r in range(tp):
@@ -202,3 +214,4 @@ def test_gather_column_is_the_column_linear_of_the_gathered_tokens(tp, batch, se
         y_r = T.tpl_column_linear_gather(p_r, slices, batch, seq, w_r, b_r, act)
         torch.cuda.synchronize()
         assert rel(f64(y_r).reshape(M, part.shard_width[r]), ref[r]) <= TOL_BF16
+        Bd.check(f64(y_r).reshape(M, part.shard_width[r]), ref[r], own[r])

@@ -16,6 +16,7 @@ import tensor_transformer_linear_b200 as T
 from workloads import configs as C
 from workloads import gen
 
+from . import _bounds as Bd
 from ._parity import TOL_BF16, TOL_FP32, check_ids, check_shard_ids, f64, rel
 
 pytestmark = pytest.mark.gpu
@@ -42,12 +43,15 @@ def test_tiny_tp_mlp_fp32_full():
     y = blk(x.to(DEV))
     torch.cuda.synchronize()
     part = O.partition_subparams([w.inter], w.tp, 1)
-    h_ref = O.column_linear(f64(x), f64(w1), None, part, w.act)
+    h_ref, h_own, _ = Bd.column(f64(x), f64(w1), None, part, w.act, simt=True)
     h_got = T.shard_views(blk._bufs["h"], blk.part, w.M)
-    for g, r in zip(h_got, h_ref):
+    for g, r, e in zip(h_got, h_ref, h_own):
         assert rel(g, r) <= TOL_FP32
+        Bd.check(f64(g), r, e, u_out=Bd.U_FP32)
     ref = O.tp_mlp(f64(x), f64(w1), f64(w2), w.tp, w.act)
     assert rel(y, ref) <= TOL_FP32
+    bref, own, car = Bd.mlp(f64(x), f64(w1), f64(w2), w.tp, w.act, bf16=False)
+    Bd.check(f64(y), bref, own, car, u_out=Bd.U_FP32)
 
 
 def test_gqa_fused_qkv_full_size():
@@ -59,10 +63,11 @@ def test_gqa_fused_qkv_full_size():
     rows = _sample_rows(w.M)
     xr = gen.rows((w.M, w.hidden), rows, 1.0, tensor_id=gen.TID_X)
     part = O.partition_subparams(list(w.sub_sizes), w.tp, w.align)
-    ref = O.column_linear(f64(xr), f64(C.qkv_w(w)), f64(C.qkv_bias(w)), part)
+    ref, own, _ = Bd.column(f64(xr), f64(C.qkv_w(w)), f64(C.qkv_bias(w)), part)
     got = [f64(v[rows]) for v in T.shard_views(y, p, w.M)]
-    for g, r in zip(got, ref):
+    for g, r, e in zip(got, ref, own):
         assert O.rel_frobenius(g, r) <= TOL_BF16
+        Bd.check(g, r, e)
     assert O.rel_frobenius(np.concatenate(got, 1), np.concatenate(ref, 1)) <= TOL_BF16
 
 
@@ -76,12 +81,15 @@ def test_rmsnorm_tp_mlp_full_size():
     torch.cuda.synchronize()
     rows = _sample_rows(w.M)
     xr = gen.rows((w.M, w.hidden), rows, 1.0, tensor_id=gen.TID_X)
-    ref = O.tp_mlp(f64(xr), f64(C.mlp_w1(w)), f64(C.mlp_w2(w)), w.tp, w.act,
-                   scale=f64(C.mlp_scale(w)), centered=True, norm=True)
+    ref, own, car = Bd.mlp(f64(xr), f64(C.mlp_w1(w)), f64(C.mlp_w2(w)), w.tp, w.act,
+                           scale=f64(C.mlp_scale(w)), centered=True, norm=True)
     assert rel(y[rows], ref) <= TOL_BF16
+    Bd.check(f64(y[rows]), ref, own, car)
     # the RMSNorm output of the same rows (first step of the block)
     xn = blk._bufs["xn"].view(w.M, w.hidden)[rows]
-    assert rel(xn, O.rmsnorm(f64(xr), f64(C.mlp_scale(w)), True)) <= TOL_BF16
+    nref, nown = Bd.rmsnorm(f64(xr), f64(C.mlp_scale(w)), True)
+    assert rel(xn, nref) <= TOL_BF16
+    Bd.check(f64(xn), nref, nown)
 
 
 def test_decode_lmhead_full_size():
@@ -98,6 +106,8 @@ def test_decode_lmhead_full_size():
     check_shard_ids(sidx.cpu().numpy(), smax.cpu().numpy(), res)
     assert torch.equal(ids, ids2) and torch.equal(sidx, sidx2) and torch.equal(smax, smax2)
     assert rel(logits.view(w.batch, w.vocab), res.logits) <= 1e-5
+    Bd.check(f64(logits.view(w.batch, w.vocab)), res.logits,
+             Bd.logits(f64(C.lm_x(w)), f64(C.lm_w(w))), u_out=Bd.U_FP32)
     # the chunk layout the ids follow (global id = r * shard + chunk offset + j)
     lay = O.vocab_layout(w.vocab, w.tp, w.n_chunks)
     assert lay.shard == 16032 and lay.split_sizes == [4008] * 4
@@ -117,10 +127,16 @@ def test_four_layer_stack_full_size():
     got = f64(x[rows])
     del layers, x
     torch.cuda.empty_cache()
-    xr = f64(gen.rows((w.M, w.hidden), rows, 1.0, tensor_id=gen.TID_X))
+    x0 = f64(gen.rows((w.M, w.hidden), rows, 1.0, tensor_id=gen.TID_X))
+    xr = x0
     for l in range(w.layers):
         w1, w2 = f64(C.mlp_w1(w, l)), f64(C.mlp_w2(w, l))
         xr = O.tp_mlp(xr, w1, w2, w.tp, w.act, norm=True, residual=True)
         del w1, w2
     err = O.rel_frobenius(got, xr)
     assert err <= TOL_BF16, err
+    # element-wise: the bound carried through all four layers
+    layers = [(f64(C.mlp_w1(w, l)), f64(C.mlp_w2(w, l))) for l in range(w.layers)]
+    bref, own, car = Bd.stack(x0, layers, w.tp, w.act)
+    del layers
+    Bd.check(got, bref, own, car)
