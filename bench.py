@@ -241,6 +241,7 @@ class Block:
         self.flops = 0.0
         self.gemm_flops = 0.0
         self.launches = []        # (part name, callable(stream)), in launch order
+        self.ws = T.gemm_workspace(dev)   # stream-K workspace, shared by the step's GEMMs
         # Attributes holding each step's inputs and results; every launch reads
         # them at call time, so the end-to-end pipeline can rotate buffer sets.
         self.io_in, self.io_out = [], []
@@ -252,7 +253,8 @@ class Block:
             self.qpart = T.tpl_partition_subparams(q.sub_sizes, q.tp, q.align)
             self.qy = torch.empty(q.M * q.out, dtype=torch.bfloat16, device=dev)
             self.launches.append(("qkv_column", lambda s: T.tpl_column_linear(
-                self.qpart, self.qx, self.qw, self.qb, "none", y=self.qy, stream=s)))
+                self.qpart, self.qx, self.qw, self.qb, "none", y=self.qy, stream=s,
+                workspace=self.ws)))
             self.flops += q.flops()
             self.gemm_flops += q.flops()
             self.io_in.append("qx")
@@ -268,10 +270,12 @@ class Block:
             self.launches += [
                 ("rmsnorm", lambda s: T.tpl_rmsnorm(self.mx, mlp.scale, True, 1e-6, y=self.xn,
                                                     stream=s)),
-                ("mlp_column_gelu", lambda s: T.tpl_column_linear(mlp.part, self.xn, mlp.w1, None,
-                                                                  m.act, y=self.h, stream=s)),
+                ("mlp_column_gelu", lambda s: T.tpl_column_linear(
+                    mlp.part, self.xn, mlp.w1, None, m.act, y=self.h, stream=s,
+                    workspace=self.ws)),
                 ("mlp_row_reduce", lambda s: T.tpl_row_linear_reduce(
-                    self.h, mlp.k_w, m.M, mlp.w2, None, None, y=self.my, stream=s))]
+                    self.h, mlp.k_w, m.M, mlp.w2, None, None, y=self.my, stream=s,
+                    workspace=self.ws))]
             self.flops += m.flops()
             self.gemm_flops += m.flops()
             self.io_in.append("mx")
@@ -325,8 +329,10 @@ class Stack:
         self.x0 = C.mlp_x(w, dev)
         self.x = self.x0.clone()
         self.io_in, self.io_out = ["x"], ["x"]   # the residual stream is updated in place
+        self.ws = T.gemm_workspace(dev)
         self.layers = [T.TPMLP(C.mlp_w1(w, l, dev), C.mlp_w2(w, l, dev), w.tp, w.act,
-                               norm=True, residual=True) for l in range(w.layers)]
+                               norm=True, residual=True, workspace=self.ws)
+                       for l in range(w.layers)]
         self.flops = w.flops()
         self.gemm_flops = w.flops()
         self.launches_per_step = 3 * w.layers
@@ -346,11 +352,12 @@ class Stack:
             T.tpl_rmsnorm(self.x, None, False, 1e-6, y=xn, stream=stream)
             if events is not None:
                 events[i + 1].record(stream)
-            T.tpl_column_linear(layer.part, xn, layer.w1, None, layer.act, y=h, stream=stream)
+            T.tpl_column_linear(layer.part, xn, layer.w1, None, layer.act, y=h, stream=stream,
+                                workspace=self.ws)
             if events is not None:
                 events[i + 2].record(stream)
             T.tpl_row_linear_reduce(h, layer.k_w, M, layer.w2, None, self.x, y=self.x,
-                                    stream=stream)
+                                    stream=stream, workspace=self.ws)
             i += 3
         if events is not None:
             events[i].record(stream)
@@ -452,6 +459,7 @@ class NextRows:
             self.hbuf = torch.empty(tp * M * kr, dtype=torch.bfloat16, device=dev)
             self.recv = [torch.empty(tp * rows * N, dtype=torch.bfloat16, device=dev)
                          for _ in range(tp)]
+            self.ws = T.gemm_workspace(dev)
 
             def norm_all(s):
                 for q in range(tp):
@@ -463,12 +471,13 @@ class NextRows:
                 for r in range(tp):
                     T.tpl_column_linear_gather(self.p_rank, slices, b, sq,
                                                self.w1[r * kr:(r + 1) * kr], None, m.act,
-                                               y=hs[r], stream=s)
+                                               y=hs[r], stream=s, workspace=self.ws)
 
             def scatter_all(s):
                 hs, ws = self.hbuf.view(tp, M, kr), self.w2p.view(tp, N, kr)
                 for r in range(tp):
-                    T.tpl_row_linear_scatter(hs[r], ws[r], b, sq, r, tp, self.recv, stream=s)
+                    T.tpl_row_linear_scatter(hs[r], ws[r], b, sq, r, tp, self.recv, stream=s,
+                                             workspace=self.ws)
 
             def reduce_all(s):
                 for q in range(tp):

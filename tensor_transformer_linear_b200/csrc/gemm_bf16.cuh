@@ -81,6 +81,19 @@ struct GemmArgs {
   // odd tiles, so a tile wave starts on the K slices the wave before it read
   // last (still in L2) when the two waves share operand blocks.
   int32_t k_serp;
+  // Stream-K (CTA-pair kernel): tiles below sk_first_tile (a multiple of the
+  // pair count) are whole work items, dealt round-robin as before.  The K steps
+  // of the tiles from sk_first_tile on are dealt out in contiguous runs of
+  // sk_units per pair (sk_units >= the K steps of one tile), so a tile is split
+  // between at most two pairs: pair p + 1 computes its K tail first thing
+  // (storing the fp32 partial in sk_partial, slot p + 1, then raising its
+  // flags to sk_epoch) and pair p its head last, adding that partial before
+  // the epilogue.  sk_units == 0: no stream-K phase.
+  int32_t sk_first_tile;
+  int32_t sk_units;
+  uint32_t sk_epoch;
+  float* sk_partial;  // [pairs][2 CTAs][kEpiWarps][4 chunks][32 rows][32 columns]
+  uint32_t* sk_flag;  // [pairs][2 CTAs][kEpiWarps]
   int32_t n_pieces;
   ColPiece pieces[kMaxPieces];
   const __nv_bfloat16* bias;
@@ -111,6 +124,70 @@ struct GemmArgs {
   int32_t a_gather;
   CUtensorMap tmGather[kMaxGather];
 };
+
+// Row mode: the rank and K block of K step ki of a tile.
+__device__ __forceinline__ void row_pos(const GemmArgs& a, int ki, int& rr, int& kb) {
+  const int n1 = max(0, min(a.r1, a.r_split) - a.r0) * a.k_iters;
+  if (ki < n1) {
+    rr = a.r0 + ki / a.k_iters;
+    kb = ki - (rr - a.r0) * a.k_iters;
+  } else {
+    const int first2 = max(a.r0, a.r_split);
+    const int k2 = ki - n1;
+    rr = first2 + k2 / a.k_iters2;
+    kb = k2 - (rr - first2) * a.k_iters2;
+  }
+}
+
+// Work items of one CTA pair: its data-parallel tiles, then its run of
+// stream-K steps (see GemmArgs), cut at tile boundaries.
+enum WorkRole : int { kWorkFull = 0, kWorkHead = 1, kWorkTail = 2 };
+
+struct WorkItem {
+  int tile;
+  int k0, k1;  // K steps [k0, k1) of the tile
+  int role;    // kWorkFull, kWorkHead (adds the next pair's partial), kWorkTail (stores one)
+};
+
+struct WorkIter {
+  int t;             // next data-parallel tile
+  int64_t u, u1;     // stream-K steps [u, u1) still to deal
+};
+
+__device__ __forceinline__ void work_begin(const GemmArgs& a, int pair, int k_total, WorkIter& w) {
+  w.t = pair;
+  w.u = w.u1 = 0;
+  if (a.sk_units > 0) {
+    const int64_t total = static_cast<int64_t>(a.num_tiles - a.sk_first_tile) * k_total;
+    w.u = min(static_cast<int64_t>(pair) * a.sk_units, total);
+    w.u1 = min(w.u + a.sk_units, total);
+  }
+}
+
+__device__ __forceinline__ bool work_next(const GemmArgs& a, int npairs, int k_total,
+                                          WorkIter& w, WorkItem& it) {
+  const int dp_end = a.sk_units > 0 ? a.sk_first_tile : a.num_tiles;
+  if (w.t < dp_end) {
+    it.tile = w.t;
+    it.k0 = 0;
+    it.k1 = k_total;
+    it.role = kWorkFull;
+    w.t += npairs;
+    return true;
+  }
+  if (w.u < w.u1) {
+    const int64_t off = w.u / k_total;
+    const int kb = static_cast<int>(w.u - off * k_total);
+    const int ke = static_cast<int>(min(static_cast<int64_t>(k_total), kb + (w.u1 - w.u)));
+    it.tile = a.sk_first_tile + static_cast<int>(off);
+    it.k0 = kb;
+    it.k1 = ke;
+    it.role = kb > 0 ? kWorkTail : (ke < k_total ? kWorkHead : kWorkFull);
+    w.u += ke - kb;
+    return true;
+  }
+  return false;
+}
 
 // Number of 64-wide K steps of one tile.
 __device__ __forceinline__ int k_steps(const GemmArgs& a) {

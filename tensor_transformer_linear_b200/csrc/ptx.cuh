@@ -75,6 +75,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// ------------------------------------------------- flags between CTAs
+
+// Release store / acquire load of a 32-bit flag in global memory, GPU scope.
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits until *p == want; gives up (false) after `limit_ns` or when
+// `abort_flag` is set, like mbar_wait.
+__device__ __forceinline__ bool flag_wait(const uint32_t* p, uint32_t want,
+                                          volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  if (ld_acquire_gpu(p) == want) return true;
+  const uint64_t t0 = globaltimer();
+  uint32_t n = 0;
+  while (ld_acquire_gpu(p) != want) {
+    __nanosleep(100);
+    if ((++n & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {

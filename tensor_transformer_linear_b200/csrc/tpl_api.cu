@@ -35,6 +35,7 @@ struct DeviceInfo {
   int sm_count = 0;
   bool gemm_attr = false;
   bool lm_attr = false;
+  uint32_t sk_epoch = 0;  // last stream-K launch epoch on this device
 };
 
 std::mutex g_mu;
@@ -119,6 +120,62 @@ int env_int(const char* name, int dflt) {
   return (e != nullptr && e[0] != '\0') ? std::atoi(e) : dflt;
 }
 
+// A caller's stream-K workspace (see tpl_gemm_workspace_size).
+struct SkWorkspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+constexpr size_t kSkSlotFloats = static_cast<size_t>(2) * tpl::kEpiWarps * 4 * 32 * 32;  // per pair
+constexpr size_t kSkSlotFlags = static_cast<size_t>(2) * tpl::kEpiWarps;
+
+size_t sk_partial_bytes(int sm_count) {
+  return static_cast<size_t>(sm_count / 2) * kSkSlotFloats * sizeof(float);
+}
+
+size_t sk_workspace_bytes(int sm_count) {
+  const size_t raw = sk_partial_bytes(sm_count) +
+                     static_cast<size_t>(sm_count / 2) * kSkSlotFlags * sizeof(uint32_t);
+  return (raw + 255) / 256 * 256;
+}
+
+// K steps of one tile (host copy of tpl::k_steps).
+int host_k_steps(const tpl::GemmArgs& a) {
+  if (a.mode != tpl::kModeRow) return a.k_iters;
+  const int n1 = std::max(0, std::min(a.r1, a.r_split) - a.r0);
+  const int n2 = std::max(0, a.r1 - std::max(a.r0, a.r_split));
+  return n1 * a.k_iters + n2 * a.k_iters2;
+}
+
+// Stream-K plan of a CTA-pair launch: the last full wave and the partial one
+// are dealt out by K steps (at least one tile's worth per pair).  Only when a
+// workspace is given, the last wave is partial, there is a full wave before it,
+// and the epilogue is the plain one (no SwiGLU pairing, no per-rank partials).
+void plan_stream_k(tpl::GemmArgs& a, int64_t tiles, int64_t pairs, DeviceInfo* dev,
+                   const SkWorkspace* ws) {
+  a.sk_first_tile = static_cast<int32_t>(tiles);
+  a.sk_units = 0;
+  if (ws == nullptr || ws->ptr == nullptr || ws->bytes < sk_workspace_bytes(dev->sm_count))
+    return;
+  if (a.mode == tpl::kModeSwiglu || a.partials != nullptr) return;
+  if (env_int("TPL_GEMM_STREAMK", 1) == 0) return;
+  const int64_t waves = tiles / pairs, rem = tiles % pairs;
+  if (waves < 1 || rem == 0) return;
+  const int64_t k_total = host_k_steps(a);
+  const int64_t first = (waves - 1) * pairs;
+  const int64_t units = (tiles - first) * k_total;
+  const int64_t per_pair = (units + pairs - 1) / pairs;
+  if (per_pair < k_total || per_pair > INT32_MAX) return;
+  a.sk_first_tile = static_cast<int32_t>(first);
+  a.sk_units = static_cast<int32_t>(per_pair);
+  a.sk_partial = static_cast<float*>(ws->ptr);
+  a.sk_flag = reinterpret_cast<uint32_t*>(static_cast<char*>(ws->ptr) +
+                                          sk_partial_bytes(dev->sm_count));
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (++dev->sk_epoch == 0) dev->sk_epoch = 1;
+  a.sk_epoch = dev->sk_epoch;
+}
+
 // CTA pairs (tcgen05 cta_group::2, 256-row tiles) unless M fits one 128-row
 // block or TPL_GEMM_CTA_PAIRS=0 asks for the single-CTA kernel.
 bool use_cta_pairs(int64_t M) {
@@ -129,7 +186,8 @@ bool use_cta_pairs(int64_t M) {
 
 // Fills the tile counts of `a` (n_tiles / n_halves already set) and launches
 // the GEMM on a single CTA per tile or on CTA pairs.
-tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, const DeviceInfo* dev, cudaStream_t st) {
+tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, DeviceInfo* dev, cudaStream_t st,
+                       const SkWorkspace* ws = nullptr) {
   const bool pairs = use_cta_pairs(M) && dev->sm_count >= 2;
   const int64_t bm = pairs ? tpl::kPairBM : tpl::kBM;
   a.m_blocks = static_cast<int32_t>((M + bm - 1) / bm);
@@ -146,8 +204,12 @@ tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, const DeviceInfo* dev, cudaS
   const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
   if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
   a.num_tiles = static_cast<int32_t>(tiles);
+  a.sk_first_tile = static_cast<int32_t>(tiles);
+  a.sk_units = 0;
   if (pairs) {
-    const int grid = 2 * static_cast<int>(std::min<int64_t>(tiles, dev->sm_count / 2));
+    const int64_t npairs = std::min<int64_t>(tiles, dev->sm_count / 2);
+    plan_stream_k(a, tiles, npairs, dev, ws);
+    const int grid = 2 * static_cast<int>(npairs);
     tpl::gemm_bf16_tcgen05_pair<<<grid, tpl::kGemmThreads, tpl::kGemmPairSmemBytes, st>>>(a);
   } else {
     const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
@@ -210,7 +272,8 @@ struct GatherA {
 
 tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
                        const void* bias, int act, void* y, cudaStream_t st,
-                       const SeqPar& sp = SeqPar{}, const GatherA* ga = nullptr) {
+                       const SeqPar& sp = SeqPar{}, const GatherA* ga = nullptr,
+                       const SkWorkspace* ws = nullptr) {
   if ((K % 8) != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 2) ||
       (bias != nullptr && !aligned(bias, 2)))
     return TPL_ERR_ALIGN;
@@ -276,7 +339,7 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
     a.n_halves = hb;
     a.vec_store = vec ? 1 : 0;
     a.n_tiles = (hb + 1) / 2;
-    if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
+    if ((s = launch_gemm(a, M, dev, st, ws)) != TPL_OK) return s;
   }
   return TPL_OK;
 }
@@ -334,7 +397,7 @@ tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t
 tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_t N, const void* w,
                     const void* bias, const void* residual, void* y, float* partials,
                     cudaStream_t st, const SeqPar& sp = SeqPar{},
-                    const PeerScatter* ps = nullptr) {
+                    const PeerScatter* ps = nullptr, const SkWorkspace* ws = nullptr) {
   for (int r = 0; r < tp; ++r)
     if (k_w[r] % 8 != 0) return TPL_ERR_ALIGN;
   if (!aligned(h, 16) || !aligned(w, 16) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||
@@ -403,7 +466,7 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
     }
     a.vec_store = vec ? 1 : 0;
   }
-  if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
+  if ((s = launch_gemm(a, M, dev, st, ws)) != TPL_OK) return s;
 
   if (partials != nullptr) {
     a.bias = nullptr;
@@ -584,9 +647,18 @@ tpl_status tpl_partition_subparams(const int64_t* sub_sizes, int32_t n_sub, int3
   return TPL_OK;
 }
 
-tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, int64_t K,
-                             const void* w, const void* bias, tpl_dtype dt, tpl_act act, void* y,
-                             void* stream) {
+tpl_status tpl_gemm_workspace_size(size_t* bytes) {
+  if (bytes == nullptr) return TPL_ERR_NULL;
+  DeviceInfo* dev = nullptr;
+  tpl_status s = device_info(&dev);
+  if (s != TPL_OK) return s;
+  *bytes = sk_workspace_bytes(dev->sm_count);
+  return TPL_OK;
+}
+
+static tpl_status column_entry(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                               const void* w, const void* bias, tpl_dtype dt, tpl_act act,
+                               void* y, void* stream, const SkWorkspace* ws) {
   if (p == nullptr) return TPL_ERR_NULL;
   if ((dt != TPL_FP32 && dt != TPL_BF16) || !act_ok(act)) return TPL_ERR_DTYPE;
   tpl_status s = check_partition(p);
@@ -595,13 +667,29 @@ tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, i
   if (M == 0) return TPL_OK;
   if (x == nullptr || w == nullptr || y == nullptr) return TPL_ERR_NULL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dt == TPL_BF16 ? column_bf16(p, x, M, K, w, bias, act, y, st)
+  return dt == TPL_BF16 ? column_bf16(p, x, M, K, w, bias, act, y, st, SeqPar{}, nullptr, ws)
                         : column_fp32(p, x, M, K, w, bias, act, y, st);
 }
 
-tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
-                                 int64_t N, const void* w, const void* bias, const void* residual,
-                                 tpl_dtype dt, void* y, float* partials, void* stream) {
+tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                             const void* w, const void* bias, tpl_dtype dt, tpl_act act, void* y,
+                             void* stream) {
+  return column_entry(p, x, M, K, w, bias, dt, act, y, stream, nullptr);
+}
+
+tpl_status tpl_column_linear_ws(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                                const void* w, const void* bias, tpl_dtype dt, tpl_act act,
+                                void* y, void* workspace, size_t ws_bytes, void* stream) {
+  if (workspace == nullptr) return TPL_ERR_NULL;
+  SkWorkspace ws;
+  ws.ptr = workspace;
+  ws.bytes = ws_bytes;
+  return column_entry(p, x, M, K, w, bias, dt, act, y, stream, &ws);
+}
+
+static tpl_status row_entry(const void* h, const int64_t* k_w, int32_t tp, int64_t M, int64_t N,
+                            const void* w, const void* bias, const void* residual, tpl_dtype dt,
+                            void* y, float* partials, void* stream, const SkWorkspace* ws) {
   if (k_w == nullptr) return TPL_ERR_NULL;
   if (dt != TPL_FP32 && dt != TPL_BF16) return TPL_ERR_DTYPE;
   if (tp < 1 || tp > TPL_MAX_TP || M < 0 || N < 1 || M > INT32_MAX || N > INT32_MAX)
@@ -615,8 +703,26 @@ tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, 
   if (M == 0) return TPL_OK;
   if (h == nullptr || w == nullptr || y == nullptr) return TPL_ERR_NULL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dt == TPL_BF16 ? row_bf16(h, k_w, tp, M, N, w, bias, residual, y, partials, st)
-                        : row_fp32(h, k_w, tp, M, N, w, bias, residual, y, partials, st);
+  return dt == TPL_BF16
+             ? row_bf16(h, k_w, tp, M, N, w, bias, residual, y, partials, st, SeqPar{}, nullptr, ws)
+             : row_fp32(h, k_w, tp, M, N, w, bias, residual, y, partials, st);
+}
+
+tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
+                                 int64_t N, const void* w, const void* bias, const void* residual,
+                                 tpl_dtype dt, void* y, float* partials, void* stream) {
+  return row_entry(h, k_w, tp, M, N, w, bias, residual, dt, y, partials, stream, nullptr);
+}
+
+tpl_status tpl_row_linear_reduce_ws(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
+                                    int64_t N, const void* w, const void* bias,
+                                    const void* residual, tpl_dtype dt, void* y, float* partials,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  if (workspace == nullptr) return TPL_ERR_NULL;
+  SkWorkspace ws;
+  ws.ptr = workspace;
+  ws.bytes = ws_bytes;
+  return row_entry(h, k_w, tp, M, N, w, bias, residual, dt, y, partials, stream, &ws);
 }
 
 tpl_status tpl_rmsnorm(const void* x, int64_t M, int64_t H, const float* scale, int32_t centered,

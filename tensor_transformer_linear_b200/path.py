@@ -46,7 +46,8 @@ class TPMLP:
 
     def __init__(self, w1: torch.Tensor, w2_full: torch.Tensor, tp: int, act: str,
                  scale: Optional[torch.Tensor] = None, centered: bool = False,
-                 norm: bool = True, residual: bool = False, eps: float = 1e-6):
+                 norm: bool = True, residual: bool = False, eps: float = 1e-6,
+                 workspace: Optional[torch.Tensor] = None):
         self.inter, self.hidden = w1.shape
         self.part = tpl_partition_subparams([self.inter], tp, 1)
         self.k_w = [self.part.shard_width[r] for r in range(tp)]
@@ -54,6 +55,7 @@ class TPMLP:
         self.w2 = pack_row_weight(w2_full, self.k_w)
         self.act, self.scale, self.centered = act, scale, centered
         self.norm, self.residual, self.eps = norm, residual, eps
+        self.workspace = workspace   # stream-K workspace of the two GEMMs (or None)
         self._bufs = {}
 
     def _buf(self, name, numel, like):
@@ -72,12 +74,12 @@ class TPMLP:
                         stream=stream)
         h = self._buf("h", M * self.inter, x)
         tpl_column_linear(self.part, xn.view(M, self.hidden), self.w1, None, self.act, y=h,
-                          stream=stream)
+                          stream=stream, workspace=self.workspace)
         if out is None:
             out = torch.empty((M, self.hidden), dtype=x.dtype, device=x.device)
         tpl_row_linear_reduce(h, self.k_w, M, self.w2, None,
                               x.view(M, self.hidden) if self.residual else None, y=out,
-                              stream=stream)
+                              stream=stream, workspace=self.workspace)
         return out
 
 

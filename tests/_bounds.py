@@ -247,3 +247,32 @@ def slot_sum(slots, res=None):
         ref = ref + res
         terms = terms + np.abs(res)
     return ref, (len(slots) + 2) * U_FP32 * terms
+
+
+def rank_mlp(x, w1, w2_full, tp, act, scale=None, centered=False, eps=1e-6, x_proxy=None):
+    """The MLP block over GPUs (RMSNorm -> c_fc + act -> c_proj, each rank's
+    c_proj partial stored in bf16 in its owner's slot, the slots and the
+    residual summed in fp32 and rounded once): (reference y, own, carried)."""
+    x = np.asarray(x, dtype=np.float64)
+    H = x.shape[1]
+    part = O.partition_subparams([w1.shape[0]], tp, 1)
+    xn, own_n = rmsnorm(x, scale, centered, eps)
+    car_n = None
+    if x_proxy is not None:
+        ms = np.mean(x * x, axis=1, keepdims=True)
+        g = np.ones(H) if scale is None else (1.0 + scale if centered else scale)
+        car_n = (np.square(g) / (ms + eps)) * x_proxy + np.square(xn) * (
+            np.sum(np.square(x) * x_proxy, axis=1, keepdims=True) / np.square(H * (ms + eps)))
+    h_ref, own_h, car_h = column(xn, w1, None, part, act, x_proxy=stored(xn, own_n, car_n, U_BF16))
+    h_proxy = [stored(h, o, c, U_BF16) for h, o, c in zip(h_ref, own_h, car_h)]
+    w2 = O.row_weight_slices(w2_full, part.shard_width)
+    parts = O.row_partials(h_ref, w2)
+    s = O.row_partials([_abs(h) for h in h_ref], [_abs(w) for w in w2])
+    car_p = [O.row_partials([hp], [_sq(w)])[0] for hp, w in zip(h_proxy, w2)]
+    y = sum(parts) + x
+    own = (tp + 2) * U_FP32 * (sum(np.abs(p) for p in parts) + np.abs(x))
+    car = sum(stored(p, acc(h.shape[1]) * si, cp, U_BF16)
+              for p, h, si, cp in zip(parts, h_ref, s, car_p))
+    if x_proxy is not None:
+        car = car + x_proxy
+    return y, own, car
