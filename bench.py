@@ -44,6 +44,7 @@ from workloads import gen  # noqa: E402
 
 METRIC = "sharded-linear TFLOP/s (% bf16 peak); LM-head decode GB/s (% HBM) at 1 B200"
 DECODE_LAUNCHES = 50
+FUSED_NORM = True   # the block's RMSNorm runs inside its c_fc GEMM
 ALONE_LAUNCHES = 30
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -241,7 +242,7 @@ class Block:
         self.flops = 0.0
         self.gemm_flops = 0.0
         self.launches = []        # (part name, callable(stream)), in launch order
-        self.ws = T.gemm_workspace(dev)   # stream-K workspace, shared by the step's GEMMs
+        self.gemm_ws = T.gemm_workspace(dev)   # stream-K workspace of the step's GEMMs
         # Attributes holding each step's inputs and results; every launch reads
         # them at call time, so the end-to-end pipeline can rotate buffer sets.
         self.io_in, self.io_out = [], []
@@ -254,7 +255,7 @@ class Block:
             self.qy = torch.empty(q.M * q.out, dtype=torch.bfloat16, device=dev)
             self.launches.append(("qkv_column", lambda s: T.tpl_column_linear(
                 self.qpart, self.qx, self.qw, self.qb, "none", y=self.qy, stream=s,
-                workspace=self.ws)))
+                workspace=self.gemm_ws)))
             self.flops += q.flops()
             self.gemm_flops += q.flops()
             self.io_in.append("qx")
@@ -262,20 +263,32 @@ class Block:
         if "mlp" in parts:
             self.mx = C.mlp_x(m, dev)
             self.mlp = T.TPMLP(C.mlp_w1(m, 0, dev), C.mlp_w2(m, 0, dev), m.tp, m.act,
-                               scale=C.mlp_scale(m, 0, dev), centered=True, norm=True)
+                               scale=C.mlp_scale(m, 0, dev), centered=True, norm=True,
+                               fused_norm=FUSED_NORM)
             self.my = torch.empty((m.M, m.hidden), dtype=torch.bfloat16, device=dev)
             self.xn = torch.empty_like(self.mx)
             self.h = torch.empty(m.M * m.inter, dtype=torch.bfloat16, device=dev)
             mlp = self.mlp
+            # the RMSNorm kernel on its own (an L2-flushed launch outside the step)
+            self.alone_launches = {"rmsnorm": lambda s: T.tpl_rmsnorm(
+                self.mx, mlp.scale, True, 1e-6, y=self.xn, stream=s)}
+            if FUSED_NORM:
+                # RMSNorm inside the c_fc GEMM: no normalised copy of x
+                self.norm_ws = mlp.norm_workspace(m.M, dev)
+                self.launches += [
+                    ("mlp_column_rmsnorm_gelu", lambda s: T.tpl_column_linear_rmsnorm(
+                        mlp.part, self.mx, mlp.w1, None, 1e-6, m.act, self.norm_ws, y=self.h,
+                        stream=s))]
+            else:
+                self.launches += [
+                    ("rmsnorm", self.alone_launches["rmsnorm"]),
+                    ("mlp_column_gelu", lambda s: T.tpl_column_linear(
+                        mlp.part, self.xn, mlp.w1, None, m.act, y=self.h, stream=s,
+                        workspace=self.gemm_ws))]
             self.launches += [
-                ("rmsnorm", lambda s: T.tpl_rmsnorm(self.mx, mlp.scale, True, 1e-6, y=self.xn,
-                                                    stream=s)),
-                ("mlp_column_gelu", lambda s: T.tpl_column_linear(
-                    mlp.part, self.xn, mlp.w1, None, m.act, y=self.h, stream=s,
-                    workspace=self.ws)),
                 ("mlp_row_reduce", lambda s: T.tpl_row_linear_reduce(
                     self.h, mlp.k_w, m.M, mlp.w2, None, None, y=self.my, stream=s,
-                    workspace=self.ws))]
+                    workspace=self.gemm_ws))]
             self.flops += m.flops()
             self.gemm_flops += m.flops()
             self.io_in.append("mx")
@@ -304,8 +317,9 @@ class Block:
             events[len(self.launches)].record(stream)
 
     def gemm_part_ids(self):
-        return [i for i, n in enumerate(self.parts) if n in ("qkv_column", "mlp_column_gelu",
-                                                              "mlp_row_reduce")]
+        return [i for i, n in enumerate(self.parts)
+                if n in ("qkv_column", "mlp_column_gelu", "mlp_column_rmsnorm_gelu",
+                         "mlp_row_reduce")]
 
     def lmhead_bytes(self):
         return self.l.algorithmic_bytes() if "lmhead" in self.sel else None
@@ -329,38 +343,47 @@ class Stack:
         self.x0 = C.mlp_x(w, dev)
         self.x = self.x0.clone()
         self.io_in, self.io_out = ["x"], ["x"]   # the residual stream is updated in place
-        self.ws = T.gemm_workspace(dev)
         self.layers = [T.TPMLP(C.mlp_w1(w, l, dev), C.mlp_w2(w, l, dev), w.tp, w.act,
-                               norm=True, residual=True, workspace=self.ws)
+                               norm=True, residual=True, fused_norm=FUSED_NORM)
                        for l in range(w.layers)]
+        # one workspace for every layer (the layers run one after another)
+        self.ws = (self.layers[0].norm_workspace(w.M, dev) if FUSED_NORM
+                   else T.gemm_workspace(dev))
         self.flops = w.flops()
         self.gemm_flops = w.flops()
-        self.launches_per_step = 3 * w.layers
         self.parts = []
         for l in range(w.layers):
-            self.parts += [f"l{l}_rmsnorm", f"l{l}_column_gelu", f"l{l}_row_reduce_residual"]
+            if FUSED_NORM:
+                self.parts += [f"l{l}_column_rmsnorm_gelu", f"l{l}_row_reduce_residual"]
+            else:
+                self.parts += [f"l{l}_rmsnorm", f"l{l}_column_gelu", f"l{l}_row_reduce_residual"]
+        self.launches_per_step = len(self.parts)
 
     def step(self, stream, events=None):
         T = self.T
+        mark = (lambda i: events[i].record(stream)) if events is not None else (lambda i: None)
         i = 0
         for layer in self.layers:
             M = self.x.shape[0]
-            xn = layer._buf("xn", self.x.numel(), self.x).view(M, -1)
             h = layer._buf("h", M * layer.inter, self.x)
-            if events is not None:
-                events[i].record(stream)
-            T.tpl_rmsnorm(self.x, None, False, 1e-6, y=xn, stream=stream)
-            if events is not None:
-                events[i + 1].record(stream)
-            T.tpl_column_linear(layer.part, xn, layer.w1, None, layer.act, y=h, stream=stream,
-                                workspace=self.ws)
-            if events is not None:
-                events[i + 2].record(stream)
+            if FUSED_NORM:
+                mark(i)
+                T.tpl_column_linear_rmsnorm(layer.part, self.x, layer.w1, None, 1e-6, layer.act,
+                                            self.ws, y=h, stream=stream)
+                i += 1
+            else:
+                xn = layer._buf("xn", self.x.numel(), self.x).view(M, -1)
+                mark(i)
+                T.tpl_rmsnorm(self.x, None, False, 1e-6, y=xn, stream=stream)
+                mark(i + 1)
+                T.tpl_column_linear(layer.part, xn, layer.w1, None, layer.act, y=h,
+                                    stream=stream, workspace=self.ws)
+                i += 2
+            mark(i)
             T.tpl_row_linear_reduce(h, layer.k_w, M, layer.w2, None, self.x, y=self.x,
                                     stream=stream, workspace=self.ws)
-            i += 3
-        if events is not None:
-            events[i].record(stream)
+            i += 1
+        mark(i)
 
     def host_inputs(self):
         return {"x": self.x0}
@@ -372,7 +395,7 @@ class Stack:
         return []
 
     def gemm_part_ids(self):
-        return [i for i in range(len(self.parts)) if i % 3 != 0]
+        return [i for i, n in enumerate(self.parts) if not n.endswith("_rmsnorm")]
 
 
 class NextRows:
@@ -524,6 +547,78 @@ class NextRows:
         return []
 
 
+class RankTP:
+    """One rank of the RMSNorm + TP MLP block split over GPUs: x[8,1024,4096],
+    4096->14336->4096, GELU(erf), tp = the number of processes, one per GPU.
+
+    Each rank holds its token slice of the residual stream ``[batch, seq/tp,
+    hidden]`` and its weight shards; a step is TPRankMLP: RMSNorm of the slice ->
+    c_fc + GELU over every rank's slice (each token tile read from the rank that
+    owns it, through a CUDA IPC mapping) -> c_proj, its partials written into
+    the owners' receive buffers -> the slots summed with the residual, in
+    place.  Barriers are one-element all-reduces on the launching stream.  The
+    whole job computes one block per step (strong scaling).  ``ops``,
+    ``exchange`` and ``barrier`` replace the library calls, the CUDA IPC mapping
+    and the stream barrier (host tests run the same orchestration on CPU)."""
+
+    kind = "tp_ranks"
+
+    def __init__(self, dev, rank, world, ops=None, exchange=None, barrier=None,
+                 workload=None, workspace=True):
+        from tensor_transformer_linear_b200 import path
+        m = workload or C.TP_MLP
+        self.m, self.rank, self.tp = m, rank, world
+        b, sq, H, I = m.batch, m.seq, m.hidden, m.inter
+        kr = I // world
+        self.rows = path.sp_rows(b, sq, world)
+        self.name = WORKLOAD_NAMES_RANKS(world)
+        full_x = C.mlp_x(m, dev)
+        self.x = path.sp_slice(full_x, b, sq, world, rank).reshape(self.rows, H)
+        del full_x
+        w1 = C.mlp_w1(m, 0, dev)[rank * kr:(rank + 1) * kr].contiguous()
+        w2 = C.mlp_w2(m, 0, dev)[:, rank * kr:(rank + 1) * kr].contiguous()
+        exchange = exchange or path.exchange_peer_buffers
+        xn = exchange(torch.empty_like(self.x))
+        recv = exchange(torch.empty(path.recv_buffer_numel(world, b, sq, H), dtype=self.x.dtype,
+                                    device=self.x.device))
+        barrier = barrier or path.stream_barrier(device=dev)
+        ws = None
+        if workspace and ops is None:
+            import tensor_transformer_linear_b200 as T
+            ws = T.gemm_workspace(dev)
+        self.block = path.TPRankMLP(w1, w2, rank, world, m.act, xn, recv, barrier,
+                                    scale=C.mlp_scale(m, 0, dev), centered=True, ops=ops,
+                                    workspace=ws)
+        self.parts = ["rank_" + s for s in path.TPRankMLP.STEPS]
+        self.flops = m.flops()                 # the whole job's work per step
+        self.gemm_flops = m.flops() / world   # this rank's GEMMs
+        self.io_in, self.io_out = ["x"], ["x"]   # the residual slice, in place
+        self.batch, self.seq = b, sq
+
+    def step(self, stream, events=None):
+        mark = None if events is None else (lambda i: events[i].record(stream))
+        self.block(self.x, self.batch, self.seq, stream=stream, on_step=mark)
+        if events is not None:
+            events[len(self.parts)].record(stream)
+
+    def gemm_part_ids(self):
+        return [self.parts.index("rank_column_gather"), self.parts.index("rank_row_scatter")]
+
+    def lmhead_bytes(self):
+        return None
+
+    def hbm_parts(self):
+        return []
+
+
+def WORKLOAD_NAMES_RANKS(world):
+    """Name of the TP MLP block split over `world` ranks, one per GPU."""
+    m = C.TP_MLP
+    return (f"tp-ranks rmsnorm-tp-mlp x[{m.batch},{m.seq},{m.hidden}] bf16 "
+            f"{m.hidden}->{m.inter}->{m.hidden} gelu-erf, {world} ranks, one per GPU "
+            "(peer-gather c_fc, peer-scatter c_proj, slot reduction)")
+
+
 # ------------------------------------------------------------------ the oracle
 #
 # The CPU baseline and the reference arm time the fp64 oracle on a bounded
@@ -652,6 +747,11 @@ L2_NOTE = ("not flushed: one step streams ~1.5 GB (block) / ~4 GB (stack), far a
 
 def workload_config(kind, world):
     """The ``config`` of a line: the same for both arms of one workload and N."""
+    if kind == "tp_ranks" and world > 1:
+        return {"workload": WORKLOAD_NAMES_RANKS(world),
+                "parallelism": f"tp{world}: one TP rank per GPU, peer memory over NVLink "
+                               "(CUDA IPC), no replicas",
+                "l2": L2_NOTE}
     par = PARALLELISM.get(kind, "tp shards of each linear computed on one GPU, cross-shard sum "
                                 "in the GEMM epilogue")
     return {"workload": WORKLOAD_NAMES[kind], "parallelism": f"{world} replica(s); " + par,
@@ -826,9 +926,11 @@ def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
         "peak": peak_t, "peak_kind": peak_label, "frac": round(achieved / peak_t, 4),
         "frac_of_burst": round(achieved / pk["bf16_tflops"], 4),
         "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
-        "rmsnorm": {"kernel": "rmsnorm_cta", "bytes_per_step": norm_bytes,
-                    "ms_per_step": round(norm_ms, 4),
-                    "achieved_gbs": round(norm_bytes / (norm_ms * 1e-3) / 1e9, 1)},
+        "rmsnorm": ({"kernel": "rmsnorm_cta", "bytes_per_step": norm_bytes,
+                     "ms_per_step": round(norm_ms, 4),
+                     "achieved_gbs": round(norm_bytes / (norm_ms * 1e-3) / 1e9, 1)}
+                    if norm_ms > 0 else "fused into each layer's c_fc GEMM "
+                                        "(tpl_column_linear_rmsnorm)"),
         "parts_ms": {n: round(v, 4) for n, v in zip(wl.parts, part_ms)},
         "gpu_launches": int(launches), "clocks": clk,
         "l2": "not flushed: one step streams ~4 GB of weights and activations, far above "
@@ -920,7 +1022,8 @@ def main():
         pg = dist
 
     import tensor_transformer_linear_b200 as T
-    wl = wl_cls(dev)
+    ranks = args.workload == "tp_ranks" and world > 1
+    wl = RankTP(dev, rank, world) if ranks else wl_cls(dev)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
@@ -955,6 +1058,7 @@ def main():
     # clean), timed with events around that launch alone; median of ALONE_LAUNCHES
     alone_ms = {}
     launch_of = dict(getattr(wl, "launches", []))
+    launch_of.update(getattr(wl, "alone_launches", {}))
     parts_alone = [h for h in wl.hbm_parts() if h[2] in launch_of]
     if parts_alone:
         flush = torch.ones(256 * 2**20 // 4, dtype=torch.float32, device=dev)
@@ -1011,8 +1115,10 @@ def main():
     if rank == 0:
         pk, pk_kind = peaks()
         step_ms = ms / args.steps
-        value = replica_rate(world, wl.flops, step_ms)
-        e2e_val = replica_rate(world, wl.flops, e_ms / e_steps)
+        # replicas: every rank did a whole step; TP ranks: the job did one step
+        copies = 1 if ranks else world
+        value = replica_rate(copies, wl.flops, step_ms)
+        e2e_val = replica_rate(copies, wl.flops, e_ms / e_steps)
         # dominant kernel: the tcgen05 GEMM (all launches of it in the step)
         gids = wl.gemm_part_ids()
         n_gemm = getattr(wl, "gemm_launches", len(gids)) if gids else 0
@@ -1025,7 +1131,8 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong" if ranks else "weak",
+            "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded SplitMix64 / Irwin-Hall normal, the pages' shapes)",
             "config": workload_config(args.workload, world),
             "roofline": {"kernel": "gemm_bf16_tcgen05_pair", "bound": "tensor",
@@ -1068,15 +1175,22 @@ def main():
                     "measured": f"{DECODE_LAUNCHES} back-to-back launches (a decode loop), "
                                 "CUDA events on the launching stream"}
         for key, kern, part, nbytes, *n_l in wl.hbm_parts():
-            p_ms = part_ms[wl.parts.index(part)]
-            gb = nbytes / (p_ms * 1e-3) / 1e9
             n_l = n_l[0] if n_l else 1
-            line[key] = {"kernel": kern, "bound": "hbm", "achieved": round(gb, 1),
-                         "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gb / pk["hbm_gbs"], 4), "bytes_per_launch": nbytes // n_l,
-                         "launches_per_step": n_l,
-                         "measured": "inside the timed steps, after the kernel before it, whose "
-                                     "dirty output lines in L2 it evicts"}
+            if part in wl.parts:
+                p_ms = part_ms[wl.parts.index(part)]
+                gb = nbytes / (p_ms * 1e-3) / 1e9
+                line[key] = {"kernel": kern, "bound": "hbm", "achieved": round(gb, 1),
+                             "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(gb / pk["hbm_gbs"], 4),
+                             "bytes_per_launch": nbytes // n_l, "launches_per_step": n_l,
+                             "measured": "inside the timed steps, after the kernel before it, "
+                                         "whose dirty output lines in L2 it evicts"}
+            else:
+                # not a launch of the step (the norm is fused into the GEMM there):
+                # the kernel timed on its own
+                line[key] = {"kernel": kern, "bound": "hbm", "unit": "GB/s",
+                             "peak": pk["hbm_gbs"], "bytes_per_launch": nbytes // n_l,
+                             "in_step": False}
             if key in alone_ms:
                 ga = nbytes / (alone_ms[key] * 1e-3) / 1e9
                 line[key]["alone"] = {
@@ -1084,6 +1198,9 @@ def main():
                     "ms": round(alone_ms[key], 4),
                     "measured": f"median of {ALONE_LAUNCHES} launches, each after a read-only "
                                 "256 MiB L2 flush, CUDA events around the launch alone"}
+                if not line[key].get("in_step", True):
+                    line[key].update(achieved=line[key]["alone"]["achieved"],
+                                     frac=line[key]["alone"]["frac"])
         if not gids:
             first = "roofline_lmhead" if "roofline_lmhead" in line else wl.hbm_parts()[0][0]
             line["roofline"] = line.pop(first)

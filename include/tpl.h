@@ -197,6 +197,49 @@ tpl_status tpl_row_linear_reduce_ws(const void* h, const int64_t* k_w, int32_t t
                                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Column-parallel linear of RMSNorm(x) with the norm fused into the GEMM
+ * (google-research allgather_layernorm; nanotron "MLP Module": RMSNorm, then
+ * c_fc).  Since RMSNorm(x) W^T = diag(rsqrt(mean(x^2) + eps)) x (W diag(g))^T,
+ * the norm's scale g is folded into the weight once (tpl_fold_norm_scale) and
+ * the per-row factor is applied in the GEMM epilogue:
+ *   Y_r = act(rsqrt(mean_k x[m][k]^2 + eps) * (x W'_r^T)[m] + b_r)
+ * The GEMM's CTAs compute every row's factor from x (fp32 sums of the bf16
+ * values) while their first tiles' MMAs run, so no normalised copy of x is
+ * written or read.  Rounding: x enters the GEMM unnormalised and g is rounded
+ * into W' once, where the unfused path rounds the normalised x to bf16.
+ *
+ *   x          device bf16 [M][K], the raw activations.
+ *   w          device bf16 [p->logical_out][K], the weight with g folded in.
+ *   bias, act, y, p   as tpl_column_linear.   eps >= 0.
+ *   workspace  device, tpl_column_linear_rmsnorm_workspace_size(M) bytes,
+ *              256-byte aligned, ZERO-FILLED before its first use, reusable;
+ *              its first tpl_gemm_workspace_size() bytes also serve as the
+ *              stream-K workspace of this call.  Calls whose work overlaps on
+ *              the GPU must not share one.
+ * bf16 only (K % 8 == 0, 16-byte aligned x and w).  Errors as
+ * tpl_column_linear, plus TPL_ERR_SHAPE for a short workspace.
+ */
+tpl_status tpl_column_linear_rmsnorm_workspace_size(int64_t M, size_t* bytes);
+
+tpl_status tpl_column_linear_rmsnorm(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                                     const void* w, const void* bias, float eps, tpl_act act,
+                                     void* y, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Folds an RMSNorm scale into the columns of the weight that follows it:
+ *   w_out[n][k] = bf16(w[n][k] * g[k]),  g = 1 + scale (centered) or scale
+ * (google-research allgather_layernorm: scale += 1.0 when centring).  A
+ * one-time weight transformation for tpl_column_linear_rmsnorm.
+ *
+ *   w      device bf16 [rows][K].   scale  device fp32 [K].
+ *   w_out  device bf16 [rows][K]; may alias w.
+ * Requirements: K % 8 == 0; w, w_out and scale 16-byte aligned (else
+ * TPL_ERR_ALIGN).  rows == 0 is a no-op.
+ */
+tpl_status tpl_fold_norm_scale(const void* w, int64_t rows, int64_t K, const float* scale,
+                               int32_t centered, void* w_out, void* stream);
+
+/*
  * RMSNorm (google-research allgather_layernorm; weight-gathered layernorm):
  *   y = x / sqrt(mean(x^2) + eps) * g,  g = 1 + scale (centered != 0),
  *   g = scale (centered == 0), or g = 1 (scale == NULL).

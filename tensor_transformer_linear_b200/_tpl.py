@@ -35,7 +35,9 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
             "tpl_argmax_merge", "tpl_column_linear_gather", "tpl_reduce_slots_allgather",
             "tpl_gemm_workspace_size", "tpl_column_linear_ws", "tpl_row_linear_reduce_ws",
-            "tpl_column_linear_gather_ws", "tpl_row_linear_scatter_ws")
+            "tpl_column_linear_gather_ws", "tpl_row_linear_scatter_ws",
+            "tpl_column_linear_rmsnorm_workspace_size", "tpl_column_linear_rmsnorm",
+            "tpl_fold_norm_scale")
 
 
 class TplError(RuntimeError):
@@ -111,6 +113,10 @@ def lib():
                                                   i32, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp]
         L.tpl_row_linear_scatter_ws.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32,
                                                 ctypes.POINTER(vp), vp, sz, vp]
+        L.tpl_column_linear_rmsnorm_workspace_size.argtypes = [i64, ctypes.POINTER(sz)]
+        L.tpl_column_linear_rmsnorm.argtypes = [ctypes.POINTER(Partition), vp, i64, i64, vp, vp,
+                                                ctypes.c_float, i32, vp, vp, sz, vp]
+        L.tpl_fold_norm_scale.argtypes = [vp, i64, i64, vp, i32, vp, vp]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -207,6 +213,62 @@ def tpl_column_linear(p: Partition, x: torch.Tensor, w: torch.Tensor,
         _check(lib().tpl_column_linear_ws(ctypes.byref(p), _ptr(x), M, K, _ptr(w), _ptr(bias),
                                           DTYPE[dt], ACT[act], _ptr(y), *_ws(workspace),
                                           _stream(stream)), "tpl_column_linear_ws")
+    return y
+
+
+def tpl_column_linear_rmsnorm_workspace_size(M: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tpl_column_linear_rmsnorm_workspace_size(int(M), ctypes.byref(n)),
+           "tpl_column_linear_rmsnorm_workspace_size")
+    return int(n.value)
+
+
+def rmsnorm_linear_workspace(M: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for tpl_column_linear_rmsnorm with up to M rows
+    (reusable across calls on one stream); its first tpl_gemm_workspace_size()
+    bytes are a stream-K workspace for the other GEMM calls too."""
+    with torch.cuda.device(device):
+        n = tpl_column_linear_rmsnorm_workspace_size(M)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def tpl_fold_norm_scale(w: torch.Tensor, scale: torch.Tensor, centered: bool = False,
+                        out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``w[n][k] * g[k]`` in bf16, g = 1 + scale (centred) or scale: an RMSNorm's
+    scale folded into the weight of the column-parallel linear that follows it."""
+    _cuda(w, "w", torch.bfloat16)
+    _cuda(scale, "scale", torch.float32)
+    K = w.shape[-1]
+    if scale.numel() != K:
+        raise ValueError("scale must be [K]")
+    if out is None:
+        out = torch.empty_like(w)
+    _cuda(out, "out", torch.bfloat16)
+    _check(lib().tpl_fold_norm_scale(_ptr(w), w.numel() // K, K, _ptr(scale), int(bool(centered)),
+                                     _ptr(out), _stream(stream)), "tpl_fold_norm_scale")
+    return out
+
+
+def tpl_column_linear_rmsnorm(p: Partition, x: torch.Tensor, w: torch.Tensor,
+                              bias: Optional[torch.Tensor], eps: float, act: str,
+                              workspace: torch.Tensor, y: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """Column-parallel linear of RMSNorm(x) with the norm fused in: ``w`` is the
+    weight with the norm's scale folded in (:func:`tpl_fold_norm_scale`), x the
+    raw activations; ``workspace`` from :func:`rmsnorm_linear_workspace`."""
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(w, "w", torch.bfloat16)
+    if bias is not None:
+        _cuda(bias, "bias", torch.bfloat16)
+    M, K = x.numel() // x.shape[-1], x.shape[-1]
+    if y is None:
+        y = torch.empty(M * p.logical_out, dtype=torch.bfloat16, device=x.device)
+    _cuda(y, "y", torch.bfloat16)
+    if y.numel() < M * p.logical_out or w.numel() != p.logical_out * K:
+        raise ValueError("y or w has the wrong size")
+    _check(lib().tpl_column_linear_rmsnorm(ctypes.byref(p), _ptr(x), M, K, _ptr(w), _ptr(bias),
+                                           float(eps), ACT[act], _ptr(y), *_ws(workspace),
+                                           _stream(stream)), "tpl_column_linear_rmsnorm")
     return y
 
 

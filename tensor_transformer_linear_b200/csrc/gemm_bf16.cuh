@@ -94,6 +94,18 @@ struct GemmArgs {
   uint32_t sk_epoch;
   float* sk_partial;  // [pairs][2 CTAs][kEpiWarps][4 chunks][32 rows][32 columns]
   uint32_t* sk_flag;  // [pairs][2 CTAs][kEpiWarps]
+  // Fused RMSNorm (column mode, google-research allgather_layernorm): A is
+  // the raw x and the norm's scale is folded into the weight, so row m of the
+  // output is act(norm_rs[m] * (x W'^T)[m] + b).  Before its first epilogue,
+  // every CTA's epilogue warps compute norm_rs[m] = rsqrt(mean(x[m]^2) + eps)
+  // for their share of the rows (in fp32, from bf16 x) and raise norm_flag[m]
+  // to sk_epoch; an epilogue scales row m once its flag is up.
+  int32_t norm;
+  float norm_eps;
+  const __nv_bfloat16* norm_x;  // x [M][k_iters * 64 >= K] rows, row stride norm_ld
+  int32_t norm_K, norm_ld;
+  float* norm_rs;        // [M]
+  uint32_t* norm_flag;   // [M]
   int32_t n_pieces;
   ColPiece pieces[kMaxPieces];
   const __nv_bfloat16* bias;
@@ -187,6 +199,62 @@ __device__ __forceinline__ bool work_next(const GemmArgs& a, int npairs, int k_t
     return true;
   }
   return false;
+}
+
+// The fused RMSNorm's statistics: rows [r0, r1) of x for this CTA's 256
+// epilogue threads, 4 adjacent lanes per row (each a quarter of the row's
+// 16-byte vectors, summed in a fixed order), 64 rows per pass.
+__device__ __forceinline__ void norm_stats(const GemmArgs& a, int r0, int r1, int tid) {
+  const int sub = tid & 3;
+  const int nv = a.norm_K / 8;
+  for (int base = r0; base < r1; base += 64) {
+    const int m = base + (tid >> 2);
+    float ss = 0.0f;
+    if (m < r1) {
+      const uint4* row = reinterpret_cast<const uint4*>(a.norm_x + static_cast<int64_t>(m) *
+                                                                       a.norm_ld);
+      int v = sub;
+      for (; v + 28 < nv; v += 32) {  // 8 vectors of this lane in flight
+        uint4 q[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) q[u] = __ldg(row + v + 4 * u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float f0 = bf16_lo(q[u].x), f1 = bf16_hi(q[u].x), f2 = bf16_lo(q[u].y),
+                      f3 = bf16_hi(q[u].y), f4 = bf16_lo(q[u].z), f5 = bf16_hi(q[u].z),
+                      f6 = bf16_lo(q[u].w), f7 = bf16_hi(q[u].w);
+          ss = fmaf(f0, f0, ss); ss = fmaf(f1, f1, ss); ss = fmaf(f2, f2, ss);
+          ss = fmaf(f3, f3, ss); ss = fmaf(f4, f4, ss); ss = fmaf(f5, f5, ss);
+          ss = fmaf(f6, f6, ss); ss = fmaf(f7, f7, ss);
+        }
+      }
+      for (; v < nv; v += 4) {
+        const uint4 q = __ldg(row + v);
+        const float f0 = bf16_lo(q.x), f1 = bf16_hi(q.x), f2 = bf16_lo(q.y), f3 = bf16_hi(q.y),
+                    f4 = bf16_lo(q.z), f5 = bf16_hi(q.z), f6 = bf16_lo(q.w), f7 = bf16_hi(q.w);
+        ss = fmaf(f0, f0, ss); ss = fmaf(f1, f1, ss); ss = fmaf(f2, f2, ss);
+        ss = fmaf(f3, f3, ss); ss = fmaf(f4, f4, ss); ss = fmaf(f5, f5, ss);
+        ss = fmaf(f6, f6, ss); ss = fmaf(f7, f7, ss);
+      }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    if (m < r1 && sub == 0) {
+      a.norm_rs[m] = rsqrtf(ss / static_cast<float>(a.norm_K) + a.norm_eps);
+      __threadfence();
+      ptx::st_release_gpu(a.norm_flag + m, a.sk_epoch);
+    }
+  }
+}
+
+// 1 / rms of row m for the fused RMSNorm, once its flag is up (bounded wait).
+__device__ __forceinline__ bool norm_row_scale(const GemmArgs& a, int m, float& rs,
+                                               volatile int* abort_flag) {
+  rs = 1.0f;
+  if (m >= a.M) return true;
+  if (!ptx::flag_wait(a.norm_flag + m, a.sk_epoch, abort_flag)) return false;
+  rs = __ldcg(a.norm_rs + m);
+  return true;
 }
 
 // Number of 64-wide K steps of one tile.
@@ -316,14 +384,16 @@ __device__ __forceinline__ void load_bias_chunk(const GemmArgs& a, const HalfInf
   }
 }
 
-// Epilogue of 32 accumulator columns of one row; bv holds the chunk's bias.
+// Epilogue of 32 accumulator columns of one row; bv holds the chunk's bias,
+// rs the row's fused-RMSNorm factor (1 without it).
 __device__ __forceinline__ void store_chunk(const GemmArgs& a, const HalfInfo& h, int m, int prow,
                                             __nv_bfloat16* ybase, int col0,
-                                            const uint32_t (&r)[32], const float (&bv)[32]) {
+                                            const uint32_t (&r)[32], const float (&bv)[32],
+                                            float rs = 1.0f) {
   const int nvalid = min(32, h.valid - col0);
   float v[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) * rs;
 
   if (a.mode == kModeRow && a.partials != nullptr) {
     float* dst = a.partials + static_cast<int64_t>(m) * h.ld + h.out_off + col0;
@@ -607,6 +677,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = q * 32 + lane;
     float* bias_s = bias_smem + ew * kHalfN;
     int it = 0;
+    if (a.norm) {
+      const int per = (a.M + gridDim.x - 1) / gridDim.x;
+      const int r0 = min(a.M, static_cast<int>(blockIdx.x) * per);
+      norm_stats(a, r0, min(a.M, r0 + per), ew * 32 + lane);
+    }
     for (int t = blockIdx.x; t < a.num_tiles; t += gridDim.x, ++it) {
       int mb, nt;
       tile_coords(a, t, mb, nt);
@@ -640,6 +715,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int m = mb * kBM + row;
         int prow;
         __nv_bfloat16* const yb = out_base(a, m, prow);
+        float rs = 1.0f;
+        if (a.norm && !__all_sync(0xffffffffu, norm_row_scale(a, m, rs, abort_flag))) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            record_timeout();
+          }
+          break;
+        }
         for (int c = 0; c < kHalfN / 32; ++c) {
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
@@ -648,7 +731,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float bv[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) bv[j] = bias_s[c * 32 + j];
-            store_chunk(a, h, m, prow, yb, c * 32, r, bv);
+            store_chunk(a, h, m, prow, yb, c * 32, r, bv, rs);
           }
         }
       }

@@ -222,6 +222,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const auto sk_flag = [&](int s) {
       return a.sk_flag + (s * 2 + static_cast<int>(rank)) * kEpiWarps + ew;
     };
+    if (a.norm) {
+      const int per = (a.M + gridDim.x - 1) / gridDim.x;
+      const int r0 = min(a.M, static_cast<int>(blockIdx.x) * per);
+      norm_stats(a, r0, min(a.M, r0 + per), ew * 32 + lane);
+    }
     for (; work_next(a, npairs, k_total, wi, w); ++it) {
       int mb, nt;
       tile_coords(a, w.tile, mb, nt);
@@ -265,6 +270,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         int prow;
         __nv_bfloat16* const yb = out_base(a, m, prow);
         const float* part = nullptr;
+        float rs = 1.0f;
+        if (a.norm && !__all_sync(0xffffffffu, norm_row_scale(a, m, rs, abort_flag))) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            record_timeout();
+          }
+          break;
+        }
         if (w.role == kWorkHead) {
           // head of a split tile: its tail's partial comes from the next pair
           int f_ok = 1;
@@ -295,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) + v.w);
             }
           }
-          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, prow, yb, c * 32, r, bv);
+          if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, prow, yb, c * 32, r, bv, rs);
         }
       }
       ptx::tc_fence_before();

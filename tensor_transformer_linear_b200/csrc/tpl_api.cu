@@ -20,6 +20,7 @@
 #include "gemm_bf16_pair.cuh"
 #include "gemm_fp32.cuh"
 #include "lmhead.cuh"
+#include "norm_fold.cuh"
 #include "rmsnorm.cuh"
 
 namespace {
@@ -171,9 +172,13 @@ void plan_stream_k(tpl::GemmArgs& a, int64_t tiles, int64_t pairs, DeviceInfo* d
   a.sk_partial = static_cast<float*>(ws->ptr);
   a.sk_flag = reinterpret_cast<uint32_t*>(static_cast<char*>(ws->ptr) +
                                           sk_partial_bytes(dev->sm_count));
+}
+
+// A fresh epoch for the flags of one launch (never 0, so zeroed flags never match).
+uint32_t next_epoch(DeviceInfo* dev) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (++dev->sk_epoch == 0) dev->sk_epoch = 1;
-  a.sk_epoch = dev->sk_epoch;
+  return dev->sk_epoch;
 }
 
 // CTA pairs (tcgen05 cta_group::2, 256-row tiles) unless M fits one 128-row
@@ -206,9 +211,14 @@ tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, DeviceInfo* dev, cudaStream_
   a.num_tiles = static_cast<int32_t>(tiles);
   a.sk_first_tile = static_cast<int32_t>(tiles);
   a.sk_units = 0;
+  a.sk_epoch = 0;
   if (pairs) {
     const int64_t npairs = std::min<int64_t>(tiles, dev->sm_count / 2);
     plan_stream_k(a, tiles, npairs, dev, ws);
+  }
+  if (a.sk_units > 0 || a.norm) a.sk_epoch = next_epoch(dev);
+  if (pairs) {
+    const int64_t npairs = std::min<int64_t>(tiles, dev->sm_count / 2);
     const int grid = 2 * static_cast<int>(npairs);
     tpl::gemm_bf16_tcgen05_pair<<<grid, tpl::kGemmThreads, tpl::kGemmPairSmemBytes, st>>>(a);
   } else {
@@ -263,6 +273,14 @@ void set_seqpar(Args& a, const SeqPar& sp) {
 
 // ------------------------------------------------------------------ column
 
+// The fused RMSNorm of a column linear (tpl_column_linear_rmsnorm): per-row
+// factors and their flags in the caller's workspace.
+struct NormFuse {
+  float eps = 0.0f;
+  float* rs = nullptr;
+  uint32_t* flag = nullptr;
+};
+
 // Token slices of the A operand held by several ranks (peer gather): rank q's
 // slice [batch][seq/tp][K] at gather[q], q < tp.
 struct GatherA {
@@ -273,7 +291,7 @@ struct GatherA {
 tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
                        const void* bias, int act, void* y, cudaStream_t st,
                        const SeqPar& sp = SeqPar{}, const GatherA* ga = nullptr,
-                       const SkWorkspace* ws = nullptr) {
+                       const SkWorkspace* ws = nullptr, const NormFuse* nf = nullptr) {
   if ((K % 8) != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 2) ||
       (bias != nullptr && !aligned(bias, 2)))
     return TPL_ERR_ALIGN;
@@ -308,6 +326,15 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
   a.mode = tpl::kModeColumn;
   a.act = act;
   a.M = static_cast<int32_t>(M);
+  if (nf != nullptr) {
+    a.norm = 1;
+    a.norm_eps = nf->eps;
+    a.norm_x = static_cast<const __nv_bfloat16*>(x);
+    a.norm_K = static_cast<int32_t>(K);
+    a.norm_ld = static_cast<int32_t>(K);
+    a.norm_rs = nf->rs;
+    a.norm_flag = nf->flag;
+  }
   set_seqpar(a, sp);
   a.k_iters = static_cast<int32_t>((K + tpl::kBK - 1) / tpl::kBK);
   a.bias = static_cast<const __nv_bfloat16*>(bias);
@@ -344,6 +371,39 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
   return TPL_OK;
 }
 
+// Launches the fp32 kernel over n_tiles x mb output tiles, splitting each
+// tile's K steps over a cluster of up to 8 CTAs (grid z) when there are too
+// few tiles to fill the GPU (the tiny MLP: 32 and 8 tiles).
+tpl_status launch_fp32(const tpl::F32Args& a, int64_t mb, cudaStream_t st) {
+  const int64_t tiles = static_cast<int64_t>(a.n_tiles) * mb;
+  int split = 1;
+  while (split < tpl::kF32MaxSplit && tiles * split < 128 && split * 2 <= a.k_steps) split *= 2;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(a.n_tiles), static_cast<unsigned>(mb),
+                     static_cast<unsigned>(split));
+  cfg.blockDim = dim3(tpl::kF32Threads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(split);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, tpl::gemm_fp32_simt, a) != cudaSuccess) return TPL_ERR_CUDA;
+  return launched();
+}
+
+// 32-wide K steps of ranks r0 .. r1-1 (row mode).
+int32_t fp32_row_steps(const tpl::F32Args& a) {
+  int64_t n = 0;
+  for (int r = a.r0; r < a.r1; ++r)
+    n += (a.koff[r + 1] - a.koff[r] + tpl::kF32BK - 1) / tpl::kF32BK;
+  return static_cast<int32_t>(n);
+}
+
 tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
                        const void* bias, int act, void* y, cudaStream_t st,
                        const SeqPar& sp = SeqPar{}) {
@@ -360,6 +420,8 @@ tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t
   a.w = static_cast<const float*>(w);
   a.bias = static_cast<const float*>(bias);
   a.y = static_cast<float*>(y);
+  a.k_steps = static_cast<int32_t>((K + tpl::kF32BK - 1) / tpl::kF32BK);
+  a.vec = (K % 4 == 0 && aligned(x, 16) && aligned(w, 16)) ? 1 : 0;
   std::vector<F32Piece> pieces;
   for (int r = 0; r < p->tp_size; ++r)
     for (int j = 0; j < p->n_sub; ++j) {
@@ -384,9 +446,7 @@ tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t
       a.pieces[i - b] = c;
     }
     a.n_tiles = nt;
-    dim3 grid(nt, static_cast<unsigned>(mb));
-    tpl::gemm_fp32_simt<<<grid, tpl::kF32Threads, 0, st>>>(a);
-    tpl_status s = launched();
+    tpl_status s = launch_fp32(a, mb, st);
     if (s != TPL_OK) return s;
   }
   return TPL_OK;
@@ -498,17 +558,21 @@ tpl_status row_fp32(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
   a.w = static_cast<const float*>(w);
   a.y = static_cast<float*>(y);
   a.koff[0] = 0;
-  for (int r = 0; r < tp; ++r) a.koff[r + 1] = a.koff[r] + k_w[r];
+  bool vec = aligned(h, 16) && aligned(w, 16);
+  for (int r = 0; r < tp; ++r) {
+    a.koff[r + 1] = a.koff[r] + k_w[r];
+    vec = vec && (k_w[r] % 4 == 0);
+  }
+  a.vec = vec ? 1 : 0;
   a.n_tiles = static_cast<int32_t>((N + tpl::kF32BN - 1) / tpl::kF32BN);
   const int64_t mb = (M + tpl::kF32BM - 1) / tpl::kF32BM;
   if (mb > 65535) return TPL_ERR_SHAPE;
-  dim3 grid(a.n_tiles, static_cast<unsigned>(mb));
   a.r0 = 0;
   a.r1 = tp;
+  a.k_steps = fp32_row_steps(a);
   a.bias = static_cast<const float*>(bias);
   a.residual = static_cast<const float*>(residual);
-  tpl::gemm_fp32_simt<<<grid, tpl::kF32Threads, 0, st>>>(a);
-  tpl_status s = launched();
+  tpl_status s = launch_fp32(a, mb, st);
   if (s != TPL_OK) return s;
   if (partials != nullptr) {
     a.bias = nullptr;
@@ -516,9 +580,9 @@ tpl_status row_fp32(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
     for (int r = 0; r < tp; ++r) {
       a.r0 = r;
       a.r1 = r + 1;
+      a.k_steps = fp32_row_steps(a);
       a.partials = partials + static_cast<int64_t>(r) * M * N;
-      tpl::gemm_fp32_simt<<<grid, tpl::kF32Threads, 0, st>>>(a);
-      if ((s = launched()) != TPL_OK) return s;
+      if ((s = launch_fp32(a, mb, st)) != TPL_OK) return s;
     }
   }
   return TPL_OK;
@@ -706,6 +770,65 @@ static tpl_status row_entry(const void* h, const int64_t* k_w, int32_t tp, int64
   return dt == TPL_BF16
              ? row_bf16(h, k_w, tp, M, N, w, bias, residual, y, partials, st, SeqPar{}, nullptr, ws)
              : row_fp32(h, k_w, tp, M, N, w, bias, residual, y, partials, st);
+}
+
+static size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+tpl_status tpl_column_linear_rmsnorm_workspace_size(int64_t M, size_t* bytes) {
+  if (bytes == nullptr) return TPL_ERR_NULL;
+  if (M < 0 || M > INT32_MAX) return TPL_ERR_SHAPE;
+  size_t sk = 0;
+  tpl_status s = tpl_gemm_workspace_size(&sk);
+  if (s != TPL_OK) return s;
+  *bytes = sk + 2 * round256(static_cast<size_t>(M) * 4);
+  return TPL_OK;
+}
+
+tpl_status tpl_column_linear_rmsnorm(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                                     const void* w, const void* bias, float eps, tpl_act act,
+                                     void* y, void* workspace, size_t ws_bytes, void* stream) {
+  if (p == nullptr) return TPL_ERR_NULL;
+  if (!act_ok(act)) return TPL_ERR_DTYPE;
+  tpl_status s = check_partition(p);
+  if (s != TPL_OK) return s;
+  if (M < 0 || K < 1 || M > INT32_MAX || K > INT32_MAX || !(eps >= 0.0f)) return TPL_ERR_SHAPE;
+  if (M == 0) return TPL_OK;
+  if (x == nullptr || w == nullptr || y == nullptr || workspace == nullptr) return TPL_ERR_NULL;
+  if (!aligned(workspace, 256)) return TPL_ERR_ALIGN;
+  size_t need = 0;
+  if ((s = tpl_column_linear_rmsnorm_workspace_size(M, &need)) != TPL_OK) return s;
+  if (ws_bytes < need) return TPL_ERR_SHAPE;
+  size_t sk = 0;
+  tpl_gemm_workspace_size(&sk);
+  SkWorkspace ws;
+  ws.ptr = workspace;
+  ws.bytes = sk;
+  NormFuse nf;
+  nf.eps = eps;
+  nf.rs = reinterpret_cast<float*>(static_cast<char*>(workspace) + sk);
+  nf.flag = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + sk +
+                                        round256(static_cast<size_t>(M) * 4));
+  return column_bf16(p, x, M, K, w, bias, act, y, static_cast<cudaStream_t>(stream), SeqPar{},
+                     nullptr, &ws, &nf);
+}
+
+tpl_status tpl_fold_norm_scale(const void* w, int64_t rows, int64_t K, const float* scale,
+                               int32_t centered, void* w_out, void* stream) {
+  if (rows < 0 || K < 1 || rows > INT32_MAX || K > INT32_MAX) return TPL_ERR_SHAPE;
+  if (rows == 0) return TPL_OK;
+  if (w == nullptr || scale == nullptr || w_out == nullptr) return TPL_ERR_NULL;
+  if (K % 8 != 0 || !aligned(w, 16) || !aligned(w_out, 16) || !aligned(scale, 16))
+    return TPL_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  tpl_status s = device_info(&dev);
+  if (s != TPL_OK) return s;
+  const int64_t vecs = rows * (K / 8);
+  const int grid = static_cast<int>(std::min<int64_t>((vecs + 255) / 256,
+                                                      static_cast<int64_t>(dev->sm_count) * 8));
+  tpl::fold_norm_scale_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(w), rows, K, scale, centered,
+      static_cast<__nv_bfloat16*>(w_out));
+  return launched();
 }
 
 tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,

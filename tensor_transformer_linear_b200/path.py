@@ -8,12 +8,15 @@ residual section.  Each step is one call into libtpl.so.
 """
 from __future__ import annotations
 
+import functools
 from typing import Callable, List, Optional, Sequence
 
 import torch
 
 from ._tpl import (Partition, TplError, tpl_argmax_merge, tpl_column_linear,
-                   tpl_column_linear_gather, tpl_get_device_status, tpl_lmhead_argmax,
+                   tpl_column_linear_gather, tpl_column_linear_rmsnorm,
+                   tpl_column_linear_rmsnorm_workspace_size, tpl_fold_norm_scale,
+                   tpl_get_device_status, tpl_lmhead_argmax,
                    tpl_lmhead_workspace_size, tpl_partition_subparams, tpl_reduce_slots,
                    tpl_reduce_slots_allgather, tpl_rmsnorm, tpl_row_linear_reduce,
                    tpl_row_linear_scatter)
@@ -42,12 +45,17 @@ def pack_row_weight(w2_full: torch.Tensor, k_w: Sequence[int]) -> torch.Tensor:
 
 
 class TPMLP:
-    """One TP MLP block: ``[x +] c_proj(act(c_fc(rmsnorm(x))))``, all shards on one GPU."""
+    """One TP MLP block: ``[x +] c_proj(act(c_fc(rmsnorm(x))))``, all shards on one GPU.
+
+    ``fused_norm``: the RMSNorm runs inside the c_fc GEMM
+    (tpl_column_linear_rmsnorm): its scale is folded into W1 here, once, and no
+    normalised copy of x is written.  Otherwise tpl_rmsnorm writes one first.
+    """
 
     def __init__(self, w1: torch.Tensor, w2_full: torch.Tensor, tp: int, act: str,
                  scale: Optional[torch.Tensor] = None, centered: bool = False,
                  norm: bool = True, residual: bool = False, eps: float = 1e-6,
-                 workspace: Optional[torch.Tensor] = None):
+                 workspace: Optional[torch.Tensor] = None, fused_norm: bool = False):
         self.inter, self.hidden = w1.shape
         self.part = tpl_partition_subparams([self.inter], tp, 1)
         self.k_w = [self.part.shard_width[r] for r in range(tp)]
@@ -56,7 +64,11 @@ class TPMLP:
         self.act, self.scale, self.centered = act, scale, centered
         self.norm, self.residual, self.eps = norm, residual, eps
         self.workspace = workspace   # stream-K workspace of the two GEMMs (or None)
+        self.fused_norm = bool(fused_norm and norm)
+        if self.fused_norm and scale is not None:
+            self.w1 = tpl_fold_norm_scale(self.w1, scale, centered)
         self._bufs = {}
+        self._norm_ws = None
 
     def _buf(self, name, numel, like):
         b = self._bufs.get(name)
@@ -65,8 +77,26 @@ class TPMLP:
             self._bufs[name] = b
         return b[:numel]
 
+    def norm_workspace(self, M: int, device) -> torch.Tensor:
+        """The fused norm's workspace for M rows (zero-filled when it grows)."""
+        need = tpl_column_linear_rmsnorm_workspace_size(M)
+        if self._norm_ws is None or self._norm_ws.numel() < need:
+            self._norm_ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        return self._norm_ws
+
     def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
         M = x.numel() // self.hidden
+        if self.fused_norm:
+            h = self._buf("h", M * self.inter, x)
+            ws = self.norm_workspace(M, x.device)
+            tpl_column_linear_rmsnorm(self.part, x.view(M, self.hidden), self.w1, None, self.eps,
+                                      self.act, ws, y=h, stream=stream)
+            if out is None:
+                out = torch.empty((M, self.hidden), dtype=x.dtype, device=x.device)
+            tpl_row_linear_reduce(h, self.k_w, M, self.w2, None,
+                                  x.view(M, self.hidden) if self.residual else None, y=out,
+                                  stream=stream, workspace=ws)
+            return out
         xn = x
         if self.norm:
             xn = self._buf("xn", x.numel(), x).view(M, self.hidden)
@@ -289,7 +319,8 @@ class TPRankMLP:
     def __init__(self, w1_shard: torch.Tensor, w2_shard: torch.Tensor, rank: int, tp: int,
                  act: str, xn: PeerBuffers, recv: PeerBuffers, barrier: Callable,
                  scale: Optional[torch.Tensor] = None, centered: bool = False,
-                 eps: float = 1e-6, ops: Optional[dict] = None):
+                 eps: float = 1e-6, ops: Optional[dict] = None,
+                 workspace: Optional[torch.Tensor] = None):
         self.w1, self.w2 = w1_shard.contiguous(), w2_shard.contiguous()
         self.rank, self.tp, self.act = rank, tp, act
         self.xn, self.recv, self.barrier = xn, recv, barrier
@@ -299,27 +330,45 @@ class TPRankMLP:
         self.rmsnorm = ops.get("rmsnorm", tpl_rmsnorm)
         self.column = ops.get("column", tpl_column_linear_gather)
         self.scatter = ops.get("scatter", tpl_row_linear_scatter)
+        if workspace is not None:   # stream-K workspace of the two GEMMs
+            if "column" not in ops:
+                self.column = functools.partial(tpl_column_linear_gather, workspace=workspace)
+            if "scatter" not in ops:
+                self.scatter = functools.partial(tpl_row_linear_scatter, workspace=workspace)
         self.reduce = ops.get("reduce", tpl_reduce_slots)
         self._h = None
 
-    def __call__(self, x_slice: torch.Tensor, batch: int, seq: int, stream=None) -> torch.Tensor:
+    STEPS = ("rmsnorm", "barrier_xn", "column_gather", "row_scatter", "barrier_slots",
+             "reduce_slots", "barrier_done")
+
+    def __call__(self, x_slice: torch.Tensor, batch: int, seq: int, stream=None,
+                 on_step: Optional[Callable] = None) -> torch.Tensor:
         """``x_slice`` ``[batch*seq/tp, hidden]``: this rank's tokens of the residual
-        stream, updated in place to ``x + MLP(RMSNorm(x))``."""
+        stream, updated in place to ``x + MLP(RMSNorm(x))``.  ``on_step(i)`` is
+        called before step i of :attr:`STEPS` (e.g. to record a CUDA event)."""
         H, tp = self.w2.shape[0], self.tp
         M = batch * seq
         sp_rows(batch, seq, tp)
+        mark = on_step or (lambda i: None)
         if self._h is None or self._h.numel() < M * self.w1.shape[0]:
             self._h = torch.empty(M * self.w1.shape[0], dtype=x_slice.dtype,
                                   device=x_slice.device)
+        mark(0)
         self.rmsnorm(x_slice, self.scale, self.centered, self.eps, y=self.xn.local,
                      stream=stream)
+        mark(1)
         self.barrier(stream)
+        mark(2)
         h = self.column(self.part, self.xn.addrs, batch, seq, self.w1, None, self.act,
                         y=self._h, stream=stream)
+        mark(3)
         self.scatter(h.view(M, -1), self.w2, batch, seq, self.rank, tp, self.recv.addrs,
                      stream=stream)
+        mark(4)
         self.barrier(stream)
+        mark(5)
         self.reduce(self.recv.local, tp, H, None, x_slice, x_slice, stream=stream)
+        mark(6)
         self.barrier(stream)
         return x_slice
 
