@@ -242,7 +242,6 @@ class Block:
         self.flops = 0.0
         self.gemm_flops = 0.0
         self.launches = []        # (part name, callable(stream)), in launch order
-        self.gemm_ws = T.gemm_workspace(dev)   # stream-K workspace of the step's GEMMs
         # Attributes holding each step's inputs and results; every launch reads
         # them at call time, so the end-to-end pipeline can rotate buffer sets.
         self.io_in, self.io_out = [], []
@@ -254,8 +253,7 @@ class Block:
             self.qpart = T.tpl_partition_subparams(q.sub_sizes, q.tp, q.align)
             self.qy = torch.empty(q.M * q.out, dtype=torch.bfloat16, device=dev)
             self.launches.append(("qkv_column", lambda s: T.tpl_column_linear(
-                self.qpart, self.qx, self.qw, self.qb, "none", y=self.qy, stream=s,
-                workspace=self.gemm_ws)))
+                self.qpart, self.qx, self.qw, self.qb, "none", y=self.qy, stream=s)))
             self.flops += q.flops()
             self.gemm_flops += q.flops()
             self.io_in.append("qx")
@@ -283,12 +281,10 @@ class Block:
                 self.launches += [
                     ("rmsnorm", self.alone_launches["rmsnorm"]),
                     ("mlp_column_gelu", lambda s: T.tpl_column_linear(
-                        mlp.part, self.xn, mlp.w1, None, m.act, y=self.h, stream=s,
-                        workspace=self.gemm_ws))]
+                        mlp.part, self.xn, mlp.w1, None, m.act, y=self.h, stream=s))]
             self.launches += [
                 ("mlp_row_reduce", lambda s: T.tpl_row_linear_reduce(
-                    self.h, mlp.k_w, m.M, mlp.w2, None, None, y=self.my, stream=s,
-                    workspace=self.gemm_ws))]
+                    self.h, mlp.k_w, m.M, mlp.w2, None, None, y=self.my, stream=s))]
             self.flops += m.flops()
             self.gemm_flops += m.flops()
             self.io_in.append("mx")
@@ -346,9 +342,8 @@ class Stack:
         self.layers = [T.TPMLP(C.mlp_w1(w, l, dev), C.mlp_w2(w, l, dev), w.tp, w.act,
                                norm=True, residual=True, fused_norm=FUSED_NORM)
                        for l in range(w.layers)]
-        # one workspace for every layer (the layers run one after another)
-        self.ws = (self.layers[0].norm_workspace(w.M, dev) if FUSED_NORM
-                   else T.gemm_workspace(dev))
+        # the fused norm's workspace, one for every layer (they run one after another)
+        self.ws = self.layers[0].norm_workspace(w.M, dev) if FUSED_NORM else None
         self.flops = w.flops()
         self.gemm_flops = w.flops()
         self.parts = []
@@ -377,11 +372,11 @@ class Stack:
                 T.tpl_rmsnorm(self.x, None, False, 1e-6, y=xn, stream=stream)
                 mark(i + 1)
                 T.tpl_column_linear(layer.part, xn, layer.w1, None, layer.act, y=h,
-                                    stream=stream, workspace=self.ws)
+                                    stream=stream)
                 i += 2
             mark(i)
             T.tpl_row_linear_reduce(h, layer.k_w, M, layer.w2, None, self.x, y=self.x,
-                                    stream=stream, workspace=self.ws)
+                                    stream=stream)
             i += 1
         mark(i)
 
@@ -482,7 +477,6 @@ class NextRows:
             self.hbuf = torch.empty(tp * M * kr, dtype=torch.bfloat16, device=dev)
             self.recv = [torch.empty(tp * rows * N, dtype=torch.bfloat16, device=dev)
                          for _ in range(tp)]
-            self.ws = T.gemm_workspace(dev)
 
             def norm_all(s):
                 for q in range(tp):
@@ -494,13 +488,12 @@ class NextRows:
                 for r in range(tp):
                     T.tpl_column_linear_gather(self.p_rank, slices, b, sq,
                                                self.w1[r * kr:(r + 1) * kr], None, m.act,
-                                               y=hs[r], stream=s, workspace=self.ws)
+                                               y=hs[r], stream=s)
 
             def scatter_all(s):
                 hs, ws = self.hbuf.view(tp, M, kr), self.w2p.view(tp, N, kr)
                 for r in range(tp):
-                    T.tpl_row_linear_scatter(hs[r], ws[r], b, sq, r, tp, self.recv, stream=s,
-                                             workspace=self.ws)
+                    T.tpl_row_linear_scatter(hs[r], ws[r], b, sq, r, tp, self.recv, stream=s)
 
             def reduce_all(s):
                 for q in range(tp):
@@ -564,7 +557,7 @@ class RankTP:
     kind = "tp_ranks"
 
     def __init__(self, dev, rank, world, ops=None, exchange=None, barrier=None,
-                 workload=None, workspace=True):
+                 workload=None):
         from tensor_transformer_linear_b200 import path
         m = workload or C.TP_MLP
         self.m, self.rank, self.tp = m, rank, world
@@ -582,13 +575,8 @@ class RankTP:
         recv = exchange(torch.empty(path.recv_buffer_numel(world, b, sq, H), dtype=self.x.dtype,
                                     device=self.x.device))
         barrier = barrier or path.stream_barrier(device=dev)
-        ws = None
-        if workspace and ops is None:
-            import tensor_transformer_linear_b200 as T
-            ws = T.gemm_workspace(dev)
         self.block = path.TPRankMLP(w1, w2, rank, world, m.act, xn, recv, barrier,
-                                    scale=C.mlp_scale(m, 0, dev), centered=True, ops=ops,
-                                    workspace=ws)
+                                    scale=C.mlp_scale(m, 0, dev), centered=True, ops=ops)
         self.parts = ["rank_" + s for s in path.TPRankMLP.STEPS]
         self.flops = m.flops()                 # the whole job's work per step
         self.gemm_flops = m.flops() / world   # this rank's GEMMs

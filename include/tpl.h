@@ -164,37 +164,6 @@ tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, 
                                  const void* residual, tpl_dtype dt, void* y, float* partials,
                                  void* stream);
 
-/*
- * The same column- and row-parallel linears with a stream-K workspace.  (The
- * pages split tensors over devices; splitting a GEMM's last tile waves over
- * the SMs is this library's own scheduling.)  A persistent GEMM deals whole
- * output tiles to its CTA pairs in waves; when the last wave is only partly
- * full, most SMs would idle through it.  With a workspace, the last full wave
- * and the partial one are dealt out by K steps instead (at least one tile's
- * worth per CTA pair), so a tile may be split between two pairs: the pair
- * that computes the tile's K tail stores its fp32 partial in the workspace,
- * the pair that computes the head adds it in the epilogue.  The sums are in
- * fp32 either way; only the order of the additions changes for those tiles.
- *
- *   workspace  device, tpl_gemm_workspace_size() bytes (ws_bytes), 256-byte
- *              aligned, ZERO-FILLED before its first use; reusable across
- *              calls without clearing.  A smaller ws_bytes runs the plain
- *              schedule.  Calls whose work overlaps on the GPU (different
- *              streams) must not share one workspace.  NULL: TPL_ERR_NULL.
- *   Other arguments, results and errors as tpl_column_linear /
- *   tpl_row_linear_reduce.  fp32, the single-CTA kernel (M <= 128) and the
- *   per-rank `partials` check run the plain schedule.
- */
-tpl_status tpl_gemm_workspace_size(size_t* bytes); /* for the current device */
-
-tpl_status tpl_column_linear_ws(const tpl_partition* p, const void* x, int64_t M, int64_t K,
-                                const void* w, const void* bias, tpl_dtype dt, tpl_act act,
-                                void* y, void* workspace, size_t ws_bytes, void* stream);
-
-tpl_status tpl_row_linear_reduce_ws(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
-                                    int64_t N, const void* w, const void* bias,
-                                    const void* residual, tpl_dtype dt, void* y, float* partials,
-                                    void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Column-parallel linear of RMSNorm(x) with the norm fused into the GEMM
@@ -211,11 +180,11 @@ tpl_status tpl_row_linear_reduce_ws(const void* h, const int64_t* k_w, int32_t t
  *   x          device bf16 [M][K], the raw activations.
  *   w          device bf16 [p->logical_out][K], the weight with g folded in.
  *   bias, act, y, p   as tpl_column_linear.   eps >= 0.
- *   workspace  device, tpl_column_linear_rmsnorm_workspace_size(M) bytes,
- *              256-byte aligned, ZERO-FILLED before its first use, reusable;
- *              its first tpl_gemm_workspace_size() bytes also serve as the
- *              stream-K workspace of this call.  Calls whose work overlaps on
- *              the GPU must not share one.
+ *   workspace  device, tpl_column_linear_rmsnorm_workspace_size(M) bytes
+ *              (the per-row factors and their ready flags), 256-byte aligned,
+ *              ZERO-FILLED before its first use, reusable without clearing
+ *              (each call stamps its flags with a value fresh to that call).
+ *              Calls whose work overlaps on the GPU must not share one.
  * bf16 only (K % 8 == 0, 16-byte aligned x and w).  Errors as
  * tpl_column_linear, plus TPL_ERR_SHAPE for a short workspace.
  */
@@ -444,21 +413,6 @@ tpl_status tpl_row_linear_scatter(const void* h, int64_t K, int64_t batch, int64
                                   const void* w, int32_t rank, int32_t tp, void* const* peer,
                                   void* stream);
 
-/*
- * tpl_column_linear_gather and tpl_row_linear_scatter with a stream-K
- * workspace (see tpl_column_linear_ws): one rank's shard of an MLP split over
- * 8 GPUs is a few tile waves (8192 x 1792: 224 tiles over 74 CTA pairs), so
- * its partial last wave costs the most.  Arguments otherwise as above.
- */
-tpl_status tpl_column_linear_gather_ws(const tpl_partition* p, void* const* peer_x, int32_t tp,
-                                       int64_t batch, int64_t seq, int64_t K, const void* w,
-                                       const void* bias, tpl_act act, void* y, void* workspace,
-                                       size_t ws_bytes, void* stream);
-
-tpl_status tpl_row_linear_scatter_ws(const void* h, int64_t K, int64_t batch, int64_t seq,
-                                     int64_t N, const void* w, int32_t rank, int32_t tp,
-                                     void* const* peer, void* workspace, size_t ws_bytes,
-                                     void* stream);
 
 /*
  * The reduction step of the reduce-scatter above, on the rank that owns a

@@ -34,8 +34,6 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_column_linear_allgather", "tpl_swiglu_column_linear", "tpl_embedding_lookup",
             "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
             "tpl_argmax_merge", "tpl_column_linear_gather", "tpl_reduce_slots_allgather",
-            "tpl_gemm_workspace_size", "tpl_column_linear_ws", "tpl_row_linear_reduce_ws",
-            "tpl_column_linear_gather_ws", "tpl_row_linear_scatter_ws",
             "tpl_column_linear_rmsnorm_workspace_size", "tpl_column_linear_rmsnorm",
             "tpl_fold_norm_scale")
 
@@ -104,15 +102,6 @@ def lib():
         L.tpl_argmax_merge.argtypes = [vp, vp, i32, i64, i64, vp, vp]
         L.tpl_column_linear_gather.argtypes = [ctypes.POINTER(Partition), ctypes.POINTER(vp), i32,
                                                i64, i64, i64, vp, vp, i32, vp, vp]
-        L.tpl_gemm_workspace_size.argtypes = [ctypes.POINTER(sz)]
-        L.tpl_column_linear_ws.argtypes = [ctypes.POINTER(Partition), vp, i64, i64, vp, vp, i32,
-                                           i32, vp, vp, sz, vp]
-        L.tpl_row_linear_reduce_ws.argtypes = [vp, ctypes.POINTER(i64), i32, i64, i64, vp, vp, vp,
-                                               i32, vp, vp, vp, sz, vp]
-        L.tpl_column_linear_gather_ws.argtypes = [ctypes.POINTER(Partition), ctypes.POINTER(vp),
-                                                  i32, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp]
-        L.tpl_row_linear_scatter_ws.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32,
-                                                ctypes.POINTER(vp), vp, sz, vp]
         L.tpl_column_linear_rmsnorm_workspace_size.argtypes = [i64, ctypes.POINTER(sz)]
         L.tpl_column_linear_rmsnorm.argtypes = [ctypes.POINTER(Partition), vp, i64, i64, vp, vp,
                                                 ctypes.c_float, i32, vp, vp, sz, vp]
@@ -163,22 +152,6 @@ def tpl_partition_subparams(sub_sizes: Sequence[int], tp: int, align: int = 1) -
     return p
 
 
-def tpl_gemm_workspace_size() -> int:
-    """Bytes of a stream-K workspace for the current device."""
-    n = ctypes.c_size_t(0)
-    _check(lib().tpl_gemm_workspace_size(ctypes.byref(n)), "tpl_gemm_workspace_size")
-    return int(n.value)
-
-
-def gemm_workspace(device="cuda") -> torch.Tensor:
-    """A zero-filled stream-K workspace for the GEMM calls' ``workspace=``
-    (reusable across calls on one stream; calls that overlap on the GPU need one
-    each)."""
-    with torch.cuda.device(device):
-        n = tpl_gemm_workspace_size()
-    return torch.zeros(n, dtype=torch.uint8, device=device)
-
-
 def _ws(workspace: Optional[torch.Tensor]):
     _cuda(workspace, "workspace")
     return _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size())
@@ -186,12 +159,8 @@ def _ws(workspace: Optional[torch.Tensor]):
 
 def tpl_column_linear(p: Partition, x: torch.Tensor, w: torch.Tensor,
                       bias: Optional[torch.Tensor] = None, act: str = "none",
-                      y: Optional[torch.Tensor] = None, stream=None,
-                      workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Returns y holding every rank's shard (rank r: ``[M, shard_width[r]]`` at M*shard_base[r]).
-
-    With a ``workspace`` (see :func:`gemm_workspace`) the GEMM's last tile waves
-    are split over the SMs by K steps (tpl_column_linear_ws)."""
+                      y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Returns y holding every rank's shard (rank r: ``[M, shard_width[r]]`` at M*shard_base[r])."""
     _cuda(x, "x")
     dt = x.dtype
     _cuda(w, "w", dt)
@@ -205,14 +174,9 @@ def tpl_column_linear(p: Partition, x: torch.Tensor, w: torch.Tensor,
         raise ValueError("y or w has the wrong size")
     if bias is not None and bias.numel() != p.logical_out:
         raise ValueError("bias size does not match the partition's output size")
-    if workspace is None:
-        _check(lib().tpl_column_linear(ctypes.byref(p), _ptr(x), M, K, _ptr(w), _ptr(bias),
-                                       DTYPE[dt], ACT[act], _ptr(y), _stream(stream)),
-               "tpl_column_linear")
-    else:
-        _check(lib().tpl_column_linear_ws(ctypes.byref(p), _ptr(x), M, K, _ptr(w), _ptr(bias),
-                                          DTYPE[dt], ACT[act], _ptr(y), *_ws(workspace),
-                                          _stream(stream)), "tpl_column_linear_ws")
+    _check(lib().tpl_column_linear(ctypes.byref(p), _ptr(x), M, K, _ptr(w), _ptr(bias),
+                                   DTYPE[dt], ACT[act], _ptr(y), _stream(stream)),
+           "tpl_column_linear")
     return y
 
 
@@ -225,8 +189,7 @@ def tpl_column_linear_rmsnorm_workspace_size(M: int) -> int:
 
 def rmsnorm_linear_workspace(M: int, device="cuda") -> torch.Tensor:
     """A zero-filled workspace for tpl_column_linear_rmsnorm with up to M rows
-    (reusable across calls on one stream); its first tpl_gemm_workspace_size()
-    bytes are a stream-K workspace for the other GEMM calls too."""
+    (reusable across calls on one stream)."""
     with torch.cuda.device(device):
         n = tpl_column_linear_rmsnorm_workspace_size(M)
     return torch.zeros(n, dtype=torch.uint8, device=device)
@@ -276,10 +239,8 @@ def tpl_row_linear_reduce(h: torch.Tensor, k_w: Sequence[int], M: int, w: torch.
                           bias: Optional[torch.Tensor] = None,
                           residual: Optional[torch.Tensor] = None,
                           y: Optional[torch.Tensor] = None,
-                          partials: Optional[torch.Tensor] = None, stream=None,
-                          workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """``Y = sum_r H_r W2_r^T (+ bias) (+ residual)``; h and w are rank-major packed blocks.
-    ``workspace``: as for :func:`tpl_column_linear`."""
+                          partials: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``Y = sum_r H_r W2_r^T (+ bias) (+ residual)``; h and w are rank-major packed blocks."""
     _cuda(h, "h")
     dt = h.dtype
     _cuda(w, "w", dt)
@@ -300,15 +261,9 @@ def tpl_row_linear_reduce(h: torch.Tensor, k_w: Sequence[int], M: int, w: torch.
         if partials.numel() != tp * M * N:
             raise ValueError("partials must hold tp * M * N floats")
     kw = (ctypes.c_int64 * tp)(*[int(k) for k in k_w])
-    if workspace is None:
-        _check(lib().tpl_row_linear_reduce(_ptr(h), kw, tp, int(M), int(N), _ptr(w), _ptr(bias),
-                                           _ptr(residual), DTYPE[dt], _ptr(y), _ptr(partials),
-                                           _stream(stream)), "tpl_row_linear_reduce")
-    else:
-        _check(lib().tpl_row_linear_reduce_ws(_ptr(h), kw, tp, int(M), int(N), _ptr(w),
-                                              _ptr(bias), _ptr(residual), DTYPE[dt], _ptr(y),
-                                              _ptr(partials), *_ws(workspace), _stream(stream)),
-               "tpl_row_linear_reduce_ws")
+    _check(lib().tpl_row_linear_reduce(_ptr(h), kw, tp, int(M), int(N), _ptr(w), _ptr(bias),
+                                       _ptr(residual), DTYPE[dt], _ptr(y), _ptr(partials),
+                                       _stream(stream)), "tpl_row_linear_reduce")
     return y
 
 
@@ -506,8 +461,7 @@ def _addresses(bufs: Sequence, name: str, dtype=torch.bfloat16):
 def tpl_column_linear_gather(p: Partition, peer_x: Sequence, batch: int, seq: int,
                              w: torch.Tensor, bias: Optional[torch.Tensor] = None,
                              act: str = "none", y: Optional[torch.Tensor] = None,
-                             stream=None, workspace: Optional[torch.Tensor] = None
-                             ) -> torch.Tensor:
+                             stream=None) -> torch.Tensor:
     """This rank's column shard over every rank's token slice ``peer_x[q]``
     (``[batch, seq // tp, K]`` bf16, a CUDA tensor or a mapped peer address)."""
     _cuda(w, "w", torch.bfloat16)
@@ -528,23 +482,15 @@ def tpl_column_linear_gather(p: Partition, peer_x: Sequence, batch: int, seq: in
     _cuda(y, "y", torch.bfloat16)
     if y.numel() < M * p.logical_out:
         raise ValueError("y must hold batch * seq * logical_out elements")
-    if workspace is None:
-        _check(lib().tpl_column_linear_gather(ctypes.byref(p), _addresses(peer_x, "peer_x"),
-                                              int(tp), int(batch), int(seq), int(K), _ptr(w),
-                                              _ptr(bias), ACT[act], _ptr(y), _stream(stream)),
-               "tpl_column_linear_gather")
-    else:
-        _check(lib().tpl_column_linear_gather_ws(ctypes.byref(p), _addresses(peer_x, "peer_x"),
-                                                 int(tp), int(batch), int(seq), int(K), _ptr(w),
-                                                 _ptr(bias), ACT[act], _ptr(y), *_ws(workspace),
-                                                 _stream(stream)),
-               "tpl_column_linear_gather_ws")
+    _check(lib().tpl_column_linear_gather(ctypes.byref(p), _addresses(peer_x, "peer_x"),
+                                          int(tp), int(batch), int(seq), int(K), _ptr(w),
+                                          _ptr(bias), ACT[act], _ptr(y), _stream(stream)),
+           "tpl_column_linear_gather")
     return y
 
 
 def tpl_row_linear_scatter(h: torch.Tensor, w: torch.Tensor, batch: int, seq: int, rank: int,
-                           tp: int, peers: Sequence, stream=None,
-                           workspace: Optional[torch.Tensor] = None) -> None:
+                           tp: int, peers: Sequence, stream=None) -> None:
     """This rank's row-parallel shard, written into every owner rank's receive buffer.
 
     ``peers[q]`` is rank q's receive buffer ``[tp][batch][seq // tp][N]`` bf16:
@@ -569,14 +515,9 @@ def tpl_row_linear_scatter(h: torch.Tensor, w: torch.Tensor, batch: int, seq: in
         else:
             addr.append(int(p))
     arr = (ctypes.c_void_p * tp)(*addr)
-    if workspace is None:
-        _check(lib().tpl_row_linear_scatter(_ptr(h), int(K), int(batch), int(seq), int(N),
-                                            _ptr(w), int(rank), int(tp), arr, _stream(stream)),
-               "tpl_row_linear_scatter")
-    else:
-        _check(lib().tpl_row_linear_scatter_ws(_ptr(h), int(K), int(batch), int(seq), int(N),
-                                               _ptr(w), int(rank), int(tp), arr, *_ws(workspace),
-                                               _stream(stream)), "tpl_row_linear_scatter_ws")
+    _check(lib().tpl_row_linear_scatter(_ptr(h), int(K), int(batch), int(seq), int(N), _ptr(w),
+                                        int(rank), int(tp), arr, _stream(stream)),
+           "tpl_row_linear_scatter")
 
 
 def tpl_reduce_slots(recv: torch.Tensor, tp: int, N: int, bias: Optional[torch.Tensor] = None,

@@ -81,26 +81,15 @@ struct GemmArgs {
   // odd tiles, so a tile wave starts on the K slices the wave before it read
   // last (still in L2) when the two waves share operand blocks.
   int32_t k_serp;
-  // Stream-K (CTA-pair kernel): tiles below sk_first_tile (a multiple of the
-  // pair count) are whole work items, dealt round-robin as before.  The K steps
-  // of the tiles from sk_first_tile on are dealt out in contiguous runs of
-  // sk_units per pair (sk_units >= the K steps of one tile), so a tile is split
-  // between at most two pairs: pair p + 1 computes its K tail first thing
-  // (storing the fp32 partial in sk_partial, slot p + 1, then raising its
-  // flags to sk_epoch) and pair p its head last, adding that partial before
-  // the epilogue.  sk_units == 0: no stream-K phase.
-  int32_t sk_first_tile;
-  int32_t sk_units;
-  uint32_t sk_epoch;
-  float* sk_partial;  // [pairs][2 CTAs][kEpiWarps][4 chunks][32 rows][32 columns]
-  uint32_t* sk_flag;  // [pairs][2 CTAs][kEpiWarps]
   // Fused RMSNorm (column mode, google-research allgather_layernorm): A is
   // the raw x and the norm's scale is folded into the weight, so row m of the
   // output is act(norm_rs[m] * (x W'^T)[m] + b).  Before its first epilogue,
   // every CTA's epilogue warps compute norm_rs[m] = rsqrt(mean(x[m]^2) + eps)
   // for their share of the rows (in fp32, from bf16 x) and raise norm_flag[m]
-  // to sk_epoch; an epilogue scales row m once its flag is up.
+  // to norm_epoch (a value fresh to every launch, so a flag left by an earlier
+  // launch never matches); an epilogue scales row m once its flag is up.
   int32_t norm;
+  uint32_t norm_epoch;
   float norm_eps;
   const __nv_bfloat16* norm_x;  // x [M][k_iters * 64 >= K] rows, row stride norm_ld
   int32_t norm_K, norm_ld;
@@ -151,56 +140,6 @@ __device__ __forceinline__ void row_pos(const GemmArgs& a, int ki, int& rr, int&
   }
 }
 
-// Work items of one CTA pair: its data-parallel tiles, then its run of
-// stream-K steps (see GemmArgs), cut at tile boundaries.
-enum WorkRole : int { kWorkFull = 0, kWorkHead = 1, kWorkTail = 2 };
-
-struct WorkItem {
-  int tile;
-  int k0, k1;  // K steps [k0, k1) of the tile
-  int role;    // kWorkFull, kWorkHead (adds the next pair's partial), kWorkTail (stores one)
-};
-
-struct WorkIter {
-  int t;             // next data-parallel tile
-  int64_t u, u1;     // stream-K steps [u, u1) still to deal
-};
-
-__device__ __forceinline__ void work_begin(const GemmArgs& a, int pair, int k_total, WorkIter& w) {
-  w.t = pair;
-  w.u = w.u1 = 0;
-  if (a.sk_units > 0) {
-    const int64_t total = static_cast<int64_t>(a.num_tiles - a.sk_first_tile) * k_total;
-    w.u = min(static_cast<int64_t>(pair) * a.sk_units, total);
-    w.u1 = min(w.u + a.sk_units, total);
-  }
-}
-
-__device__ __forceinline__ bool work_next(const GemmArgs& a, int npairs, int k_total,
-                                          WorkIter& w, WorkItem& it) {
-  const int dp_end = a.sk_units > 0 ? a.sk_first_tile : a.num_tiles;
-  if (w.t < dp_end) {
-    it.tile = w.t;
-    it.k0 = 0;
-    it.k1 = k_total;
-    it.role = kWorkFull;
-    w.t += npairs;
-    return true;
-  }
-  if (w.u < w.u1) {
-    const int64_t off = w.u / k_total;
-    const int kb = static_cast<int>(w.u - off * k_total);
-    const int ke = static_cast<int>(min(static_cast<int64_t>(k_total), kb + (w.u1 - w.u)));
-    it.tile = a.sk_first_tile + static_cast<int>(off);
-    it.k0 = kb;
-    it.k1 = ke;
-    it.role = kb > 0 ? kWorkTail : (ke < k_total ? kWorkHead : kWorkFull);
-    w.u += ke - kb;
-    return true;
-  }
-  return false;
-}
-
 // The fused RMSNorm's statistics: rows [r0, r1) of x for this CTA's 256
 // epilogue threads, 4 adjacent lanes per row (each a quarter of the row's
 // 16-byte vectors, summed in a fixed order), 64 rows per pass.
@@ -242,7 +181,7 @@ __device__ __forceinline__ void norm_stats(const GemmArgs& a, int r0, int r1, in
     if (m < r1 && sub == 0) {
       a.norm_rs[m] = rsqrtf(ss / static_cast<float>(a.norm_K) + a.norm_eps);
       __threadfence();
-      ptx::st_release_gpu(a.norm_flag + m, a.sk_epoch);
+      ptx::st_release_gpu(a.norm_flag + m, a.norm_epoch);
     }
   }
 }
@@ -252,7 +191,7 @@ __device__ __forceinline__ bool norm_row_scale(const GemmArgs& a, int m, float& 
                                                volatile int* abort_flag) {
   rs = 1.0f;
   if (m >= a.M) return true;
-  if (!ptx::flag_wait(a.norm_flag + m, a.sk_epoch, abort_flag)) return false;
+  if (!ptx::flag_wait(a.norm_flag + m, a.norm_epoch, abort_flag)) return false;
   rs = __ldcg(a.norm_rs + m);
   return true;
 }
@@ -543,6 +482,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above overlaps the previous kernel's tail; global memory after
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   const int k_total = k_steps(a);
 

@@ -76,6 +76,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   ptx::cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above overlaps the previous kernel's tail; global memory after
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   const int k_total = k_steps(a);
   const uint32_t full_lead = ptx::mapa_shared(&full[0], 0);      // full[s] at + 8 s
@@ -88,26 +91,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      WorkIter wi;
-      WorkItem w;
-      work_begin(a, pair, k_total, wi);
-      while (ok && work_next(a, npairs, k_total, wi, w)) {
+      for (int t = pair; ok && t < a.num_tiles; t += npairs, ++it) {
         int mb, nt;
-        tile_coords(a, w.tile, mb, nt);
+        tile_coords(a, t, mb, nt);
         const bool has1 = 2 * nt + 1 < a.n_halves;
         // This CTA's half of B; an odd last half is padded with the even one.
         const HalfInfo h = decode_half(a, (rank == 1 && has1) ? 2 * nt + 1 : 2 * nt);
         const int m_row = mb * kPairBM + static_cast<int>(rank) * kBM;
         int arow;
         const CUtensorMap* mAcol = a_source(a, m_row, arow);
-        // whole tiles alternate their K direction; stream-K runs go forward
-        const bool rev = a.k_serp && (it & 1) && w.role == kWorkFull;
-        ++it;
+        const bool rev = a.k_serp && (it & 1);
         // row mode: rank and K block of the next step (walking backwards when rev)
         int rr = 0, kb = 0;
-        if (a.mode == kModeRow) row_pos(a, rev ? w.k1 - 1 : w.k0, rr, kb);
-        for (int kstep = 0; kstep < w.k1 - w.k0; ++kstep) {
-          const int ki = rev ? w.k1 - 1 - kstep : w.k0 + kstep;
+        if (a.mode == kModeRow) row_pos(a, rev ? k_total - 1 : 0, rr, kb);
+        for (int kstep = 0; kstep < k_total; ++kstep) {
+          const int ki = rev ? k_total - 1 - kstep : kstep;
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -158,10 +156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool any_mma = false;
       int it = 0;
-      WorkIter wi;
-      WorkItem w;
-      work_begin(a, pair, k_total, wi);
-      for (; ok && work_next(a, npairs, k_total, wi, w); ++it) {
+      for (int t = pair; ok && t < a.num_tiles; t += npairs, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -170,7 +165,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
-        for (int ki = w.k0; ki < w.k1; ++ki) {
+        for (int ki = 0; ki < k_total; ++ki) {
           if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -181,8 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint64_t bdesc = ptx::sdesc_kmajor_sw128(sA + kABytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            ptx::umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                (ki != w.k0) || (kk != 0));
+            ptx::umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ki | kk) != 0);
           ptx::umma_commit_pair(&empty[stage], 0x3);
           any_mma = true;
           if (++stage == kPairStages) {
@@ -210,26 +204,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int hh = ew >> 2;
     const int row = q * 32 + lane;
     int it = 0;
-    WorkIter wi;
-    WorkItem w;
-    work_begin(a, pair, k_total, wi);
-    // this warp's share of a stream-K partial tile, and its flag, in slot s
-    const auto sk_slot = [&](int s) {
-      return a.sk_partial +
-             (static_cast<size_t>(s * 2 + static_cast<int>(rank)) * kEpiWarps + ew) *
-                 (4 * 32 * 32);
-    };
-    const auto sk_flag = [&](int s) {
-      return a.sk_flag + (s * 2 + static_cast<int>(rank)) * kEpiWarps + ew;
-    };
     if (a.norm) {
       const int per = (a.M + gridDim.x - 1) / gridDim.x;
       const int r0 = min(a.M, static_cast<int>(blockIdx.x) * per);
       norm_stats(a, r0, min(a.M, r0 + per), ew * 32 + lane);
     }
-    for (; work_next(a, npairs, k_total, wi, w); ++it) {
+    for (int t = pair; t < a.num_tiles; t += npairs, ++it) {
       int mb, nt;
-      tile_coords(a, w.tile, mb, nt);
+      tile_coords(a, t, mb, nt);
       const bool active = (hh == 0) || (2 * nt + 1 < a.n_halves);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
@@ -248,28 +230,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (a.mode == kModeSwiglu) {
         swiglu_epilogue(a, nt, mb * kPairBM + static_cast<int>(rank) * kBM + row, hh,
                         tmem_base + ((q * 32u) << 16) + acc * kAccCols);
-      } else if (active && w.role == kWorkTail) {
-        // K tail of a split tile: hand this warp's fp32 partial to the pair
-        // that computes the tile's head (it reads slot `pair`).
-        float* dst = sk_slot(pair);
-        for (int c = 0; c < kHalfN / 32; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
-          ptx::tmem_ld_wait();
-          float4* d4 = reinterpret_cast<float4*>(dst + (c * 32 + lane) * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-        }
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) ptx::st_release_gpu(sk_flag(pair), a.sk_epoch);
       } else if (active) {
         const int m = mb * kPairBM + static_cast<int>(rank) * kBM + row;
         int prow;
         __nv_bfloat16* const yb = out_base(a, m, prow);
-        const float* part = nullptr;
         float rs = 1.0f;
         if (a.norm && !__all_sync(0xffffffffu, norm_row_scale(a, m, rs, abort_flag))) {
           if (lane == 0) {
@@ -278,36 +242,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           break;
         }
-        if (w.role == kWorkHead) {
-          // head of a split tile: its tail's partial comes from the next pair
-          int f_ok = 1;
-          if (lane == 0) f_ok = ptx::flag_wait(sk_flag(pair + 1), a.sk_epoch, abort_flag);
-          if (!__shfl_sync(0xffffffffu, f_ok, 0)) {
-            if (lane == 0) {
-              *abort_flag = 1;
-              record_timeout();
-            }
-            break;
-          }
-          part = sk_slot(pair + 1);
-        }
         for (int c = 0; c < kHalfN / 32; ++c) {
           float bv[32];
           if (a.bias != nullptr && c * 32 < h.valid) load_bias_chunk(a, h, c * 32, bv);
           uint32_t r[32];
           ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + acc * kAccCols + hh * kHalfN + c * 32, r);
           ptx::tmem_ld_wait();
-          if (part != nullptr) {
-            const float4* p4 = reinterpret_cast<const float4*>(part + (c * 32 + lane) * 32);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 v = __ldcg(p4 + j);
-              r[4 * j] = __float_as_uint(__uint_as_float(r[4 * j]) + v.x);
-              r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) + v.y);
-              r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) + v.z);
-              r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) + v.w);
-            }
-          }
           if (m < a.M && c * 32 < h.valid) store_chunk(a, h, m, prow, yb, c * 32, r, bv, rs);
         }
       }

@@ -18,6 +18,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace tpl {
 
@@ -128,6 +129,8 @@ __global__ void __launch_bounds__(kF32Threads) gemm_fp32_simt(const __grid_const
   const int nt = blockIdx.x;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kF32BM;
   const int split = gridDim.z, z = blockIdx.z;
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   // Output column mapping of this tile.
   int32_t wrow0, valid, ld, bias0;

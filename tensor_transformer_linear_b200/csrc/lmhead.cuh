@@ -116,6 +116,9 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above overlaps the previous kernel's tail; global memory after
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {

@@ -75,6 +75,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// --------------------------------------------- programmatic dependent launch
+
+// Waits until the kernels this one depends on (earlier work on the stream)
+// have completed and their memory is visible; returns at once when the kernel
+// was not launched as a programmatic dependent.  Every global-memory access
+// of a kernel comes after it.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel on the stream (launched as a programmatic dependent)
+// be scheduled: its CTAs start their prologues on SMs that free up and wait
+// in griddep_wait until this kernel has completed.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------- flags between CTAs
 
 // Release store / acquire load of a 32-bit flag in global memory, GPU scope.

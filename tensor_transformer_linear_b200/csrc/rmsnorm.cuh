@@ -10,6 +10,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace tpl {
 
@@ -59,6 +60,8 @@ template <typename T, int VPL>
 __global__ void __launch_bounds__(kNormWarps * 32)
     rmsnorm_reg(const T* x, T* y, const float* __restrict__ scale, int centered, float eps,
                 int64_t M, int H) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   using VT = VecTraits<T>;
   constexpr int P = VT::kPer;
   const int lane = threadIdx.x & 31;
@@ -122,6 +125,8 @@ template <typename T, int VPT>
 __global__ void __launch_bounds__(kNormCtaThreads)
     rmsnorm_cta(const T* x, T* y, const float* __restrict__ scale, int centered, float eps,
                 int64_t M, int H) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   using VT = VecTraits<T>;
   constexpr int P = VT::kPer;
   __shared__ float part[kNormCtaThreads / 32];
@@ -186,6 +191,8 @@ template <typename T>
 __global__ void __launch_bounds__(kNormWarps * 32)
     rmsnorm_generic(const T* x, T* y, const float* __restrict__ scale, int centered, float eps,
                     int64_t M, int64_t H) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   using VT = VecTraits<T>;
   const int lane = threadIdx.x & 31;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * kNormWarps + (threadIdx.x >> 5); row < M;

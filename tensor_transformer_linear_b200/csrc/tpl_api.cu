@@ -36,7 +36,7 @@ struct DeviceInfo {
   int sm_count = 0;
   bool gemm_attr = false;
   bool lm_attr = false;
-  uint32_t sk_epoch = 0;  // last stream-K launch epoch on this device
+  uint32_t epoch = 0;  // last flag epoch handed to a launch on this device
 };
 
 std::mutex g_mu;
@@ -121,64 +121,41 @@ int env_int(const char* name, int dflt) {
   return (e != nullptr && e[0] != '\0') ? std::atoi(e) : dflt;
 }
 
-// A caller's stream-K workspace (see tpl_gemm_workspace_size).
-struct SkWorkspace {
-  void* ptr = nullptr;
-  size_t bytes = 0;
-};
-
-constexpr size_t kSkSlotFloats = static_cast<size_t>(2) * tpl::kEpiWarps * 4 * 32 * 32;  // per pair
-constexpr size_t kSkSlotFlags = static_cast<size_t>(2) * tpl::kEpiWarps;
-
-size_t sk_partial_bytes(int sm_count) {
-  return static_cast<size_t>(sm_count / 2) * kSkSlotFloats * sizeof(float);
-}
-
-size_t sk_workspace_bytes(int sm_count) {
-  const size_t raw = sk_partial_bytes(sm_count) +
-                     static_cast<size_t>(sm_count / 2) * kSkSlotFlags * sizeof(uint32_t);
-  return (raw + 255) / 256 * 256;
-}
-
-// K steps of one tile (host copy of tpl::k_steps).
-int host_k_steps(const tpl::GemmArgs& a) {
-  if (a.mode != tpl::kModeRow) return a.k_iters;
-  const int n1 = std::max(0, std::min(a.r1, a.r_split) - a.r0);
-  const int n2 = std::max(0, a.r1 - std::max(a.r0, a.r_split));
-  return n1 * a.k_iters + n2 * a.k_iters2;
-}
-
-// Stream-K plan of a CTA-pair launch: the last full wave and the partial one
-// are dealt out by K steps (at least one tile's worth per pair).  Only when a
-// workspace is given, the last wave is partial, there is a full wave before it,
-// and the epilogue is the plain one (no SwiGLU pairing, no per-rank partials).
-void plan_stream_k(tpl::GemmArgs& a, int64_t tiles, int64_t pairs, DeviceInfo* dev,
-                   const SkWorkspace* ws) {
-  a.sk_first_tile = static_cast<int32_t>(tiles);
-  a.sk_units = 0;
-  if (ws == nullptr || ws->ptr == nullptr || ws->bytes < sk_workspace_bytes(dev->sm_count))
-    return;
-  if (a.mode == tpl::kModeSwiglu || a.partials != nullptr) return;
-  if (env_int("TPL_GEMM_STREAMK", 1) == 0) return;
-  const int64_t waves = tiles / pairs, rem = tiles % pairs;
-  if (waves < 1 || rem == 0) return;
-  const int64_t k_total = host_k_steps(a);
-  const int64_t first = (waves - 1) * pairs;
-  const int64_t units = (tiles - first) * k_total;
-  const int64_t per_pair = (units + pairs - 1) / pairs;
-  if (per_pair < k_total || per_pair > INT32_MAX) return;
-  a.sk_first_tile = static_cast<int32_t>(first);
-  a.sk_units = static_cast<int32_t>(per_pair);
-  a.sk_partial = static_cast<float*>(ws->ptr);
-  a.sk_flag = reinterpret_cast<uint32_t*>(static_cast<char*>(ws->ptr) +
-                                          sk_partial_bytes(dev->sm_count));
-}
-
 // A fresh epoch for the flags of one launch (never 0, so zeroed flags never match).
 uint32_t next_epoch(DeviceInfo* dev) {
   std::lock_guard<std::mutex> lk(g_mu);
-  if (++dev->sk_epoch == 0) dev->sk_epoch = 1;
-  return dev->sk_epoch;
+  if (++dev->epoch == 0) dev->epoch = 1;
+  return dev->epoch;
+}
+
+// Kernels of the path are launched as programmatic dependents of the work
+// before them on the stream (CUDA programmatic dependent launch): a kernel's
+// CTAs start their prologue (barrier init, TMEM allocation, descriptor
+// prefetch) on SMs the previous kernel has left, and wait in griddep_wait
+// until it has completed.  TPL_PDL=0 launches them plainly.
+bool pdl_enabled() {
+  static const bool on = env_int("TPL_PDL", 1) != 0;
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+tpl_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  if (pdl_enabled()) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) return TPL_ERR_CUDA;
+  return launched();
 }
 
 // CTA pairs (tcgen05 cta_group::2, 256-row tiles) unless M fits one 128-row
@@ -191,8 +168,7 @@ bool use_cta_pairs(int64_t M) {
 
 // Fills the tile counts of `a` (n_tiles / n_halves already set) and launches
 // the GEMM on a single CTA per tile or on CTA pairs.
-tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, DeviceInfo* dev, cudaStream_t st,
-                       const SkWorkspace* ws = nullptr) {
+tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, DeviceInfo* dev, cudaStream_t st) {
   const bool pairs = use_cta_pairs(M) && dev->sm_count >= 2;
   const int64_t bm = pairs ? tpl::kPairBM : tpl::kBM;
   a.m_blocks = static_cast<int32_t>((M + bm - 1) / bm);
@@ -209,23 +185,16 @@ tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, DeviceInfo* dev, cudaStream_
   const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
   if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
   a.num_tiles = static_cast<int32_t>(tiles);
-  a.sk_first_tile = static_cast<int32_t>(tiles);
-  a.sk_units = 0;
-  a.sk_epoch = 0;
-  if (pairs) {
-    const int64_t npairs = std::min<int64_t>(tiles, dev->sm_count / 2);
-    plan_stream_k(a, tiles, npairs, dev, ws);
-  }
-  if (a.sk_units > 0 || a.norm) a.sk_epoch = next_epoch(dev);
+  if (a.norm) a.norm_epoch = next_epoch(dev);
   if (pairs) {
     const int64_t npairs = std::min<int64_t>(tiles, dev->sm_count / 2);
     const int grid = 2 * static_cast<int>(npairs);
-    tpl::gemm_bf16_tcgen05_pair<<<grid, tpl::kGemmThreads, tpl::kGemmPairSmemBytes, st>>>(a);
-  } else {
-    const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
-    tpl::gemm_bf16_tcgen05<<<grid, tpl::kGemmThreads, tpl::kGemmSmemBytes, st>>>(a);
+    return launch_ex(tpl::gemm_bf16_tcgen05_pair, dim3(grid), dim3(tpl::kGemmThreads),
+                     tpl::kGemmPairSmemBytes, st, a);
   }
-  return launched();
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->sm_count));
+  return launch_ex(tpl::gemm_bf16_tcgen05, dim3(grid), dim3(tpl::kGemmThreads),
+                   tpl::kGemmSmemBytes, st, a);
 }
 
 tpl_status check_partition(const tpl_partition* p) {
@@ -291,7 +260,7 @@ struct GatherA {
 tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t K, const void* w,
                        const void* bias, int act, void* y, cudaStream_t st,
                        const SeqPar& sp = SeqPar{}, const GatherA* ga = nullptr,
-                       const SkWorkspace* ws = nullptr, const NormFuse* nf = nullptr) {
+                       const NormFuse* nf = nullptr) {
   if ((K % 8) != 0 || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 2) ||
       (bias != nullptr && !aligned(bias, 2)))
     return TPL_ERR_ALIGN;
@@ -366,7 +335,7 @@ tpl_status column_bf16(const tpl_partition* p, const void* x, int64_t M, int64_t
     a.n_halves = hb;
     a.vec_store = vec ? 1 : 0;
     a.n_tiles = (hb + 1) / 2;
-    if ((s = launch_gemm(a, M, dev, st, ws)) != TPL_OK) return s;
+    if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
   }
   return TPL_OK;
 }
@@ -385,13 +354,18 @@ tpl_status launch_fp32(const tpl::F32Args& a, int64_t mb, cudaStream_t st) {
   cfg.blockDim = dim3(tpl::kF32Threads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = static_cast<unsigned>(split);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (pdl_enabled()) {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
+  }
   if (cudaLaunchKernelEx(&cfg, tpl::gemm_fp32_simt, a) != cudaSuccess) return TPL_ERR_CUDA;
   return launched();
 }
@@ -457,7 +431,7 @@ tpl_status column_fp32(const tpl_partition* p, const void* x, int64_t M, int64_t
 tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_t N, const void* w,
                     const void* bias, const void* residual, void* y, float* partials,
                     cudaStream_t st, const SeqPar& sp = SeqPar{},
-                    const PeerScatter* ps = nullptr, const SkWorkspace* ws = nullptr) {
+                    const PeerScatter* ps = nullptr) {
   for (int r = 0; r < tp; ++r)
     if (k_w[r] % 8 != 0) return TPL_ERR_ALIGN;
   if (!aligned(h, 16) || !aligned(w, 16) || !aligned(y, 2) || (bias && !aligned(bias, 2)) ||
@@ -526,7 +500,7 @@ tpl_status row_bf16(const void* h, const int64_t* k_w, int tp, int64_t M, int64_
     }
     a.vec_store = vec ? 1 : 0;
   }
-  if ((s = launch_gemm(a, M, dev, st, ws)) != TPL_OK) return s;
+  if ((s = launch_gemm(a, M, dev, st)) != TPL_OK) return s;
 
   if (partials != nullptr) {
     a.bias = nullptr;
@@ -615,30 +589,41 @@ tpl_status rmsnorm_launch(const void* x, int64_t M, int64_t H, const float* scal
     const int gc = static_cast<int>(std::min<int64_t>(M, INT32_MAX));
     const int tc = tpl::kNormCtaThreads;
     if (cta_vec <= 2)
-      tpl::rmsnorm_cta<T, 2><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_cta<T, 2>, dim3(gc), dim3(tc), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else if (cta_vec <= 4)
-      tpl::rmsnorm_cta<T, 4><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_cta<T, 4>, dim3(gc), dim3(tc), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else if (cta_vec <= 8)
-      tpl::rmsnorm_cta<T, 8><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_cta<T, 8>, dim3(gc), dim3(tc), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else
-      tpl::rmsnorm_cta<T, 16><<<gc, tc, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_cta<T, 16>, dim3(gc), dim3(tc), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
   } else if (vec && lanes_vec <= 32) {
     if (lanes_vec <= 1)
-      tpl::rmsnorm_reg<T, 1><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_reg<T, 1>, dim3(g), dim3(t), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else if (lanes_vec <= 2)
-      tpl::rmsnorm_reg<T, 2><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_reg<T, 2>, dim3(g), dim3(t), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else if (lanes_vec <= 4)
-      tpl::rmsnorm_reg<T, 4><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_reg<T, 4>, dim3(g), dim3(t), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else if (lanes_vec <= 8)
-      tpl::rmsnorm_reg<T, 8><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_reg<T, 8>, dim3(g), dim3(t), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else if (lanes_vec <= 16)
-      tpl::rmsnorm_reg<T, 16><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_reg<T, 16>, dim3(g), dim3(t), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
     else
-      tpl::rmsnorm_reg<T, 32><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, Hi);
+      s = launch_ex(tpl::rmsnorm_reg<T, 32>, dim3(g), dim3(t), 0, st, xp, yp, scale,
+                    centered, eps, M, Hi);
   } else {
-    tpl::rmsnorm_generic<T><<<g, t, 0, st>>>(xp, yp, scale, centered, eps, M, H);
+    s = launch_ex(tpl::rmsnorm_generic<T>, dim3(g), dim3(t), 0, st, xp, yp, scale, centered, eps,
+                  M, H);
   }
-  return launched();
+  return s;
 }
 
 }  // namespace
@@ -711,18 +696,9 @@ tpl_status tpl_partition_subparams(const int64_t* sub_sizes, int32_t n_sub, int3
   return TPL_OK;
 }
 
-tpl_status tpl_gemm_workspace_size(size_t* bytes) {
-  if (bytes == nullptr) return TPL_ERR_NULL;
-  DeviceInfo* dev = nullptr;
-  tpl_status s = device_info(&dev);
-  if (s != TPL_OK) return s;
-  *bytes = sk_workspace_bytes(dev->sm_count);
-  return TPL_OK;
-}
-
-static tpl_status column_entry(const tpl_partition* p, const void* x, int64_t M, int64_t K,
-                               const void* w, const void* bias, tpl_dtype dt, tpl_act act,
-                               void* y, void* stream, const SkWorkspace* ws) {
+tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, int64_t K,
+                             const void* w, const void* bias, tpl_dtype dt, tpl_act act, void* y,
+                             void* stream) {
   if (p == nullptr) return TPL_ERR_NULL;
   if ((dt != TPL_FP32 && dt != TPL_BF16) || !act_ok(act)) return TPL_ERR_DTYPE;
   tpl_status s = check_partition(p);
@@ -731,29 +707,13 @@ static tpl_status column_entry(const tpl_partition* p, const void* x, int64_t M,
   if (M == 0) return TPL_OK;
   if (x == nullptr || w == nullptr || y == nullptr) return TPL_ERR_NULL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dt == TPL_BF16 ? column_bf16(p, x, M, K, w, bias, act, y, st, SeqPar{}, nullptr, ws)
+  return dt == TPL_BF16 ? column_bf16(p, x, M, K, w, bias, act, y, st)
                         : column_fp32(p, x, M, K, w, bias, act, y, st);
 }
 
-tpl_status tpl_column_linear(const tpl_partition* p, const void* x, int64_t M, int64_t K,
-                             const void* w, const void* bias, tpl_dtype dt, tpl_act act, void* y,
-                             void* stream) {
-  return column_entry(p, x, M, K, w, bias, dt, act, y, stream, nullptr);
-}
-
-tpl_status tpl_column_linear_ws(const tpl_partition* p, const void* x, int64_t M, int64_t K,
-                                const void* w, const void* bias, tpl_dtype dt, tpl_act act,
-                                void* y, void* workspace, size_t ws_bytes, void* stream) {
-  if (workspace == nullptr) return TPL_ERR_NULL;
-  SkWorkspace ws;
-  ws.ptr = workspace;
-  ws.bytes = ws_bytes;
-  return column_entry(p, x, M, K, w, bias, dt, act, y, stream, &ws);
-}
-
-static tpl_status row_entry(const void* h, const int64_t* k_w, int32_t tp, int64_t M, int64_t N,
-                            const void* w, const void* bias, const void* residual, tpl_dtype dt,
-                            void* y, float* partials, void* stream, const SkWorkspace* ws) {
+tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
+                                 int64_t N, const void* w, const void* bias, const void* residual,
+                                 tpl_dtype dt, void* y, float* partials, void* stream) {
   if (k_w == nullptr) return TPL_ERR_NULL;
   if (dt != TPL_FP32 && dt != TPL_BF16) return TPL_ERR_DTYPE;
   if (tp < 1 || tp > TPL_MAX_TP || M < 0 || N < 1 || M > INT32_MAX || N > INT32_MAX)
@@ -767,9 +727,8 @@ static tpl_status row_entry(const void* h, const int64_t* k_w, int32_t tp, int64
   if (M == 0) return TPL_OK;
   if (h == nullptr || w == nullptr || y == nullptr) return TPL_ERR_NULL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dt == TPL_BF16
-             ? row_bf16(h, k_w, tp, M, N, w, bias, residual, y, partials, st, SeqPar{}, nullptr, ws)
-             : row_fp32(h, k_w, tp, M, N, w, bias, residual, y, partials, st);
+  return dt == TPL_BF16 ? row_bf16(h, k_w, tp, M, N, w, bias, residual, y, partials, st)
+                        : row_fp32(h, k_w, tp, M, N, w, bias, residual, y, partials, st);
 }
 
 static size_t round256(size_t n) { return (n + 255) / 256 * 256; }
@@ -777,10 +736,7 @@ static size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 tpl_status tpl_column_linear_rmsnorm_workspace_size(int64_t M, size_t* bytes) {
   if (bytes == nullptr) return TPL_ERR_NULL;
   if (M < 0 || M > INT32_MAX) return TPL_ERR_SHAPE;
-  size_t sk = 0;
-  tpl_status s = tpl_gemm_workspace_size(&sk);
-  if (s != TPL_OK) return s;
-  *bytes = sk + 2 * round256(static_cast<size_t>(M) * 4);
+  *bytes = 2 * round256(static_cast<size_t>(M) * 4);
   return TPL_OK;
 }
 
@@ -798,18 +754,13 @@ tpl_status tpl_column_linear_rmsnorm(const tpl_partition* p, const void* x, int6
   size_t need = 0;
   if ((s = tpl_column_linear_rmsnorm_workspace_size(M, &need)) != TPL_OK) return s;
   if (ws_bytes < need) return TPL_ERR_SHAPE;
-  size_t sk = 0;
-  tpl_gemm_workspace_size(&sk);
-  SkWorkspace ws;
-  ws.ptr = workspace;
-  ws.bytes = sk;
   NormFuse nf;
   nf.eps = eps;
-  nf.rs = reinterpret_cast<float*>(static_cast<char*>(workspace) + sk);
-  nf.flag = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + sk +
+  nf.rs = static_cast<float*>(workspace);
+  nf.flag = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) +
                                         round256(static_cast<size_t>(M) * 4));
   return column_bf16(p, x, M, K, w, bias, act, y, static_cast<cudaStream_t>(stream), SeqPar{},
-                     nullptr, &ws, &nf);
+                     nullptr, &nf);
 }
 
 tpl_status tpl_fold_norm_scale(const void* w, int64_t rows, int64_t K, const float* scale,
@@ -829,23 +780,6 @@ tpl_status tpl_fold_norm_scale(const void* w, int64_t rows, int64_t K, const flo
       static_cast<const __nv_bfloat16*>(w), rows, K, scale, centered,
       static_cast<__nv_bfloat16*>(w_out));
   return launched();
-}
-
-tpl_status tpl_row_linear_reduce(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
-                                 int64_t N, const void* w, const void* bias, const void* residual,
-                                 tpl_dtype dt, void* y, float* partials, void* stream) {
-  return row_entry(h, k_w, tp, M, N, w, bias, residual, dt, y, partials, stream, nullptr);
-}
-
-tpl_status tpl_row_linear_reduce_ws(const void* h, const int64_t* k_w, int32_t tp, int64_t M,
-                                    int64_t N, const void* w, const void* bias,
-                                    const void* residual, tpl_dtype dt, void* y, float* partials,
-                                    void* workspace, size_t ws_bytes, void* stream) {
-  if (workspace == nullptr) return TPL_ERR_NULL;
-  SkWorkspace ws;
-  ws.ptr = workspace;
-  ws.bytes = ws_bytes;
-  return row_entry(h, k_w, tp, M, N, w, bias, residual, dt, y, partials, stream, &ws);
 }
 
 tpl_status tpl_rmsnorm(const void* x, int64_t M, int64_t H, const float* scale, int32_t centered,
@@ -963,8 +897,8 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
 }
 
 tpl_status lmhead_launch(const tpl::LmArgs& a, int smem, int grid, cudaStream_t st) {
-  tpl::lmhead_argmax_tcgen05<<<grid, tpl::kLmThreads, smem, st>>>(a);
-  return launched();
+  return launch_ex(tpl::lmhead_argmax_tcgen05, dim3(grid), dim3(tpl::kLmThreads),
+                   static_cast<size_t>(smem), st, a);
 }
 
 }  // namespace

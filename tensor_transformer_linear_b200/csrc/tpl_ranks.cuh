@@ -170,7 +170,7 @@ namespace {
 
 tpl_status column_gather(const tpl_partition* p, void* const* peer_x, int32_t tp, int64_t batch,
                          int64_t seq, int64_t K, const void* w, const void* bias, tpl_act act,
-                         void* y, void* stream, const SkWorkspace* ws) {
+                         void* y, void* stream) {
   if (p == nullptr || peer_x == nullptr) return TPL_ERR_NULL;
   if (!act_ok(act)) return TPL_ERR_DTYPE;
   tpl_status s = check_partition(p);
@@ -188,12 +188,12 @@ tpl_status column_gather(const tpl_partition* p, void* const* peer_x, int32_t tp
   ga.tp = tp;
   ga.gather = peer_x;
   return column_bf16(p, peer_x[0], batch * seq, K, w, bias, act, y,
-                     static_cast<cudaStream_t>(stream), sp, &ga, ws);
+                     static_cast<cudaStream_t>(stream), sp, &ga);
 }
 
 tpl_status row_scatter(const void* h, int64_t K, int64_t batch, int64_t seq, int64_t N,
-                       const void* w, int32_t rank, int32_t tp, void* const* peer, void* stream,
-                       const SkWorkspace* ws) {
+                       const void* w, int32_t rank, int32_t tp, void* const* peer,
+                       void* stream) {
   if (peer == nullptr) return TPL_ERR_NULL;
   SeqPar sp;
   tpl_status s = seqpar_of(batch, seq, tp, &sp);
@@ -211,7 +211,7 @@ tpl_status row_scatter(const void* h, int64_t K, int64_t batch, int64_t seq, int
   ps.peer = peer;
   const int64_t kw[1] = {K};
   return row_bf16(h, kw, 1, batch * seq, N, w, nullptr, nullptr, nullptr, nullptr,
-                  static_cast<cudaStream_t>(stream), sp, &ps, ws);
+                  static_cast<cudaStream_t>(stream), sp, &ps);
 }
 
 }  // namespace
@@ -221,36 +221,15 @@ extern "C" {
 tpl_status tpl_column_linear_gather(const tpl_partition* p, void* const* peer_x, int32_t tp,
                                     int64_t batch, int64_t seq, int64_t K, const void* w,
                                     const void* bias, tpl_act act, void* y, void* stream) {
-  return column_gather(p, peer_x, tp, batch, seq, K, w, bias, act, y, stream, nullptr);
-}
-
-tpl_status tpl_column_linear_gather_ws(const tpl_partition* p, void* const* peer_x, int32_t tp,
-                                       int64_t batch, int64_t seq, int64_t K, const void* w,
-                                       const void* bias, tpl_act act, void* y, void* workspace,
-                                       size_t ws_bytes, void* stream) {
-  if (workspace == nullptr) return TPL_ERR_NULL;
-  SkWorkspace ws;
-  ws.ptr = workspace;
-  ws.bytes = ws_bytes;
-  return column_gather(p, peer_x, tp, batch, seq, K, w, bias, act, y, stream, &ws);
+  return column_gather(p, peer_x, tp, batch, seq, K, w, bias, act, y, stream);
 }
 
 tpl_status tpl_row_linear_scatter(const void* h, int64_t K, int64_t batch, int64_t seq, int64_t N,
                                   const void* w, int32_t rank, int32_t tp, void* const* peer,
                                   void* stream) {
-  return row_scatter(h, K, batch, seq, N, w, rank, tp, peer, stream, nullptr);
+  return row_scatter(h, K, batch, seq, N, w, rank, tp, peer, stream);
 }
 
-tpl_status tpl_row_linear_scatter_ws(const void* h, int64_t K, int64_t batch, int64_t seq,
-                                     int64_t N, const void* w, int32_t rank, int32_t tp,
-                                     void* const* peer, void* workspace, size_t ws_bytes,
-                                     void* stream) {
-  if (workspace == nullptr) return TPL_ERR_NULL;
-  SkWorkspace ws;
-  ws.ptr = workspace;
-  ws.bytes = ws_bytes;
-  return row_scatter(h, K, batch, seq, N, w, rank, tp, peer, stream, &ws);
-}
 
 tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t N,
                             const void* bias, const void* residual, void* y, void* stream) {

@@ -8,7 +8,6 @@ residual section.  Each step is one call into libtpl.so.
 """
 from __future__ import annotations
 
-import functools
 from typing import Callable, List, Optional, Sequence
 
 import torch
@@ -55,7 +54,7 @@ class TPMLP:
     def __init__(self, w1: torch.Tensor, w2_full: torch.Tensor, tp: int, act: str,
                  scale: Optional[torch.Tensor] = None, centered: bool = False,
                  norm: bool = True, residual: bool = False, eps: float = 1e-6,
-                 workspace: Optional[torch.Tensor] = None, fused_norm: bool = False):
+                 fused_norm: bool = False):
         self.inter, self.hidden = w1.shape
         self.part = tpl_partition_subparams([self.inter], tp, 1)
         self.k_w = [self.part.shard_width[r] for r in range(tp)]
@@ -63,7 +62,6 @@ class TPMLP:
         self.w2 = pack_row_weight(w2_full, self.k_w)
         self.act, self.scale, self.centered = act, scale, centered
         self.norm, self.residual, self.eps = norm, residual, eps
-        self.workspace = workspace   # stream-K workspace of the two GEMMs (or None)
         self.fused_norm = bool(fused_norm and norm)
         if self.fused_norm and scale is not None:
             self.w1 = tpl_fold_norm_scale(self.w1, scale, centered)
@@ -95,7 +93,7 @@ class TPMLP:
                 out = torch.empty((M, self.hidden), dtype=x.dtype, device=x.device)
             tpl_row_linear_reduce(h, self.k_w, M, self.w2, None,
                                   x.view(M, self.hidden) if self.residual else None, y=out,
-                                  stream=stream, workspace=ws)
+                                  stream=stream)
             return out
         xn = x
         if self.norm:
@@ -104,12 +102,12 @@ class TPMLP:
                         stream=stream)
         h = self._buf("h", M * self.inter, x)
         tpl_column_linear(self.part, xn.view(M, self.hidden), self.w1, None, self.act, y=h,
-                          stream=stream, workspace=self.workspace)
+                          stream=stream)
         if out is None:
             out = torch.empty((M, self.hidden), dtype=x.dtype, device=x.device)
         tpl_row_linear_reduce(h, self.k_w, M, self.w2, None,
                               x.view(M, self.hidden) if self.residual else None, y=out,
-                              stream=stream, workspace=self.workspace)
+                              stream=stream)
         return out
 
 
@@ -319,8 +317,7 @@ class TPRankMLP:
     def __init__(self, w1_shard: torch.Tensor, w2_shard: torch.Tensor, rank: int, tp: int,
                  act: str, xn: PeerBuffers, recv: PeerBuffers, barrier: Callable,
                  scale: Optional[torch.Tensor] = None, centered: bool = False,
-                 eps: float = 1e-6, ops: Optional[dict] = None,
-                 workspace: Optional[torch.Tensor] = None):
+                 eps: float = 1e-6, ops: Optional[dict] = None):
         self.w1, self.w2 = w1_shard.contiguous(), w2_shard.contiguous()
         self.rank, self.tp, self.act = rank, tp, act
         self.xn, self.recv, self.barrier = xn, recv, barrier
@@ -330,11 +327,6 @@ class TPRankMLP:
         self.rmsnorm = ops.get("rmsnorm", tpl_rmsnorm)
         self.column = ops.get("column", tpl_column_linear_gather)
         self.scatter = ops.get("scatter", tpl_row_linear_scatter)
-        if workspace is not None:   # stream-K workspace of the two GEMMs
-            if "column" not in ops:
-                self.column = functools.partial(tpl_column_linear_gather, workspace=workspace)
-            if "scatter" not in ops:
-                self.scatter = functools.partial(tpl_row_linear_scatter, workspace=workspace)
         self.reduce = ops.get("reduce", tpl_reduce_slots)
         self._h = None
 

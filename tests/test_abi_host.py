@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 28, names
+    assert len(names) == 23, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
