@@ -304,11 +304,12 @@ class Block:
             self.io_out += ["ids", "smax", "sidx"]
         self.parts = [n for n, _ in self.launches]
 
-    def step(self, stream, events=None):
-        for i, (_, fn) in enumerate(self.launches):
+    def step(self, stream, events=None, skip=()):
+        for i, (name, fn) in enumerate(self.launches):
             if events is not None:
                 events[i].record(stream)
-            fn(stream)
+            if name not in skip:
+                fn(stream)
         if events is not None:
             events[len(self.launches)].record(stream)
 
@@ -510,11 +511,12 @@ class NextRows:
             raise ValueError(kind)
         self.parts = [n for n, _ in self.launches]
 
-    def step(self, stream, events=None):
-        for i, (_, fn) in enumerate(self.launches):
+    def step(self, stream, events=None, skip=()):
+        for i, (name, fn) in enumerate(self.launches):
             if events is not None:
                 events[i].record(stream)
-            fn(stream)
+            if name not in skip:
+                fn(stream)
         if events is not None:
             events[len(self.launches)].record(stream)
 
@@ -836,19 +838,34 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def step_region_ms(wl, stream, steps, skip=()):
+    """Device time of ``steps`` steps with events only around the region (no
+    event between launches, so programmatic dependent launches overlap as in a
+    real run)."""
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        wl.step(stream, skip=skip) if skip else wl.step(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(stop)
+
+
 def timed_steps(wl, stream, steps, pg, dev):
-    """Times ``steps`` steps of ``wl`` on ``stream`` with CUDA events (whole region
-    and per launch), sampling the SM clock meanwhile.  A run under a hardware or
-    thermal slowdown (or a stale clock lock) is taken again once; every rank
-    makes the same decision.  Returns (region ms, mean ms per part, library
-    launches in the region, clock record)."""
+    """Times ``steps`` steps of ``wl`` on ``stream`` with CUDA events, sampling the
+    SM clock meanwhile.  The step time comes from a region with events only at
+    its ends; the time of each launch from a second pass with an event between
+    every two launches.  (An event between two kernels stops the next one from
+    starting its prologue during the previous one's tail, so the parts of the
+    second pass can add up to slightly more than a step.)  A run under a
+    hardware or thermal slowdown (or a stale clock lock) is taken again once;
+    every rank makes the same decision.  Returns (region ms, mean ms per part,
+    library launches in the region, clock record)."""
     import tensor_transformer_linear_b200 as T
     n_ev = len(wl.parts) + 1
 
     def region():
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-               for _ in range(steps)]
-        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         clocks = ClockSampler(torch.cuda.current_device())
         if pg is not None:
             pg.barrier()
@@ -857,11 +874,7 @@ def timed_steps(wl, stream, steps, pg, dev):
         time.sleep(0.3)   # nvidia-smi is sampling before the timed steps start
         n0 = T.tpl_launch_count()
         t0 = datetime.datetime.now()
-        start.record(stream)
-        for k in range(steps):
-            wl.step(stream, evs[k])
-        stop.record(stream)
-        torch.cuda.synchronize()
+        ms = step_region_ms(wl, stream, steps)
         t1 = datetime.datetime.now()
         launches = T.tpl_launch_count() - n0
         clk = clocks.stop(t0, t1)
@@ -869,9 +882,17 @@ def timed_steps(wl, stream, steps, pg, dev):
             pg.barrier()
         if T.tpl_get_device_status(stream) != 0:
             raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
+        # per-launch times: a second pass with an event between every two launches
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+               for _ in range(steps)]
+        for k in range(steps):
+            wl.step(stream, evs[k])
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
         part_ms = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1])
                                    for k in range(steps)) for i in range(n_ev - 1)]
-        return start.elapsed_time(stop), part_ms, launches, clk
+        return ms, part_ms, launches, clk
 
     ms, part_ms, launches, clk = region()
     bad = torch.tensor([1.0 if clocks_rejected(clk) else 0.0], device=dev)
@@ -884,6 +905,16 @@ def timed_steps(wl, stream, steps, pg, dev):
         clk["remeasured"] = remeasured
     return ms, part_ms, launches, clk
 
+
+def marginal_part_ms(wl, stream, steps, part, rounds=5):
+    """A part's cost inside the step as it really runs (no events around it):
+    the median, over ``rounds`` interleaved pairs, of (step time) - (step time
+    without that launch), per step."""
+    with_p, without = [], []
+    for _ in range(rounds):
+        with_p.append(step_region_ms(wl, stream, steps) / steps)
+        without.append(step_region_ms(wl, stream, steps, skip=(part,)) / steps)
+    return statistics.median(w - o for w, o in zip(with_p, without))
 
 def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
     """The 4-layer residual stack x[4,4096,8192] at full size, timed in the same
@@ -1025,6 +1056,13 @@ def main():
     # ---- device-timed region: K steps, per-launch events on the launching stream
     ms, part_ms, launches, clk = timed_steps(wl, stream, args.steps, pg, dev)
 
+    # ---- the LM head's cost inside the step as it runs (no events around it)
+    lm_marginal_ms = None
+    if "lmhead_argmax" in getattr(wl, "parts", []) and len(wl.parts) > 1:
+        lm_marginal_ms = marginal_part_ms(wl, stream, args.steps, "lmhead_argmax")
+        if pg is not None:
+            lm_marginal_ms = max_over_ranks([lm_marginal_ms], dev)[0]
+
     # ---- the LM head in a decode loop: back-to-back launches, as once per decode step
     decode_ms = None
     lm = dict(getattr(wl, "launches", [])).get("lmhead_argmax")
@@ -1150,10 +1188,20 @@ def main():
                 "kernel": "lmhead_argmax_tcgen05", "bound": "hbm", "achieved": round(gbs, 1),
                 "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
                 "frac_of_8000": round(gbs / 8000.0, 4), "bytes_per_launch": lb,
-                "measured": "inside the timed block steps, right after the GEMMs "
-                            "(power-capped clocks)",
+                "ms": round(lm_ms, 4),
+                "measured": "inside the block steps, right after the GEMMs, from CUDA events "
+                            "around the launch",
                 "traffic": ncu_traffic("lmhead_argmax_tcgen05", "lmhead",
                                        ["lmhead.cuh", "ptx.cuh", "common.cuh"])}
+            if lm_marginal_ms is not None and lm_marginal_ms > 0:
+                gm = lb / (lm_marginal_ms * 1e-3) / 1e9
+                line["roofline_lmhead"]["in_step_marginal"] = {
+                    "achieved": round(gm, 1), "frac": round(gm / pk["hbm_gbs"], 4),
+                    "frac_of_8000": round(gm / 8000.0, 4), "ms": round(lm_marginal_ms, 4),
+                    "measured": "step time minus the step time without the LM head launch, "
+                                "each from events around 20-step regions with no event "
+                                "between launches (the launch overlaps the GEMM's tail as it "
+                                "does in a real step), median of 5 interleaved pairs"}
             if decode_ms is not None:
                 dg = lb / (decode_ms * 1e-3) / 1e9
                 line["roofline_lmhead_decode"] = {
