@@ -6,20 +6,23 @@ One step is one pass of the whole hot path over one batch of synthetic input
 
   1. GQA fused-QKV column-parallel linear  x[4,1024,4096] bf16, 32 q + 8 kv
      heads of 128, tp 8, bias                      (sub-parameter partition)
-  2. RMSNorm (eps 1e-6, centred scale) -> c_fc 4096->14336 column-parallel
-     + GELU(erf) -> c_proj 14336->4096 row-parallel with the partial-sum
-     reduction in the epilogue                     x[8,1024,4096] bf16, tp 8
+  2. RMSNorm (eps 1e-6, centred scale) fused into c_fc 4096->14336
+     column-parallel + GELU(erf) -> c_proj 14336->4096 row-parallel with the
+     partial-sum reduction in the epilogue         x[8,1024,4096] bf16, tp 8
   3. decode LM head x[32,4096] over W[128256,4096] bf16, 8 vocab shards x 4
      chunks, fp32 logits kept on chip, per-shard + global argmax
 
 ``value`` is the sharded-linear FLOP rate of the step (algorithmic FLOPs of
 the three contractions / step time).  ``--workload stack`` runs the 4-layer
-residual stack x[4,4096,8192], 8192->28672->8192 instead.
+residual stack x[4,4096,8192], 8192->28672->8192 instead; the other workloads
+(``qkv``, ``mlp``, ``lmhead``, ``swiglu``, ``seqpar``, ``embed``, ``tp_ranks``)
+time one part or a next-step variant of the path.
 
-``--impl reference`` times the fp64 CPU oracle (the reference of this build)
-on a bounded sample of the same workload.  Under torchrun (N > 1) every rank
-runs an independent replica (the path is single-GPU; there is no exchange)
-and the step time is the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload, on the host cores, without loading the CUDA library.  Under torchrun
+(N > 1) every rank runs an independent replica (the single-GPU path has no
+exchange) and the step time is the max over ranks; ``--workload tp_ranks``
+instead runs one tensor-parallel rank per GPU, exchanging through peer memory.
 """
 from __future__ import annotations
 
@@ -84,18 +87,49 @@ def ncu_traffic(kernel: str, workload: str, sources):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and throttle reasons during the timed region, from two sources:
+    nvidia-smi every 100 ms, and NVML read every ~2 ms by a host thread.  A
+    block region of a few ms holds no nvidia-smi sample, but NVML samples fall
+    inside it; the record prefers the samples taken inside the region."""
 
     Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h: nvmlClocksEventReason*)
+    NVML_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                 "hw_thermal_slowdown": 0x40}
+    POLL_S = 0.002
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.polls = []
+        self.nvml_max = None
+
+    def _nvml_handle(self):
+        import pynvml as N
+        N.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            return N, N.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+        except Exception:
+            return N, N.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _poll(self, N, h):
+        while not self.halt.is_set():
+            try:
+                t = datetime.datetime.now()
+                sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.polls.append((t, float(sm), int(r)))
+            except Exception:
+                return
+            self.halt.wait(self.POLL_S)
 
     def start(self):
+        import threading
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -105,12 +139,18 @@ class ClockSampler:
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        try:
+            N, h = self._nvml_handle()
+            self.nvml_max = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+            self.halt = threading.Event()
+            self.thread = threading.Thread(target=self._poll, args=(N, h), daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
 
-    def stop(self, t0=None, t1=None):
-        """Median SM clock and the throttle reasons seen; with a host-time window
-        [t0, t1] (datetime.now() values) only the samples taken inside it count."""
+    def _smi_rows(self):
         if self.proc is None:
-            return None
+            return []
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -127,20 +167,42 @@ class ClockSampler:
                     continue
                 rows.append((ts, f[1:]))
         os.unlink(self.path)
+        return rows
+
+    def stop(self, t0=None, t1=None):
+        """Median SM clock and the throttle reasons seen; with a host-time window
+        [t0, t1] (datetime.now() values) only the samples taken inside it count
+        (all samples if none falls inside)."""
+        if self.thread is not None:
+            self.halt.set()
+            self.thread.join(timeout=5)
+        rows = self._smi_rows()
+        polls = list(self.polls)
         if t0 is not None and t1 is not None:
-            inside = [r for ts, r in rows if t0 <= ts <= t1]
-            rows = inside if inside else [r for _, r in rows]
+            rows_in = [r for ts, r in rows if t0 <= ts <= t1]
+            polls_in = [p for p in polls if t0 <= p[0] <= t1]
         else:
-            rows = [r for _, r in rows]
-        if not rows:
+            rows_in, polls_in = [r for _, r in rows], polls
+        if not rows and not polls:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        smi = rows_in if (rows_in or polls_in) else [r for _, r in rows]
+        reasons = {names[i] for r in smi for i in range(4) if r[5 + i] == "Active"}
+        reasons |= {n for _, _, bits in polls_in for n, b in self.NVML_BITS.items() if bits & b}
+        if polls_in:
+            sm = [p[1] for p in polls_in]
+            source = "NVML every 2 ms inside the timed region"
+        else:
+            sm = [float(r[1]) for r in smi if r[1].replace(".", "").isdigit()]
+            source = ("nvidia-smi inside the timed region" if rows_in
+                      else "nvidia-smi around the timed region (no sample inside it)")
+        mx = [float(r[2]) for _, r in rows if r[2].replace(".", "").isdigit()]
+        if self.nvml_max:
+            mx.append(self.nvml_max)
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+                "sm_min_mhz": min(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm), "smi_samples_inside": len(rows_in), "source": source}
 
 
 def clocks_rejected(clk) -> bool:
@@ -916,6 +978,57 @@ def marginal_part_ms(wl, stream, steps, part, rounds=5):
         without.append(step_region_ms(wl, stream, steps, skip=(part,)) / steps)
     return statistics.median(w - o for w, o in zip(with_p, without))
 
+TENSOR_FLOP_PER_CYCLE_SM = 8192   # dense bf16 tcgen05, per SM
+
+
+def kernel_clocks(wl, stream, steps=3, decode=10):
+    """The SM clock each launch really ran at, from the library's per-CTA
+    timing records (tpl_trace_set: %clock64 and %globaltimer of every CTA), on
+    an untimed pass of ``steps`` steps (the first is dropped: it starts from
+    idle) and a decode loop of ``decode`` LM-head launches.  nvidia-smi and NVML
+    sample a clock that a launch of a few hundred microseconds does not show.
+    Per part: median over launches of the median CTA clock, the span (first
+    CTA start to last CTA end) and the median CTA duration."""
+    import tensor_transformer_linear_b200 as T
+    launches = getattr(wl, "launches", None)
+    if not launches:
+        return None
+    dev = torch.cuda.current_device()
+    seq_of = []
+    with T.Trace(16384, dev) as tr:
+        with torch.cuda.stream(stream):
+            for k in range(steps):
+                for name, fn in launches:
+                    n0 = T.tpl_launch_count()
+                    fn(stream)
+                    seq_of.append((n0, T.tpl_launch_count(), name, k))
+            lm = dict(launches).get("lmhead_argmax")
+            if lm is not None:
+                for k in range(decode):
+                    n0 = T.tpl_launch_count()
+                    lm(stream)
+                    seq_of.append((n0, T.tpl_launch_count(), "lmhead_decode_loop", k))
+        torch.cuda.synchronize()
+    by_seq = {l["seq"]: l for l in tr.launches()}
+    per, total = {}, {}
+    for n0, n1, name, k in seq_of:
+        if k == 0:
+            continue            # the first step starts from idle
+        # a part may be several launches (one per rank); element-wise kernels leave no record
+        ls = [by_seq[q] for q in range(n0, n1) if q in by_seq]
+        if ls:
+            per.setdefault(name, []).extend(ls)
+            total.setdefault(name, []).append(sum(l["span_us"] for l in ls))
+    out = {}
+    for name, ls in per.items():
+        out[name] = {"sm_mhz": round(statistics.median(l["sm_mhz"] for l in ls), 1),
+                     "span_us": round(statistics.median(l["span_us"] for l in ls), 1),
+                     "cta_us": round(statistics.median(l["cta_us"] for l in ls), 1),
+                     "launches": len(ls),
+                     "span_us_per_call": round(statistics.median(total[name]), 1)}
+    return out
+
+
 def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
     """The 4-layer residual stack x[4,4096,8192] at full size, timed in the same
     process: long enough (about a second) to run in the power-capped regime."""
@@ -1079,6 +1192,9 @@ def main():
         if pg is not None:
             decode_ms = max_over_ranks([decode_ms], dev)[0]
 
+    # ---- the SM clock inside each launch (per-CTA timing records, untimed pass)
+    kclk = kernel_clocks(wl, stream)
+
     # ---- the HBM-bound parts alone: each launch after a read-only L2 flush (a
     # 256 MiB sum, which evicts earlier kernels' dirty lines and leaves L2
     # clean), timed with events around that launch alone; median of ALONE_LAUNCHES
@@ -1180,6 +1296,26 @@ def main():
                               f"streams over {E2E_SETS} device buffer sets, so step k+1's "
                               "upload and step k-1's download overlap step k's compute"},
         }
+        if kclk:
+            line["kernel_clocks"] = {
+                "parts": kclk,
+                "measured": "per-CTA %clock64 / %globaltimer records (tpl_trace_set) of an "
+                            "untimed pass of 3 steps, the first dropped, and a 10-launch LM-head "
+                            "decode loop; sm_mhz = median CTA cycles / duration"}
+            g = [wl.parts[i] for i in gids if wl.parts[i] in kclk]
+            if g and len(g) == len(gids):
+                span_s = sum(kclk[n]["span_us_per_call"] for n in g) * 1e-6
+                cyc = sum(kclk[n]["span_us_per_call"] * kclk[n]["sm_mhz"] for n in g)
+                mhz = cyc / sum(kclk[n]["span_us_per_call"] for n in g)
+                sms = torch.cuda.get_device_properties(dev).multi_processor_count
+                pipe = sms * TENSOR_FLOP_PER_CYCLE_SM * mhz * 1e6 / 1e12
+                a_span = wl.gemm_flops / span_s / 1e12
+                line["roofline"]["tensor_pipe_at_kernel_clock"] = {
+                    "sm_mhz": round(mhz, 1), "peak": round(pipe, 1),
+                    "achieved_in_span": round(a_span, 1), "frac": round(a_span / pipe, 4),
+                    "note": f"{sms} SMs x {TENSOR_FLOP_PER_CYCLE_SM} bf16 FLOP/cycle at the "
+                            "span-weighted SM clock the GEMM launches ran at; achieved from "
+                            "their traced spans"}
         lb = wl.lmhead_bytes()
         if lb is not None:
             lm_ms = part_ms[wl.parts.index("lmhead_argmax")]

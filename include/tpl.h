@@ -39,10 +39,10 @@
  *   - A kernel that gives up waiting on its own pipeline records
  *     TPL_ERR_TIMEOUT in a per-device status word; tpl_get_device_status reads
  *     and clears it.
- *   - The library allocates no device memory.  Its only device state is two
+ *   - The library allocates no device memory.  Its only device state is three
  *     module-level variables per device, loaded with the library: the status
- *     word and the fixed scratch of tpl_lmhead_argmax_static.  The calls are
- *     thread-safe.
+ *     word, the fixed scratch of tpl_lmhead_argmax_static and the pointer to
+ *     an optional trace buffer (tpl_trace_set).  The calls are thread-safe.
  */
 #ifndef TPL_H
 #define TPL_H
@@ -64,7 +64,7 @@ typedef enum {
   TPL_ERR_ALIGN = 5,        /* a pointer or row stride breaks the 16-byte rule     */
   TPL_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed                   */
   TPL_ERR_TIMEOUT = 7,      /* a kernel gave up waiting on its pipeline            */
-  TPL_ERR_UNSUPPORTED = 8   /* valid request outside what this build implements    */
+  TPL_ERR_UNSUPPORTED = 8   /* valid request outside what this library implements  */
 } tpl_status;
 
 typedef enum { TPL_FP32 = 0, TPL_BF16 = 1 } tpl_dtype;
@@ -500,6 +500,43 @@ const char* tpl_status_string(tpl_status s);
 /* Number of tensor-core/CUDA kernels this library enqueued in the calling
  * process since load (host-side count, for launch accounting). */
 uint64_t tpl_launch_count(void);
+
+/*
+ * Timing records of the tensor-core kernels.  (No counterpart on the pages: a
+ * measurement aid of this library.)
+ *
+ * With a trace buffer installed on the current device, every CTA of the GEMM
+ * kernels (tpl_column_linear, tpl_row_linear_reduce and the other GEMM entry
+ * points) and of the LM-head kernel appends one tpl_trace_record when it
+ * finishes.  t0_ns is %globaltimer when the CTA passed its wait on the kernel
+ * before it, t1_ns when it finished, cycles the SM clock cycles (%clock64)
+ * between the two; cycles / (t1_ns - t0_ns) is the SM clock the CTA ran at.
+ * seq is the launch's number, the value tpl_launch_count returned just before
+ * the launch, so the records of one launch share it.
+ *
+ * buffer     device memory of TPL_TRACE_HEADER_BYTES + capacity * 32 bytes,
+ *            16-byte aligned, owned by the caller; NULL removes the buffer
+ *            (tracing off, the default).  The call writes the header: a
+ *            uint32 record count (starting at 0), then the uint32 capacity.
+ *            The count keeps rising past the capacity; the records beyond
+ *            it are dropped.
+ * capacity   records the buffer holds, 1 .. UINT32_MAX.
+ * The call synchronises the device.  Install or remove the buffer while no
+ * kernel of this library runs on the device: a running kernel may record
+ * into either buffer.  Several threads sharing a device share one buffer.
+ * Errors: TPL_ERR_SHAPE (capacity out of range), TPL_ERR_ALIGN (buffer not
+ * 16-byte aligned), TPL_ERR_CUDA (the copy or the synchronisation failed).
+ */
+#define TPL_TRACE_HEADER_BYTES 16
+typedef struct tpl_trace_record {
+  uint32_t seq;
+  uint16_t kind;   /* 1: single-CTA GEMM, 2: CTA-pair GEMM, 3: LM head */
+  uint16_t cta;    /* blockIdx.x */
+  uint64_t t0_ns;
+  uint64_t t1_ns;
+  uint64_t cycles;
+} tpl_trace_record;
+tpl_status tpl_trace_set(void* buffer, int64_t capacity);
 
 #ifdef __cplusplus
 }

@@ -35,7 +35,7 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
             "tpl_argmax_merge", "tpl_column_linear_gather", "tpl_reduce_slots_allgather",
             "tpl_column_linear_rmsnorm_workspace_size", "tpl_column_linear_rmsnorm",
-            "tpl_fold_norm_scale")
+            "tpl_fold_norm_scale", "tpl_trace_set")
 
 
 class TplError(RuntimeError):
@@ -106,6 +106,7 @@ def lib():
         L.tpl_column_linear_rmsnorm.argtypes = [ctypes.POINTER(Partition), vp, i64, i64, vp, vp,
                                                 ctypes.c_float, i32, vp, vp, sz, vp]
         L.tpl_fold_norm_scale.argtypes = [vp, i64, i64, vp, i32, vp, vp]
+        L.tpl_trace_set.argtypes = [vp, i64]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -615,3 +616,66 @@ def tpl_status_string(code: int) -> str:
 
 def tpl_launch_count() -> int:
     return int(lib().tpl_launch_count())
+
+
+TRACE_HEADER_BYTES = 16
+TRACE_RECORD_BYTES = 32
+TRACE_KINDS = {1: "gemm", 2: "gemm_pair", 3: "lmhead"}
+
+
+class Trace:
+    """A trace buffer for tpl_trace_set: per-CTA timing records of the GEMM and
+    LM-head kernels (launch number, kind, CTA, %globaltimer at start and end,
+    SM cycles).  ``with Trace(capacity, device) as t: ...`` installs it on the
+    current device for the block and removes it after; ``t.records()`` reads
+    them back, ``t.launches()`` groups them per launch."""
+
+    def __init__(self, capacity: int, device="cuda"):
+        import torch
+        self.capacity = int(capacity)
+        n = (TRACE_HEADER_BYTES + TRACE_RECORD_BYTES * self.capacity) // 8
+        self.buf = torch.zeros(n, dtype=torch.int64, device=device)
+
+    def __enter__(self):
+        _check(lib().tpl_trace_set(self.buf.data_ptr(), self.capacity), "tpl_trace_set")
+        return self
+
+    def __exit__(self, *exc):
+        _check(lib().tpl_trace_set(None, 0), "tpl_trace_set")
+        return False
+
+    def records(self):
+        """[(seq, kind, cta, t0_ns, t1_ns, cycles)] in the order the CTAs finished."""
+        import numpy as np
+        raw = self.buf.cpu().numpy()
+        count = int(raw[:2].view(np.uint32)[0])
+        rec = raw[TRACE_HEADER_BYTES // 8:].view(np.uint64).reshape(-1, 4)[:min(count, self.capacity)]
+        out = []
+        for w0, t0, t1, cyc in rec.tolist():
+            out.append((w0 & 0xFFFFFFFF, (w0 >> 32) & 0xFFFF, w0 >> 48, t0, t1, cyc))
+        return out
+
+    def dropped(self) -> int:
+        import numpy as np
+        count = int(self.buf[:2].cpu().numpy().view(np.uint32)[0])
+        return max(0, count - self.capacity)
+
+    def launches(self):
+        """Per launch, in launch order: {seq, kind, ctas, span_us (first CTA start
+        to last CTA end), cta_us (median CTA duration), sm_mhz (median over CTAs
+        of cycles / duration)}."""
+        import statistics
+        by = {}
+        for seq, kind, cta, t0, t1, cyc in self.records():
+            by.setdefault(seq, []).append((kind, t0, t1, cyc))
+        out = []
+        for seq in sorted(by):
+            r = by[seq]
+            dur = [t1 - t0 for _, t0, t1, _ in r]
+            mhz = [c / (t1 - t0) * 1e3 for _, t0, t1, c in r if t1 > t0]
+            out.append({"seq": seq, "kind": TRACE_KINDS.get(r[0][0], str(r[0][0])),
+                        "ctas": len(r),
+                        "span_us": (max(x[2] for x in r) - min(x[1] for x in r)) / 1e3,
+                        "cta_us": statistics.median(dur) / 1e3,
+                        "sm_mhz": statistics.median(mhz) if mhz else None})
+        return out

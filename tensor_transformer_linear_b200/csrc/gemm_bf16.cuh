@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "trace.cuh"
 
 namespace tpl {
 
@@ -81,6 +82,7 @@ struct GemmArgs {
   // odd tiles, so a tile wave starts on the K slices the wave before it read
   // last (still in L2) when the two waves share operand blocks.
   int32_t k_serp;
+  uint32_t trace_seq;  // launch number for the optional timing records (trace.cuh)
   // Fused RMSNorm (column mode, google-research allgather_layernorm): A is
   // the raw x and the norm's scale is folded into the weight, so row m of the
   // output is act(norm_rs[m] * (x W'^T)[m] + b).  Before its first epilogue,
@@ -485,6 +487,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // the prologue above overlaps the previous kernel's tail; global memory after
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
+  const TraceStamp trace = trace_begin();
 
   const int k_total = k_steps(a);
 
@@ -685,6 +688,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) trace_end(trace, kTraceGemm, a.trace_seq);
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, 2 * kAccCols);

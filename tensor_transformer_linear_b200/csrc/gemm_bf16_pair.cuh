@@ -79,6 +79,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // the prologue above overlaps the previous kernel's tail; global memory after
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
+  const TraceStamp trace = trace_begin();
 
   const int k_total = k_steps(a);
   const uint32_t full_lead = ptx::mapa_shared(&full[0], 0);      // full[s] at + 8 s
@@ -260,6 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   ptx::tc_fence_before();
   __syncwarp();
   ptx::cluster_sync();  // every MMA, remote arrival and epilogue of the pair is done
+  if (threadIdx.x == 0) trace_end(trace, kTraceGemmPair, a.trace_seq);
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc_pair(tmem_base, 2 * kAccCols);

@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "trace.cuh"
 
 namespace tpl {
 
@@ -47,6 +48,7 @@ struct LmArgs {
   int32_t* ids;
   unsigned long long* keys;  // [tp][B], zero on entry and on exit
   unsigned int* counter;
+  uint32_t trace_seq;  // launch number for the optional timing records (trace.cuh)
 };
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).
@@ -119,6 +121,7 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
   // the prologue above overlaps the previous kernel's tail; global memory after
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
+  const TraceStamp trace = trace_begin();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -339,6 +342,7 @@ __global__ void __launch_bounds__(kLmThreads, 1) lmhead_argmax_tcgen05(const __g
 
   ptx::tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) trace_end(trace, kTraceLmHead, a.trace_seq);
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, a.tmem_cols);

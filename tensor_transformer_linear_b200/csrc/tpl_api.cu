@@ -186,6 +186,7 @@ tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, DeviceInfo* dev, cudaStream_
   if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
   a.num_tiles = static_cast<int32_t>(tiles);
   if (a.norm) a.norm_epoch = next_epoch(dev);
+  a.trace_seq = static_cast<uint32_t>(g_launch_count.load(std::memory_order_relaxed));
   if (pairs) {
     const int64_t npairs = std::min<int64_t>(tiles, dev->sm_count / 2);
     const int grid = 2 * static_cast<int>(npairs);
@@ -896,7 +897,9 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
   return TPL_OK;
 }
 
-tpl_status lmhead_launch(const tpl::LmArgs& a, int smem, int grid, cudaStream_t st) {
+tpl_status lmhead_launch(const tpl::LmArgs& args, int smem, int grid, cudaStream_t st) {
+  tpl::LmArgs a = args;
+  a.trace_seq = static_cast<uint32_t>(g_launch_count.load(std::memory_order_relaxed));
   return launch_ex(tpl::lmhead_argmax_tcgen05, dim3(grid), dim3(tpl::kLmThreads),
                    static_cast<size_t>(smem), st, a);
 }
@@ -915,6 +918,23 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
                                 workspace, ws_bytes, &a, &smem, &grid);
   if (s != TPL_OK) return s;
   return lmhead_launch(a, smem, grid, static_cast<cudaStream_t>(stream));
+}
+
+tpl_status tpl_trace_set(void* buffer, int64_t capacity) {
+  static_assert(sizeof(tpl::TraceRecord) == sizeof(tpl_trace_record), "record layout");
+  static_assert(sizeof(tpl::TraceHeader) == TPL_TRACE_HEADER_BYTES, "header layout");
+  tpl::TraceHeader* h = nullptr;
+  if (buffer != nullptr) {
+    if (capacity <= 0 || capacity > static_cast<int64_t>(UINT32_MAX)) return TPL_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(buffer) % 16 != 0) return TPL_ERR_ALIGN;
+    tpl::TraceHeader hdr{};
+    hdr.capacity = static_cast<uint32_t>(capacity);
+    if (cudaMemcpy(buffer, &hdr, sizeof(hdr), cudaMemcpyHostToDevice) != cudaSuccess)
+      return TPL_ERR_CUDA;
+    h = static_cast<tpl::TraceHeader*>(buffer);
+  }
+  if (cudaMemcpyToSymbol(tpl::g_trace, &h, sizeof(h)) != cudaSuccess) return TPL_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? TPL_OK : TPL_ERR_CUDA;
 }
 
 tpl_status tpl_get_device_status(void* stream) {

@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 23, names
+    assert len(names) == 24, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -252,3 +252,10 @@ def test_selftest_rejections():
     assert L.tpl_selftest_wait_timeout(0, None, None) == 2
     assert L.tpl_selftest_wait_timeout(2_000_000_000, None, None) == 2
     assert L.tpl_selftest_wait_timeout(1000, FAKE_ODD, None) == 5
+
+
+def test_trace_set_rejections():
+    L = T.lib()
+    assert L.tpl_trace_set(FAKE, 0) == 2                # capacity out of range
+    assert L.tpl_trace_set(FAKE, 2**32) == 2
+    assert L.tpl_trace_set(FAKE_ODD, 16) == 5           # not 16-byte aligned

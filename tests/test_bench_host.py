@@ -40,8 +40,24 @@ def test_clock_samples_outside_the_timed_window_are_dropped():
             (1300, "Active", "Not Active"), (1965, "Not Active", "Not Active")]
     c = _sampler_with(rows, now)
     clk = c.stop(now + datetime.timedelta(seconds=0.5), now + datetime.timedelta(seconds=2.5))
-    assert clk == {"sm_mhz": 1350.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
-                   "samples": 2}
+    assert {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")} == {
+        "sm_mhz": 1350.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    assert clk["source"] == "nvidia-smi inside the timed region"
+
+
+def test_nvml_samples_inside_the_window_take_precedence():
+    now = datetime.datetime.now()
+    c = _sampler_with([(1965, "Not Active", "Not Active")], now)
+    ms = datetime.timedelta(milliseconds=1)
+    # NVML polls: two inside [now+10ms, now+20ms] (one with the power-cap bit),
+    # one before it with a hardware-slowdown bit that must not count
+    c.polls = [(now + 5 * ms, 1900.0, 0x8), (now + 12 * ms, 1500.0, 0x4),
+               (now + 15 * ms, 1450.0, 0x0)]
+    c.nvml_max = 1965.0
+    clk = c.stop(now + 10 * ms, now + 20 * ms)
+    assert clk["sm_mhz"] == 1475.0 and clk["sm_min_mhz"] == 1450.0
+    assert clk["reasons"] == ["sw_power_cap"] and clk["samples"] == 2
+    assert clk["smi_samples_inside"] == 0 and clk["source"].startswith("NVML")
 
 
 def test_clock_window_with_no_samples_keeps_them_all():
