@@ -991,18 +991,23 @@ def kernel_clocks(wl, stream, steps=3, decode=10):
     CTA start to last CTA end) and the median CTA duration."""
     import tensor_transformer_linear_b200 as T
     launches = getattr(wl, "launches", None)
-    if not launches:
-        return None
     dev = torch.cuda.current_device()
     seq_of = []
     with T.Trace(16384, dev) as tr:
         with torch.cuda.stream(stream):
             for k in range(steps):
-                for name, fn in launches:
+                if launches:
+                    for name, fn in launches:
+                        n0 = T.tpl_launch_count()
+                        fn(stream)
+                        seq_of.append((n0, T.tpl_launch_count(), name, k))
+                else:
+                    # one library launch per part, in order (the stack)
                     n0 = T.tpl_launch_count()
-                    fn(stream)
-                    seq_of.append((n0, T.tpl_launch_count(), name, k))
-            lm = dict(launches).get("lmhead_argmax")
+                    wl.step(stream)
+                    for q in range(n0, min(T.tpl_launch_count(), n0 + len(wl.parts))):
+                        seq_of.append((q, q + 1, wl.parts[q - n0], k))
+            lm = dict(launches or []).get("lmhead_argmax")
             if lm is not None:
                 for k in range(decode):
                     n0 = T.tpl_launch_count()
@@ -1029,6 +1034,25 @@ def kernel_clocks(wl, stream, steps=3, decode=10):
     return out
 
 
+def tensor_pipe_at_clock(wl, kclk, dev):
+    """The GEMM launches' rate over their traced spans against the tensor
+    pipe's peak at the (span-weighted) SM clock they ran at."""
+    gids = wl.gemm_part_ids()
+    g = [wl.parts[i] for i in gids if wl.parts[i] in kclk]
+    if not g or len(g) != len(gids):
+        return None
+    span_us = sum(kclk[n]["span_us_per_call"] for n in g)
+    mhz = sum(kclk[n]["span_us_per_call"] * kclk[n]["sm_mhz"] for n in g) / span_us
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    pipe = sms * TENSOR_FLOP_PER_CYCLE_SM * mhz * 1e6 / 1e12
+    a_span = wl.gemm_flops / (span_us * 1e-6) / 1e12
+    return {"sm_mhz": round(mhz, 1), "peak": round(pipe, 1),
+            "achieved_in_span": round(a_span, 1), "frac": round(a_span / pipe, 4),
+            "note": f"{sms} SMs x {TENSOR_FLOP_PER_CYCLE_SM} bf16 FLOP/cycle at the "
+                    "span-weighted SM clock the GEMM launches ran at; achieved from "
+                    "their traced spans"}
+
+
 def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
     """The 4-layer residual stack x[4,4096,8192] at full size, timed in the same
     process: long enough (about a second) to run in the power-capped regime."""
@@ -1038,6 +1062,7 @@ def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
         wl.step(stream)
     torch.cuda.synchronize()
     ms, part_ms, launches, clk = timed_steps(wl, stream, steps, pg, dev)
+    kclk = kernel_clocks(wl, stream, steps=3)   # untimed, right after the timed steps
     if pg is not None:
         ms = max_over_ranks([ms], dev)[0]
         part_ms = max_over_ranks(part_ms, dev)
@@ -1070,6 +1095,14 @@ def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
         "measured": "CUDA events around every launch on the launching stream, mean over "
                     "the timed steps; the GEMM rate is the step's GEMM FLOPs over the sum "
                     "of its GEMM launch times"}
+    if kclk:
+        rec["kernel_clocks"] = {
+            "parts": kclk,
+            "measured": "per-CTA %clock64 / %globaltimer records (tpl_trace_set) of an untimed "
+                        "pass of 3 steps right after the timed ones, the first dropped"}
+        tp_clk = tensor_pipe_at_clock(wl, kclk, dev)
+        if tp_clk:
+            rec["tensor_pipe_at_kernel_clock"] = tp_clk
     del wl
     torch.cuda.empty_cache()
     return rec
@@ -1193,7 +1226,7 @@ def main():
             decode_ms = max_over_ranks([decode_ms], dev)[0]
 
     # ---- the SM clock inside each launch (per-CTA timing records, untimed pass)
-    kclk = kernel_clocks(wl, stream)
+    kclk = None if ranks else kernel_clocks(wl, stream)
 
     # ---- the HBM-bound parts alone: each launch after a read-only L2 flush (a
     # 256 MiB sum, which evicts earlier kernels' dirty lines and leaves L2
@@ -1302,20 +1335,9 @@ def main():
                 "measured": "per-CTA %clock64 / %globaltimer records (tpl_trace_set) of an "
                             "untimed pass of 3 steps, the first dropped, and a 10-launch LM-head "
                             "decode loop; sm_mhz = median CTA cycles / duration"}
-            g = [wl.parts[i] for i in gids if wl.parts[i] in kclk]
-            if g and len(g) == len(gids):
-                span_s = sum(kclk[n]["span_us_per_call"] for n in g) * 1e-6
-                cyc = sum(kclk[n]["span_us_per_call"] * kclk[n]["sm_mhz"] for n in g)
-                mhz = cyc / sum(kclk[n]["span_us_per_call"] for n in g)
-                sms = torch.cuda.get_device_properties(dev).multi_processor_count
-                pipe = sms * TENSOR_FLOP_PER_CYCLE_SM * mhz * 1e6 / 1e12
-                a_span = wl.gemm_flops / span_s / 1e12
-                line["roofline"]["tensor_pipe_at_kernel_clock"] = {
-                    "sm_mhz": round(mhz, 1), "peak": round(pipe, 1),
-                    "achieved_in_span": round(a_span, 1), "frac": round(a_span / pipe, 4),
-                    "note": f"{sms} SMs x {TENSOR_FLOP_PER_CYCLE_SM} bf16 FLOP/cycle at the "
-                            "span-weighted SM clock the GEMM launches ran at; achieved from "
-                            "their traced spans"}
+            tp_clk = tensor_pipe_at_clock(wl, kclk, dev)
+            if tp_clk:
+                line["roofline"]["tensor_pipe_at_kernel_clock"] = tp_clk
         lb = wl.lmhead_bytes()
         if lb is not None:
             lm_ms = part_ms[wl.parts.index("lmhead_argmax")]
