@@ -273,6 +273,8 @@ class E2EPipeline:
             self.stream.wait_event(self.ev_down[b])
         for a, t in bufs.items():
             setattr(wl, a, t)
+        if hasattr(wl, "inputs_replaced"):
+            wl.inputs_replaced()   # fresh inputs: nothing computed from the last ones holds
         wl.step(self.stream)
         self.ev_cmp[b].record(self.stream)
         self.down.wait_event(self.ev_cmp[b])
@@ -286,6 +288,8 @@ class E2EPipeline:
         torch.cuda.synchronize()
         for a, t in self.sets[0].items():
             setattr(self.wl, a, t)
+        if hasattr(self.wl, "inputs_replaced"):
+            self.wl.inputs_replaced()
 
 
 # ------------------------------------------------------------------ workloads
@@ -559,21 +563,37 @@ class NextRows:
                     T.tpl_row_linear_scatter(hs[r], ws[r], b, sq, r, tp, self.recv, stream=s)
 
             def reduce_all(s):
+                # each rank's slots summed into its slice of the residual stream,
+                # with the RMSNorm of the result written for the next step
                 for q in range(tp):
                     x_q = self.xs[q].view(rows, N)
-                    T.tpl_reduce_slots(self.recv[q], tp, N, None, x_q, y=x_q, stream=s)
-            self.launches += [("rank_rmsnorm", norm_all), ("rank_gather_gemms", gather_all),
+                    T.tpl_reduce_slots_rmsnorm(self.recv[q], tp, N, self.xn[q].view(rows, N),
+                                               self.scale, True, 1e-6, None, x_q, y=x_q,
+                                               stream=s)
+                self.xn_ready = True
+
+            # A step is the block applied again to its own output (a stack of
+            # identical layers), so each step's slot reductions also produce the
+            # next step's normalised slices; the RMSNorm launches run only after
+            # new inputs (first step, or every end-to-end step).
+            self.norm_all = norm_all
+            self.xn_ready = False
+            self.alone_launches = {"rank_rmsnorm": norm_all}
+            self.launches += [("rank_gather_gemms", gather_all),
                               ("rank_scatter_gemms", scatter_all),
                               ("rank_slot_reductions", reduce_all)]
             self.flops = self.gemm_flops = m.flops()
             self.gemm_launches = 2 * tp         # one gather and one scatter GEMM per rank
-            self.reduce_bytes = tp * (tp + 2) * rows * N * 2
+            # per rank: tp slots and the residual read, y and xn written
+            self.reduce_bytes = tp * (tp + 3) * rows * N * 2
             self.io_in, self.io_out = ["xs"], ["xs"]   # the residual stream, in place
         else:
             raise ValueError(kind)
         self.parts = [n for n, _ in self.launches]
 
     def step(self, stream, events=None, skip=()):
+        if self.kind == "tp_ranks" and not self.xn_ready:
+            self.norm_all(stream)
         for i, (name, fn) in enumerate(self.launches):
             if events is not None:
                 events[i].record(stream)
@@ -581,6 +601,9 @@ class NextRows:
                 fn(stream)
         if events is not None:
             events[len(self.launches)].record(stream)
+
+    def inputs_replaced(self):
+        self.xn_ready = False
 
     def gemm_part_ids(self):
         return [i for i, n in enumerate(self.parts)
@@ -599,7 +622,7 @@ class NextRows:
         if self.kind == "tp_ranks":
             return [("roofline_rmsnorm", "rmsnorm_cta", "rank_rmsnorm",
                      2 * 2 * self.m.M * self.m.hidden, self.m.tp),
-                    ("roofline_reduce", "reduce_slots_kernel", "rank_slot_reductions",
+                    ("roofline_reduce", "reduce_slots_rmsnorm_kernel", "rank_slot_reductions",
                      self.reduce_bytes, self.m.tp)]
         return []
 
@@ -646,12 +669,21 @@ class RankTP:
         self.gemm_flops = m.flops() / world   # this rank's GEMMs
         self.io_in, self.io_out = ["x"], ["x"]   # the residual slice, in place
         self.batch, self.seq = b, sq
+        self.xn_ready = False
 
     def step(self, stream, events=None):
+        # a step is the layer applied again to its own output (a stack of
+        # identical layers): the slot reduction also writes the next step's
+        # normalised slice, so only the first step after new inputs normalises
         mark = None if events is None else (lambda i: events[i].record(stream))
-        self.block(self.x, self.batch, self.seq, stream=stream, on_step=mark)
+        self.block(self.x, self.batch, self.seq, stream=stream, on_step=mark,
+                   normed=self.xn_ready, norm_next=self.block)
+        self.xn_ready = True
         if events is not None:
             events[len(self.parts)].record(stream)
+
+    def inputs_replaced(self):
+        self.xn_ready = False
 
     def gemm_part_ids(self):
         return [self.parts.index("rank_column_gather"), self.parts.index("rank_row_scatter")]
@@ -1302,7 +1334,8 @@ def main():
         gemm_achieved = wl.gemm_flops / (gemm_ms * 1e-3) / 1e12 if n_gemm else 0.0
         peak_t, peak_label = tensor_peak(pk, pk_kind, clk)
         traffic = ncu_traffic("gemm_bf16_tcgen05_pair", args.workload,
-                              ["gemm_bf16.cuh", "gemm_bf16_pair.cuh", "ptx.cuh", "common.cuh"])
+                              ["gemm_bf16.cuh", "gemm_bf16_pair.cuh", "ptx.cuh", "common.cuh",
+                               "trace.cuh"])
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
@@ -1350,7 +1383,7 @@ def main():
                 "measured": "inside the block steps, right after the GEMMs, from CUDA events "
                             "around the launch",
                 "traffic": ncu_traffic("lmhead_argmax_tcgen05", "lmhead",
-                                       ["lmhead.cuh", "ptx.cuh", "common.cuh"])}
+                                       ["lmhead.cuh", "ptx.cuh", "common.cuh", "trace.cuh"])}
             if lm_marginal_ms is not None and lm_marginal_ms > 0:
                 gm = lb / (lm_marginal_ms * 1e-3) / 1e9
                 line["roofline_lmhead"]["in_step_marginal"] = {

@@ -429,6 +429,29 @@ tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t 
                             const void* bias, const void* residual, void* y, void* stream);
 
 /*
+ * tpl_reduce_slots and the RMSNorm of its result in one pass (google-research
+ * allgather_layernorm applied to the next layer's input): the residual stream
+ * and the next layer's normalised input come out of one read of the slots, so
+ * the next layer needs no RMSNorm launch of its own.
+ *   y[i][n]  = bf16( sum_{s < tp} recv[s][i][n] + bias[n] + residual[i][n] ),
+ *              exactly as tpl_reduce_slots;
+ *   xn[i][n] = bf16( y[i][n] * rsqrt(mean_n y[i][n]^2 + eps) * g[n] ), on the
+ *              bf16 values of y, g = 1 + scale (centered), scale, or 1 (scale
+ *              NULL): the arithmetic of tpl_rmsnorm on y (bit for bit when
+ *              N >= 2048).
+ *   recv, bias, residual, y  as tpl_reduce_slots (y may alias residual).
+ *   scale     device fp32 [N] or NULL.   xn  device bf16 [rows][N]; aliases
+ *             none of the other buffers.
+ * rows == 0 is a no-op.  Errors: as tpl_reduce_slots, plus TPL_ERR_SHAPE for
+ * eps < 0 or NaN, TPL_ERR_NULL for a NULL xn, TPL_ERR_ALIGN unless N % 8 == 0
+ * and every buffer is 16-byte aligned, TPL_ERR_UNSUPPORTED for N > 16384.
+ */
+tpl_status tpl_reduce_slots_rmsnorm(const void* recv, int32_t tp, int64_t rows, int64_t N,
+                                    const void* bias, const void* residual, void* y,
+                                    const float* scale, int32_t centered, float eps, void* xn,
+                                    void* stream);
+
+/*
  * The same reduction, with the slice stored into EVERY rank's full output
  * (google-research: the row-parallel partials reduced over the sharded
  * contraction axis; nanotron "MLP Module" without sequence parallelism, where

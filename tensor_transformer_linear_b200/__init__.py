@@ -11,7 +11,7 @@ from ._tpl import (EXPORTED, Partition, TplError, lib, lmhead_workspace,  # noqa
                    tpl_row_linear_reduce_scatter, tpl_column_linear_allgather,
                    tpl_swiglu_column_linear, tpl_embedding_lookup, tpl_selftest_wait_timeout,
                    tpl_row_linear_scatter, tpl_reduce_slots, tpl_argmax_merge,
-                   tpl_column_linear_gather, tpl_reduce_slots_allgather,
+                   tpl_column_linear_gather, tpl_reduce_slots_allgather, tpl_reduce_slots_rmsnorm,
                    tpl_fold_norm_scale, Trace,
                    tpl_column_linear_rmsnorm, tpl_column_linear_rmsnorm_workspace_size,
                    rmsnorm_linear_workspace)

@@ -35,7 +35,7 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
             "tpl_argmax_merge", "tpl_column_linear_gather", "tpl_reduce_slots_allgather",
             "tpl_column_linear_rmsnorm_workspace_size", "tpl_column_linear_rmsnorm",
-            "tpl_fold_norm_scale", "tpl_trace_set")
+            "tpl_fold_norm_scale", "tpl_trace_set", "tpl_reduce_slots_rmsnorm")
 
 
 class TplError(RuntimeError):
@@ -97,6 +97,8 @@ def lib():
         L.tpl_row_linear_scatter.argtypes = [vp, i64, i64, i64, i64, vp, i32, i32,
                                              ctypes.POINTER(vp), vp]
         L.tpl_reduce_slots.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+        L.tpl_reduce_slots_rmsnorm.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, i32,
+                                               ctypes.c_float, vp, vp]
         L.tpl_reduce_slots_allgather.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32,
                                                  ctypes.POINTER(vp), vp]
         L.tpl_argmax_merge.argtypes = [vp, vp, i32, i64, i64, vp, vp]
@@ -544,6 +546,42 @@ def tpl_reduce_slots(recv: torch.Tensor, tp: int, N: int, bias: Optional[torch.T
         raise ValueError("y must be [rows][N]")
     _check(lib().tpl_reduce_slots(_ptr(recv), int(tp), int(rows), int(N), _ptr(bias),
                                   _ptr(residual), _ptr(y), _stream(stream)), "tpl_reduce_slots")
+    return y
+
+
+def tpl_reduce_slots_rmsnorm(recv: torch.Tensor, tp: int, N: int, xn: torch.Tensor,
+                             scale: Optional[torch.Tensor] = None, centered: bool = False,
+                             eps: float = 1e-6, bias: Optional[torch.Tensor] = None,
+                             residual: Optional[torch.Tensor] = None,
+                             y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """:func:`tpl_reduce_slots` plus ``xn = RMSNorm(y)`` (fp32 ``scale``, centred or
+    not) written in the same pass: the next layer's normalised input."""
+    _cuda(recv, "recv", torch.bfloat16)
+    if recv.numel() % (tp * N) != 0:
+        raise ValueError("recv must be [tp][rows][N]")
+    rows = recv.numel() // (tp * N)
+    if y is None:
+        y = torch.empty((rows, N), dtype=torch.bfloat16, device=recv.device)
+    _cuda(y, "y", torch.bfloat16)
+    _cuda(xn, "xn", torch.bfloat16)
+    if bias is not None:
+        _cuda(bias, "bias", torch.bfloat16)
+        if bias.numel() != N:
+            raise ValueError("bias must be [N]")
+    if residual is not None:
+        _cuda(residual, "residual", torch.bfloat16)
+        if residual.numel() != rows * N:
+            raise ValueError("residual must be [rows][N]")
+    if scale is not None:
+        _cuda(scale, "scale", torch.float32)
+        if scale.numel() != N:
+            raise ValueError("scale must be [N]")
+    if y.numel() != rows * N or xn.numel() != rows * N:
+        raise ValueError("y and xn must be [rows][N]")
+    _check(lib().tpl_reduce_slots_rmsnorm(_ptr(recv), int(tp), int(rows), int(N), _ptr(bias),
+                                          _ptr(residual), _ptr(y), _ptr(scale), int(bool(centered)),
+                                          float(eps), _ptr(xn), _stream(stream)),
+           "tpl_reduce_slots_rmsnorm")
     return y
 
 

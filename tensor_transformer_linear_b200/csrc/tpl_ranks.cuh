@@ -14,6 +14,8 @@
 //   tpl_reduce_slots        once every rank's scatter has completed, a rank sums
 //       its tp slots (in rank order, fp32) plus bias and residual: its token
 //       slice of the reduced output (the reduce-scatter).
+//   tpl_reduce_slots_rmsnorm  the same sum, plus the RMSNorm of the result (the
+//       next layer's normalised input) in the same pass over the row.
 //   tpl_reduce_slots_allgather  the same sum, stored into every rank's full
 //       [batch * seq][N] output at the rank's token rows (peer stores), so that
 //       once every rank has run it, every rank holds the whole reduced output:
@@ -76,6 +78,102 @@ __global__ void __launch_bounds__(kReduceThreads)
       if (bias != nullptr) acc += bf16_to_f(bias[i % N]);
       if (residual != nullptr) acc += bf16_to_f(residual[i]);
       y[i] = __float2bfloat16_rn(acc);
+    }
+  }
+}
+
+// reduce_slots_kernel for one row, then the RMSNorm of the rounded result
+// (rmsnorm_cta's arithmetic, so xn equals tpl_rmsnorm applied to y for rows of
+// 256 or more vectors): one 128-thread CTA per row; thread t owns the row's
+// 16-byte vectors t, t + 128, ... and keeps them in registers between the two
+// halves.  y may alias residual; xn aliases nothing.
+template <int VPT>
+__global__ void __launch_bounds__(kNormCtaThreads)
+    reduce_slots_rmsnorm_kernel(const __nv_bfloat16* __restrict__ recv, int tp, int64_t rows,
+                                int N, const __nv_bfloat16* __restrict__ bias,
+                                const __nv_bfloat16* residual, __nv_bfloat16* y,
+                                const float* __restrict__ scale, int centered, float eps,
+                                __nv_bfloat16* __restrict__ xn) {
+  __shared__ float part[kNormCtaThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int nvec = N / 8;
+  const int64_t total = rows * N;
+  const float inv_n = 1.0f / static_cast<float>(N);
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    uint4 q[VPT];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = tid + kNormCtaThreads * i;
+      if (v < nvec) {
+        const int64_t e = row * N + static_cast<int64_t>(v) * 8;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int sl = 0; sl < tp; ++sl) {
+          const uint4 r = __ldcs(reinterpret_cast<const uint4*>(recv + sl * total + e));
+          acc[0] += bf16_lo(r.x); acc[1] += bf16_hi(r.x);
+          acc[2] += bf16_lo(r.y); acc[3] += bf16_hi(r.y);
+          acc[4] += bf16_lo(r.z); acc[5] += bf16_hi(r.z);
+          acc[6] += bf16_lo(r.w); acc[7] += bf16_hi(r.w);
+        }
+        if (bias != nullptr) {
+          const uint4 r = __ldg(reinterpret_cast<const uint4*>(bias + v * 8));
+          acc[0] += bf16_lo(r.x); acc[1] += bf16_hi(r.x);
+          acc[2] += bf16_lo(r.y); acc[3] += bf16_hi(r.y);
+          acc[4] += bf16_lo(r.z); acc[5] += bf16_hi(r.z);
+          acc[6] += bf16_lo(r.w); acc[7] += bf16_hi(r.w);
+        }
+        if (residual != nullptr) {
+          const uint4 r = *reinterpret_cast<const uint4*>(residual + e);
+          acc[0] += bf16_lo(r.x); acc[1] += bf16_hi(r.x);
+          acc[2] += bf16_lo(r.y); acc[3] += bf16_hi(r.y);
+          acc[4] += bf16_lo(r.z); acc[5] += bf16_hi(r.z);
+          acc[6] += bf16_lo(r.w); acc[7] += bf16_hi(r.w);
+        }
+        q[i].x = pack_bf16x2(acc[0], acc[1]);
+        q[i].y = pack_bf16x2(acc[2], acc[3]);
+        q[i].z = pack_bf16x2(acc[4], acc[5]);
+        q[i].w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(y + e) = q[i];
+        float f[8];
+        VecTraits<__nv_bfloat16>::unpack(q[i], f);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss = fmaf(f[k], f[k], ss);
+      }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) part[w] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNormCtaThreads / 32; ++i) tot += part[i];
+    __syncthreads();  // part[] is rewritten by the next row
+    const float rinv = rsqrtf(tot * inv_n + eps);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = tid + kNormCtaThreads * i;
+      if (v < nvec) {
+        float f[8];
+        VecTraits<__nv_bfloat16>::unpack(q[i], f);
+        if (scale != nullptr) {
+          const float4* s4 = reinterpret_cast<const float4*>(scale + v * 8);
+#pragma unroll
+          for (int e4 = 0; e4 < 2; ++e4) {
+            float4 sc = __ldg(s4 + e4);
+            if (centered) {
+              sc.x += 1.f; sc.y += 1.f; sc.z += 1.f; sc.w += 1.f;
+            }
+            f[4 * e4 + 0] = f[4 * e4 + 0] * rinv * sc.x;
+            f[4 * e4 + 1] = f[4 * e4 + 1] * rinv * sc.y;
+            f[4 * e4 + 2] = f[4 * e4 + 2] * rinv * sc.z;
+            f[4 * e4 + 3] = f[4 * e4 + 3] * rinv * sc.w;
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) f[k] *= rinv;
+        }
+        __stcs(reinterpret_cast<uint4*>(xn + row * N) + v,
+               VecTraits<__nv_bfloat16>::pack(f));
+      }
     }
   }
 }
@@ -261,6 +359,45 @@ tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t 
     tpl::reduce_slots_kernel<true><<<grid, tpl::kReduceThreads, 0, st>>>(rv, tp, total, Ni, bv, res, yv);
   else
     tpl::reduce_slots_kernel<false><<<grid, tpl::kReduceThreads, 0, st>>>(rv, tp, total, Ni, bv, res, yv);
+  return launched();
+}
+
+tpl_status tpl_reduce_slots_rmsnorm(const void* recv, int32_t tp, int64_t rows, int64_t N,
+                                    const void* bias, const void* residual, void* y,
+                                    const float* scale, int32_t centered, float eps, void* xn,
+                                    void* stream) {
+  if (tp < 1 || tp > TPL_MAX_TP || rows < 0 || N < 1 || N > INT32_MAX || !(eps >= 0.0f))
+    return TPL_ERR_SHAPE;
+  if (rows > INT64_MAX / (N * tp)) return TPL_ERR_SHAPE;
+  if (rows == 0) return TPL_OK;
+  if (recv == nullptr || y == nullptr || xn == nullptr) return TPL_ERR_NULL;
+  if (N % 8 != 0 || !aligned(recv, 16) || !aligned(y, 16) || !aligned(xn, 16) ||
+      (bias && !aligned(bias, 16)) || (residual && !aligned(residual, 16)) ||
+      (scale && !aligned(scale, 16)))
+    return TPL_ERR_ALIGN;
+  const int64_t cta_vec = (N / 8 + tpl::kNormCtaThreads - 1) / tpl::kNormCtaThreads;
+  if (cta_vec > 16) return TPL_ERR_UNSUPPORTED;  // N > 16384: more than the registers hold
+  const int grid = static_cast<int>(std::min<int64_t>(rows, INT32_MAX));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* rv = static_cast<const __nv_bfloat16*>(recv);
+  const auto* bv = static_cast<const __nv_bfloat16*>(bias);
+  const auto* res = static_cast<const __nv_bfloat16*>(residual);
+  auto* yv = static_cast<__nv_bfloat16*>(y);
+  auto* xv = static_cast<__nv_bfloat16*>(xn);
+  const int Ni = static_cast<int>(N);
+  const int tc = tpl::kNormCtaThreads;
+  if (cta_vec <= 2)
+    tpl::reduce_slots_rmsnorm_kernel<2><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv, scale,
+                                                             centered, eps, xv);
+  else if (cta_vec <= 4)
+    tpl::reduce_slots_rmsnorm_kernel<4><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv, scale,
+                                                             centered, eps, xv);
+  else if (cta_vec <= 8)
+    tpl::reduce_slots_rmsnorm_kernel<8><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv, scale,
+                                                             centered, eps, xv);
+  else
+    tpl::reduce_slots_rmsnorm_kernel<16><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv,
+                                                              scale, centered, eps, xv);
   return launched();
 }
 

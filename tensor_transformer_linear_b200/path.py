@@ -17,7 +17,8 @@ from ._tpl import (Partition, TplError, tpl_argmax_merge, tpl_column_linear,
                    tpl_column_linear_rmsnorm_workspace_size, tpl_fold_norm_scale,
                    tpl_get_device_status, tpl_lmhead_argmax,
                    tpl_lmhead_workspace_size, tpl_partition_subparams, tpl_reduce_slots,
-                   tpl_reduce_slots_allgather, tpl_rmsnorm, tpl_row_linear_reduce,
+                   tpl_reduce_slots_allgather, tpl_reduce_slots_rmsnorm, tpl_rmsnorm,
+                   tpl_row_linear_reduce,
                    tpl_row_linear_scatter)
 
 
@@ -328,16 +329,26 @@ class TPRankMLP:
         self.column = ops.get("column", tpl_column_linear_gather)
         self.scatter = ops.get("scatter", tpl_row_linear_scatter)
         self.reduce = ops.get("reduce", tpl_reduce_slots)
+        self.reduce_norm = ops.get("reduce_norm", tpl_reduce_slots_rmsnorm)
         self._h = None
 
     STEPS = ("rmsnorm", "barrier_xn", "column_gather", "row_scatter", "barrier_slots",
              "reduce_slots", "barrier_done")
 
     def __call__(self, x_slice: torch.Tensor, batch: int, seq: int, stream=None,
-                 on_step: Optional[Callable] = None) -> torch.Tensor:
+                 on_step: Optional[Callable] = None, normed: bool = False,
+                 norm_next: Optional["TPRankMLP"] = None) -> torch.Tensor:
         """``x_slice`` ``[batch*seq/tp, hidden]``: this rank's tokens of the residual
         stream, updated in place to ``x + MLP(RMSNorm(x))``.  ``on_step(i)`` is
-        called before step i of :attr:`STEPS` (e.g. to record a CUDA event)."""
+        called before step i of :attr:`STEPS` (e.g. to record a CUDA event).
+
+        ``norm_next`` (the next layer, possibly this one again) makes the slot
+        reduction also write RMSNorm of the updated slice, with that layer's
+        scale, into that layer's ``xn`` (tpl_reduce_slots_rmsnorm); the next
+        call then passes ``normed=True`` and skips its RMSNorm and the barrier
+        after it: the barrier that ends this call already orders every rank's
+        normalised slice before any rank's gather.  Every rank must pass the
+        same flags (they decide which barriers run)."""
         H, tp = self.w2.shape[0], self.tp
         M = batch * seq
         sp_rows(batch, seq, tp)
@@ -346,10 +357,12 @@ class TPRankMLP:
             self._h = torch.empty(M * self.w1.shape[0], dtype=x_slice.dtype,
                                   device=x_slice.device)
         mark(0)
-        self.rmsnorm(x_slice, self.scale, self.centered, self.eps, y=self.xn.local,
-                     stream=stream)
+        if not normed:
+            self.rmsnorm(x_slice, self.scale, self.centered, self.eps, y=self.xn.local,
+                         stream=stream)
         mark(1)
-        self.barrier(stream)
+        if not normed:
+            self.barrier(stream)
         mark(2)
         h = self.column(self.part, self.xn.addrs, batch, seq, self.w1, None, self.act,
                         y=self._h, stream=stream)
@@ -359,7 +372,12 @@ class TPRankMLP:
         mark(4)
         self.barrier(stream)
         mark(5)
-        self.reduce(self.recv.local, tp, H, None, x_slice, x_slice, stream=stream)
+        if norm_next is None:
+            self.reduce(self.recv.local, tp, H, None, x_slice, x_slice, stream=stream)
+        else:
+            self.reduce_norm(self.recv.local, tp, H, norm_next.xn.local, norm_next.scale,
+                             norm_next.centered, norm_next.eps, None, x_slice, x_slice,
+                             stream=stream)
         mark(6)
         self.barrier(stream)
         return x_slice

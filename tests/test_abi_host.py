@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 24, names
+    assert len(names) == 25, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -259,3 +259,17 @@ def test_trace_set_rejections():
     assert L.tpl_trace_set(FAKE, 0) == 2                # capacity out of range
     assert L.tpl_trace_set(FAKE, 2**32) == 2
     assert L.tpl_trace_set(FAKE_ODD, 16) == 5           # not 16-byte aligned
+
+
+def test_reduce_slots_rmsnorm_rejections():
+    L = T.lib()
+    s = None
+    assert L.tpl_reduce_slots_rmsnorm(FAKE, 0, 4, 64, None, None, FAKE, None, 0, 1e-6, FAKE, s) == 2
+    assert L.tpl_reduce_slots_rmsnorm(FAKE, 2, 4, 64, None, None, FAKE, None, 0, -1.0, FAKE, s) == 2
+    assert L.tpl_reduce_slots_rmsnorm(FAKE, 2, 4, 64, None, None, FAKE, None, 0, 1e-6, None, s) == 1
+    assert L.tpl_reduce_slots_rmsnorm(FAKE, 2, 4, 60, None, None, FAKE, None, 0, 1e-6, FAKE, s) == 5
+    assert L.tpl_reduce_slots_rmsnorm(FAKE, 2, 4, 64, None, None, FAKE, FAKE_ODD, 0, 1e-6, FAKE,
+                                      s) == 5
+    assert L.tpl_reduce_slots_rmsnorm(FAKE, 2, 4, 16392, None, None, FAKE, None, 0, 1e-6, FAKE,
+                                      s) == 8
+    assert L.tpl_reduce_slots_rmsnorm(None, 2, 0, 64, None, None, None, None, 0, 1e-6, None, s) == 0

@@ -73,12 +73,26 @@ def _worker(rank, port, out):
             y_.copy_(recv_.view(tp_, -1, N_).sum(0) + res_)
             return y_
 
+        def reduce_norm(recv_, tp_, N_, xn_, scale_, centered_, eps_, bias_, res_, y_,
+                        stream=None):
+            reduce(recv_, tp_, N_, bias_, res_, y_)
+            xn_.copy_(torch.from_numpy(O.rmsnorm(y_.numpy(), scale_.double().numpy(),
+                                                 centered_, eps_)))
+            return y_
+
         wl = bench.RankTP("cpu", rank, WORLD, workload=m, exchange=exchange,
                           barrier=path.stream_barrier(),
                           ops=dict(rmsnorm=rmsnorm, column=column, scatter=scatter,
-                                   reduce=reduce))
+                                   reduce=reduce, reduce_norm=reduce_norm))
+        calls = []
+        wl.block.rmsnorm = lambda *a, **k: (calls.append("rmsnorm"), rmsnorm(*a, **k))[1]
         for _ in range(2):
             wl.step(None)
+        # the second step's RMSNorm came out of the first step's slot reduction
+        assert calls == ["rmsnorm"]
+        wl.inputs_replaced()
+        wl.step(None)
+        assert calls == ["rmsnorm", "rmsnorm"]
         out[rank] = (wl.x.numpy().copy(), wl.flops, wl.gemm_flops, wl.parts,
                      wl.gemm_part_ids())
     finally:
@@ -101,7 +115,7 @@ def test_rank_mode_of_the_bench_over_two_processes():
     x = C.mlp_x(m).numpy()
     w1, w2, s = C.mlp_w1(m).numpy(), C.mlp_w2(m).numpy(), C.mlp_scale(m).double().numpy()
     ref = x
-    for _ in range(2):            # two steps with the same weights, in place
+    for _ in range(3):            # three steps with the same weights, in place
         ref = O.tp_mlp(ref, w1, w2, WORLD, m.act, scale=s, centered=True, norm=True,
                        residual=True)
     ref_sp = O.seq_scatter(ref, m.batch, m.seq, WORLD)

@@ -159,6 +159,39 @@ def test_reduce_slots_in_place_on_the_residual():
     Bd.check(f64(y), sref, own)
 
 
+@pytest.mark.parametrize("tp,rows,N,with_bias,scale_mode,in_place", [
+    (8, 100, 4096, True, "centered", True),    # the MLP's hidden: rmsnorm_cta's arithmetic
+    (3, 37, 264, False, None, False),           # narrow rows: 33 vectors, most threads idle
+    (2, 5, 16384, False, "plain", True),        # 16 vectors per thread, the widest row
+])
+def test_reduce_slots_rmsnorm(tp, rows, N, with_bias, scale_mode, in_place):
+    recv = _t((tp, rows, N), 1.0, 6).to(DEV)
+    res = _t((rows, N), 1.0, 7)
+    bias = _t((N,), 0.02, 8).to(DEV) if with_bias else None
+    scale = (gen.normal((N,), 0.1, tensor_id=9, dtype=torch.float32).to(DEV)
+             if scale_mode else None)
+    centered = scale_mode == "centered"
+    y = res.to(DEV) if in_place else torch.empty((rows, N), dtype=torch.bfloat16, device=DEV)
+    xn = torch.empty((rows, N), dtype=torch.bfloat16, device=DEV)
+    T.tpl_reduce_slots_rmsnorm(recv, tp, N, xn, scale=scale, centered=centered, bias=bias,
+                               residual=y if in_place else res.to(DEV), y=y)
+    y_plain = T.tpl_reduce_slots(recv, tp, N, bias, res.to(DEV))
+    torch.cuda.synchronize()
+    # the residual stream: tpl_reduce_slots' arithmetic, bit for bit, and the oracle
+    assert torch.equal(y, y_plain)
+    slots = list(f64(recv)) + ([np.broadcast_to(f64(bias), (rows, N))] if with_bias else [])
+    sref, own = Bd.slot_sum(slots, f64(res))
+    Bd.check(f64(y), sref, own)
+    # the next layer's input: RMSNorm of the stored bf16 y (google-research
+    # allgather_layernorm), against the oracle ...
+    xref, own_n = Bd.rmsnorm(f64(y), None if scale is None else f64(scale), centered)
+    assert rel(xn, xref) <= TOL_BF16
+    Bd.check(f64(xn), xref, own_n)
+    # ... and, on rows of 256 or more vectors, tpl_rmsnorm's own result bit for bit
+    if N >= 2048:
+        assert torch.equal(xn, T.tpl_rmsnorm(y, scale, centered, 1e-6))
+
+
 @pytest.mark.parametrize("B,K,V,tp", [(32, 256, 4999, 4), (5, 64, 37, 8)])
 def test_lmhead_argmax_merged_over_ranks(B, K, V, tp):
     x = _t((B, K), 1.0, 0)
