@@ -437,8 +437,8 @@ tpl_status tpl_reduce_slots(const void* recv, int32_t tp, int64_t rows, int64_t 
  *              exactly as tpl_reduce_slots;
  *   xn[i][n] = bf16( y[i][n] * rsqrt(mean_n y[i][n]^2 + eps) * g[n] ), on the
  *              bf16 values of y, g = 1 + scale (centered), scale, or 1 (scale
- *              NULL): the arithmetic of tpl_rmsnorm on y (bit for bit when
- *              N >= 2048).
+ *              NULL), in fp32 as tpl_rmsnorm (the sum of squares in another
+ *              order, so the last bit of an element can differ).
  *   recv, bias, residual, y  as tpl_reduce_slots (y may alias residual).
  *   scale     device fp32 [N] or NULL.   xn  device bf16 [rows][N]; aliases
  *             none of the other buffers.

@@ -82,38 +82,54 @@ __global__ void __launch_bounds__(kReduceThreads)
   }
 }
 
-// reduce_slots_kernel for one row, then the RMSNorm of the rounded result
-// (rmsnorm_cta's arithmetic, so xn equals tpl_rmsnorm applied to y for rows of
-// 256 or more vectors): one 128-thread CTA per row; thread t owns the row's
-// 16-byte vectors t, t + 128, ... and keeps them in registers between the two
-// halves.  y may alias residual; xn aliases nothing.
+// reduce_slots_kernel for one row, then the RMSNorm of the rounded result: one
+// CTA per row, of up to kRowThreads threads, thread t owning the row's 16-byte
+// vectors t, t + blockDim, ... (VPT of them at most) in registers between the
+// two halves.  A thread loads all of a vector's slots (up to kSlots at a time)
+// before adding any, in rank order, so a row's loads are in flight together:
+// with a few rows per SM, the kernel would otherwise wait on one load round
+// trip per slot.  y may alias residual; xn aliases nothing.
+constexpr int kRowThreads = 256;
+
 template <int VPT>
-__global__ void __launch_bounds__(kNormCtaThreads)
+__global__ void __launch_bounds__(kRowThreads, 4)
     reduce_slots_rmsnorm_kernel(const __nv_bfloat16* __restrict__ recv, int tp, int64_t rows,
                                 int N, const __nv_bfloat16* __restrict__ bias,
                                 const __nv_bfloat16* residual, __nv_bfloat16* y,
                                 const float* __restrict__ scale, int centered, float eps,
                                 __nv_bfloat16* __restrict__ xn) {
-  __shared__ float part[kNormCtaThreads / 32];
+  __shared__ float part[kRowThreads / 32];
+  constexpr int kSlots = 8;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int nthr = blockDim.x;
   const int nvec = N / 8;
   const int64_t total = rows * N;
   const float inv_n = 1.0f / static_cast<float>(N);
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     uint4 q[VPT];
     float ss = 0.f;
+    const int64_t base = row * N;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const int v = tid + kNormCtaThreads * i;
+      const int v = tid + nthr * i;
       if (v < nvec) {
-        const int64_t e = row * N + static_cast<int64_t>(v) * 8;
+        const int64_t e = base + static_cast<int64_t>(v) * 8;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int sl = 0; sl < tp; ++sl) {
-          const uint4 r = __ldcs(reinterpret_cast<const uint4*>(recv + sl * total + e));
-          acc[0] += bf16_lo(r.x); acc[1] += bf16_hi(r.x);
-          acc[2] += bf16_lo(r.y); acc[3] += bf16_hi(r.y);
-          acc[4] += bf16_lo(r.z); acc[5] += bf16_hi(r.z);
-          acc[6] += bf16_lo(r.w); acc[7] += bf16_hi(r.w);
+        for (int s0 = 0; s0 < tp; s0 += kSlots) {
+          uint4 r[kSlots];
+#pragma unroll
+          for (int j = 0; j < kSlots; ++j)
+            if (s0 + j < tp)
+              r[j] = __ldcs(reinterpret_cast<const uint4*>(recv + (s0 + j) * total + e));
+#pragma unroll
+          for (int j = 0; j < kSlots; ++j) {   // added in rank order
+            if (s0 + j < tp) {
+              acc[0] += bf16_lo(r[j].x); acc[1] += bf16_hi(r[j].x);
+              acc[2] += bf16_lo(r[j].y); acc[3] += bf16_hi(r[j].y);
+              acc[4] += bf16_lo(r[j].z); acc[5] += bf16_hi(r[j].z);
+              acc[6] += bf16_lo(r[j].w); acc[7] += bf16_hi(r[j].w);
+            }
+          }
         }
         if (bias != nullptr) {
           const uint4 r = __ldg(reinterpret_cast<const uint4*>(bias + v * 8));
@@ -144,13 +160,12 @@ __global__ void __launch_bounds__(kNormCtaThreads)
     if (lane == 0) part[w] = ss;
     __syncthreads();
     float tot = 0.f;
-#pragma unroll
-    for (int i = 0; i < kNormCtaThreads / 32; ++i) tot += part[i];
+    for (int i = 0; i < (nthr >> 5); ++i) tot += part[i];
     __syncthreads();  // part[] is rewritten by the next row
     const float rinv = rsqrtf(tot * inv_n + eps);
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const int v = tid + kNormCtaThreads * i;
+      const int v = tid + nthr * i;
       if (v < nvec) {
         float f[8];
         VecTraits<__nv_bfloat16>::unpack(q[i], f);
@@ -375,8 +390,11 @@ tpl_status tpl_reduce_slots_rmsnorm(const void* recv, int32_t tp, int64_t rows, 
       (bias && !aligned(bias, 16)) || (residual && !aligned(residual, 16)) ||
       (scale && !aligned(scale, 16)))
     return TPL_ERR_ALIGN;
-  const int64_t cta_vec = (N / 8 + tpl::kNormCtaThreads - 1) / tpl::kNormCtaThreads;
-  if (cta_vec > 16) return TPL_ERR_UNSUPPORTED;  // N > 16384: more than the registers hold
+  const int64_t nvec = N / 8;
+  const int64_t vpt = (nvec + tpl::kRowThreads - 1) / tpl::kRowThreads;
+  if (vpt > 8) return TPL_ERR_UNSUPPORTED;  // N > 16384: more than the registers hold
+  // threads per row: one vector per thread up to N = 2048, then up to 8 each
+  const int tc = static_cast<int>(std::min<int64_t>(tpl::kRowThreads, (nvec + 31) / 32 * 32));
   const int grid = static_cast<int>(std::min<int64_t>(rows, INT32_MAX));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto* rv = static_cast<const __nv_bfloat16*>(recv);
@@ -385,19 +403,18 @@ tpl_status tpl_reduce_slots_rmsnorm(const void* recv, int32_t tp, int64_t rows, 
   auto* yv = static_cast<__nv_bfloat16*>(y);
   auto* xv = static_cast<__nv_bfloat16*>(xn);
   const int Ni = static_cast<int>(N);
-  const int tc = tpl::kNormCtaThreads;
-  if (cta_vec <= 2)
+  if (vpt <= 1)
+    tpl::reduce_slots_rmsnorm_kernel<1><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv, scale,
+                                                             centered, eps, xv);
+  else if (vpt <= 2)
     tpl::reduce_slots_rmsnorm_kernel<2><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv, scale,
                                                              centered, eps, xv);
-  else if (cta_vec <= 4)
+  else if (vpt <= 4)
     tpl::reduce_slots_rmsnorm_kernel<4><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv, scale,
                                                              centered, eps, xv);
-  else if (cta_vec <= 8)
+  else
     tpl::reduce_slots_rmsnorm_kernel<8><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv, scale,
                                                              centered, eps, xv);
-  else
-    tpl::reduce_slots_rmsnorm_kernel<16><<<grid, tc, 0, st>>>(rv, tp, rows, Ni, bv, res, yv,
-                                                              scale, centered, eps, xv);
   return launched();
 }
 
