@@ -1142,20 +1142,16 @@ def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
 
 def measure_tiny(dev, stream, reps=200):
     """The tiny fp32 TP MLP (x[2,16,256], 256->1024->256, tp 4, GELU tanh): the
-    latency of one block (c_fc + c_proj).  Median over ``reps`` blocks, each
-    bracketed by CUDA events, two ways: replays of the block captured once in a
-    CUDA graph (device latency: the two kernels back to back, no host work in
-    between) and eager calls through the Python binding (each launch also waits
-    for its host-side argument marshalling)."""
+    latency of one block.  Median over ``reps`` blocks, each bracketed by CUDA
+    events, two ways: replays of the block captured once in a CUDA graph (device
+    latency, no host work in between) and eager calls through the Python
+    binding (each launch also waits for its host-side argument marshalling).
+    The block runs as one fused launch (tpl_tp_mlp_fp32); the two-launch form
+    (c_fc, then c_proj with the partial-sum reduction) is timed beside it."""
     import tensor_transformer_linear_b200 as T
     w = C.TINY_MLP
     x = C.mlp_x(w, dev)
-    blk = T.TPMLP(C.mlp_w1(w, 0, dev), C.mlp_w2(w, 0, dev), w.tp, w.act, norm=False)
     y = torch.empty((w.M, w.hidden), dtype=w.dtype, device=dev)
-    with torch.cuda.stream(stream):
-        for _ in range(10):
-            blk(x, out=y)
-    torch.cuda.synchronize()
 
     def timed(run):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -1168,19 +1164,39 @@ def measure_tiny(dev, stream, reps=200):
         torch.cuda.synchronize()
         return sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
 
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        blk(x, out=y)
-    torch.cuda.synchronize()
-    tg = timed(graph.replay)
-    te = timed(lambda: blk(x, out=y))
-    del graph
+    out = {}
+    for key, fused in (("fused", True), ("two_launch", False)):
+        blk = T.TPMLP(C.mlp_w1(w, 0, dev), C.mlp_w2(w, 0, dev), w.tp, w.act, norm=False,
+                      fused_fp32=fused)
+        with torch.cuda.stream(stream):
+            for _ in range(10):
+                blk(x, out=y)
+        torch.cuda.synchronize()
+        n0 = T.tpl_launch_count()
+        with torch.cuda.stream(stream):
+            blk(x, out=y)
+        launches = T.tpl_launch_count() - n0
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            blk(x, out=y)
+        torch.cuda.synchronize()
+        tg = timed(graph.replay)
+        te = timed(lambda: blk(x, out=y))
+        del graph
+        out[key] = (tg, te, launches, blk.fused_fp32)
+    tg, te, launches, fused = out["fused"]
     us = statistics.median(tg)
     return {"workload": w.name, "dtype": "f32", "us_per_block": round(us, 2),
             "p10_us": round(tg[len(tg) // 10], 2), "p90_us": round(tg[9 * len(tg) // 10], 2),
             "eager_us_per_block": round(statistics.median(te), 2),
-            "launches_per_block": 2, "kernel": "gemm_fp32_simt", "flops_per_block": w.flops(),
+            "launches_per_block": launches,
+            "kernel": "mlp_fp32_fused" if fused else "gemm_fp32_simt",
+            "flops_per_block": w.flops(),
             "gflops": round(w.flops() / (us * 1e-6) / 1e9, 1), "bound": "latency",
+            "two_launch": {"us_per_block": round(statistics.median(out["two_launch"][0]), 2),
+                           "eager_us_per_block": round(statistics.median(out["two_launch"][1]), 2),
+                           "launches_per_block": out["two_launch"][2],
+                           "kernel": "gemm_fp32_simt"},
             "measured": f"median of {reps} blocks, CUDA events around each block on the "
                         "launching stream; us_per_block replays the block captured in a CUDA "
                         "graph, eager_us_per_block calls it through the Python binding"}

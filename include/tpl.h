@@ -500,6 +500,39 @@ tpl_status tpl_argmax_merge(const float* shard_max, const int32_t* shard_idx, in
                             int64_t B, int64_t id_stride, int32_t* ids, void* stream);
 
 /*
+ * The whole TP MLP block in fp32 in one launch, for latency (nanotron "MLP
+ * Module": c_fc column-parallel, activation, c_proj row-parallel with the
+ * partial-sum reduction; google-research residual section):
+ *   y = act(x W1^T + b1) W2^T (+ b2) (+ residual)
+ * computed as the TP shards are.  I is cut into 16 slices, each inside one
+ * rank's shard; a cluster of 16 CTAs takes one 8-row token tile and CTA s
+ * computes slice s of h (kept in shared memory: h never reaches global
+ * memory) and its partial product with W2.  The 16 partials are summed in
+ * slice order, which is rank order, then b2 and the residual are added.
+ *   x         device fp32 [M][H].
+ *   w1        device fp32 [I][H], nn.Linear layout (rank r's shard: rows
+ *             r*I/tp .. (r+1)*I/tp - 1).
+ *   b1        device fp32 [I] or NULL.
+ *   w2        device fp32; rank r's block [H][I/tp] starts at element
+ *             H * r * I/tp (the layout tpl_row_linear_reduce takes).
+ *   b2        device fp32 [H] or NULL.   residual  device fp32 [M][H] or
+ *             NULL; may alias y.
+ *   y         device fp32 [M][H].
+ * M == 0 is a no-op.  Errors: TPL_ERR_DTYPE (act), TPL_ERR_SHAPE (sizes out
+ * of range, more than 65535 tiles of 8 rows), TPL_ERR_INDIVISIBLE
+ * (I % tp != 0), TPL_ERR_NULL, TPL_ERR_ALIGN (x, w1, w2, y not 16-byte
+ * aligned).  TPL_ERR_UNSUPPORTED for the shapes this kernel does not take:
+ * 16 % tp != 0, I % 64 != 0, H % 16 != 0, shared memory
+ * 4 * (8 H + (I/16)(H + 4) + H (I/16 + 4) + 8 (I/16 + 4)) bytes above 227 KB
+ * (the tiny MLP, H 256 and I 1024, needs 147 KB), or a device that cannot
+ * hold a 16-CTA cluster of that size; the caller then runs
+ * tpl_column_linear and tpl_row_linear_reduce.
+ */
+tpl_status tpl_tp_mlp_fp32(const float* x, int64_t M, int64_t H, const float* w1,
+                          const float* b1, int64_t I, int32_t tp, tpl_act act, const float* w2,
+                          const float* b2, const float* residual, float* y, void* stream);
+
+/*
  * Self-test of the failure path.  (No counterpart on the pages: a diagnostic
  * of this library.)  Launches one thread that waits, with the bounded wait the
  * pipelines use, on an mbarrier nothing arrives on; after limit_ns (1 ns .. 1 s)

@@ -12,7 +12,7 @@ from ._tpl import (EXPORTED, Partition, TplError, lib, lmhead_workspace,  # noqa
                    tpl_swiglu_column_linear, tpl_embedding_lookup, tpl_selftest_wait_timeout,
                    tpl_row_linear_scatter, tpl_reduce_slots, tpl_argmax_merge,
                    tpl_column_linear_gather, tpl_reduce_slots_allgather, tpl_reduce_slots_rmsnorm,
-                   tpl_fold_norm_scale, Trace,
+                   tpl_fold_norm_scale, Trace, tpl_tp_mlp_fp32,
                    tpl_column_linear_rmsnorm, tpl_column_linear_rmsnorm_workspace_size,
                    rmsnorm_linear_workspace)
 from .path import (TPMLP, TPLMHeadRank, TPRankMLP, TPRowParallelAllReduceRank,  # noqa: F401

@@ -35,7 +35,8 @@ EXPORTED = ("tpl_partition_subparams", "tpl_column_linear", "tpl_row_linear_redu
             "tpl_selftest_wait_timeout", "tpl_row_linear_scatter", "tpl_reduce_slots",
             "tpl_argmax_merge", "tpl_column_linear_gather", "tpl_reduce_slots_allgather",
             "tpl_column_linear_rmsnorm_workspace_size", "tpl_column_linear_rmsnorm",
-            "tpl_fold_norm_scale", "tpl_trace_set", "tpl_reduce_slots_rmsnorm")
+            "tpl_fold_norm_scale", "tpl_trace_set", "tpl_reduce_slots_rmsnorm",
+            "tpl_tp_mlp_fp32")
 
 
 class TplError(RuntimeError):
@@ -109,6 +110,7 @@ def lib():
                                                 ctypes.c_float, i32, vp, vp, sz, vp]
         L.tpl_fold_norm_scale.argtypes = [vp, i64, i64, vp, i32, vp, vp]
         L.tpl_trace_set.argtypes = [vp, i64]
+        L.tpl_tp_mlp_fp32.argtypes = [vp, i64, i64, vp, vp, i64, i32, i32, vp, vp, vp, vp, vp]
         L.tpl_get_device_status.argtypes = [vp]
         L.tpl_status_string.argtypes = [i32]
         L.tpl_status_string.restype = ctypes.c_char_p
@@ -546,6 +548,40 @@ def tpl_reduce_slots(recv: torch.Tensor, tp: int, N: int, bias: Optional[torch.T
         raise ValueError("y must be [rows][N]")
     _check(lib().tpl_reduce_slots(_ptr(recv), int(tp), int(rows), int(N), _ptr(bias),
                                   _ptr(residual), _ptr(y), _stream(stream)), "tpl_reduce_slots")
+    return y
+
+
+def tpl_tp_mlp_fp32(x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor, tp: int, act: str,
+                    b1: Optional[torch.Tensor] = None, b2: Optional[torch.Tensor] = None,
+                    residual: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """The fp32 TP MLP block in one launch: ``act(x W1^T + b1) W2^T + b2 (+ residual)``;
+    ``w2`` in the per-rank packed layout of :func:`pack_row_weight` (equal widths).
+    Raises TplError TPL_ERR_UNSUPPORTED for shapes the fused kernel does not take."""
+    _cuda(x, "x", torch.float32)
+    _cuda(w1, "w1", torch.float32)
+    _cuda(w2, "w2", torch.float32)
+    I, H = w1.shape
+    M = x.numel() // H
+    if x.shape[-1] != H or w2.numel() != H * I:
+        raise ValueError("x must be [M][H], w1 [I][H] and w2 hold H * I elements")
+    for t, n, name in ((b1, I, "b1"), (b2, H, "b2")):
+        if t is not None:
+            _cuda(t, name, torch.float32)
+            if t.numel() != n:
+                raise ValueError(f"{name} must hold {n} elements")
+    if residual is not None:
+        _cuda(residual, "residual", torch.float32)
+        if residual.numel() != M * H:
+            raise ValueError("residual must be [M][H]")
+    if y is None:
+        y = torch.empty((M, H), dtype=torch.float32, device=x.device)
+    _cuda(y, "y", torch.float32)
+    if y.numel() != M * H:
+        raise ValueError("y must be [M][H]")
+    _check(lib().tpl_tp_mlp_fp32(_ptr(x), int(M), int(H), _ptr(w1), _ptr(b1), int(I), int(tp),
+                                 ACT[act], _ptr(w2), _ptr(b2), _ptr(residual), _ptr(y),
+                                 _stream(stream)), "tpl_tp_mlp_fp32")
     return y
 
 

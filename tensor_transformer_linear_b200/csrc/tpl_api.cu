@@ -20,6 +20,7 @@
 #include "gemm_bf16_pair.cuh"
 #include "gemm_fp32.cuh"
 #include "lmhead.cuh"
+#include "mlp_fp32.cuh"
 #include "norm_fold.cuh"
 #include "rmsnorm.cuh"
 
@@ -36,6 +37,8 @@ struct DeviceInfo {
   int sm_count = 0;
   bool gemm_attr = false;
   bool lm_attr = false;
+  bool mlp_attr = false;
+  int mlp_clusters = -1;  // clusters of the fused fp32 MLP that fit at once (-1: not asked yet)
   uint32_t epoch = 0;  // last flag epoch handed to a launch on this device
 };
 
@@ -72,6 +75,14 @@ tpl_status device_info(DeviceInfo** out) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return TPL_ERR_CUDA;
     d.lm_attr = true;
+  }
+  if (!d.mlp_attr) {
+    if (cudaFuncSetAttribute(tpl::mlp_fp32_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(tpl::mlp_fp32_fused,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return TPL_ERR_CUDA;
+    d.mlp_attr = true;
   }
   *out = &d;
   return TPL_OK;
@@ -918,6 +929,77 @@ tpl_status tpl_lmhead_argmax(const void* x, int64_t B, int64_t K, const void* w,
                                 workspace, ws_bytes, &a, &smem, &grid);
   if (s != TPL_OK) return s;
   return lmhead_launch(a, smem, grid, static_cast<cudaStream_t>(stream));
+}
+
+tpl_status tpl_tp_mlp_fp32(const float* x, int64_t M, int64_t H, const float* w1,
+                          const float* b1, int64_t I, int32_t tp, tpl_act act, const float* w2,
+                          const float* b2, const float* residual, float* y, void* stream) {
+  if (act != TPL_ACT_NONE && act != TPL_ACT_GELU_ERF && act != TPL_ACT_GELU_TANH)
+    return TPL_ERR_DTYPE;
+  if (M < 0 || H < 1 || I < 1 || tp < 1 || tp > TPL_MAX_TP || H > INT32_MAX || I > INT32_MAX)
+    return TPL_ERR_SHAPE;
+  if (I % tp != 0) return TPL_ERR_INDIVISIBLE;
+  // slices of I / 16 columns, each inside one rank's shard; 16-byte vectors
+  if (tpl::kMlpSlices % tp != 0 || I % (4 * tpl::kMlpSlices) != 0 ||
+      H % tpl::kMlpSlices != 0 || H % 4 != 0)
+    return TPL_ERR_UNSUPPORTED;
+  const int hc = static_cast<int>(I / tpl::kMlpSlices);
+  const int64_t smem = tpl::mlp_smem_floats(static_cast<int>(H), hc) * 4;
+  if (smem > 227 * 1024) return TPL_ERR_UNSUPPORTED;
+  const int64_t mtiles = (M + tpl::kMlpRows - 1) / tpl::kMlpRows;
+  if (mtiles > 65535) return TPL_ERR_SHAPE;
+  if (M == 0) return TPL_OK;
+  if (x == nullptr || w1 == nullptr || w2 == nullptr || y == nullptr) return TPL_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(y, 16) ||
+      (b1 && !aligned(b1, 4)) || (b2 && !aligned(b2, 4)) || (residual && !aligned(residual, 4)))
+    return TPL_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  tpl_status s = device_info(&dev);
+  if (s != TPL_OK) return s;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(tpl::kMlpSlices, static_cast<unsigned>(mtiles));
+  cfg.blockDim = dim3(tpl::kMlpThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = tpl::kMlpSlices;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  {
+    // a 16-CTA cluster of this shared-memory size must fit one GPC of the device
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev->mlp_clusters < 0) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, tpl::mlp_fp32_fused, &cfg) != cudaSuccess) n = 0;
+      dev->mlp_clusters = n;
+    }
+    if (dev->mlp_clusters == 0) return TPL_ERR_UNSUPPORTED;
+  }
+  if (pdl_enabled()) {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
+  }
+  tpl::MlpArgs a;
+  a.x = x;
+  a.w1 = w1;
+  a.b1 = b1;
+  a.w2 = w2;
+  a.b2 = b2;
+  a.residual = residual;
+  a.y = y;
+  a.M = M;
+  a.H = static_cast<int32_t>(H);
+  a.I = static_cast<int32_t>(I);
+  a.kr = static_cast<int32_t>(I / tp);
+  a.hc = hc;
+  a.act = act;
+  if (cudaLaunchKernelEx(&cfg, tpl::mlp_fp32_fused, a) != cudaSuccess) return TPL_ERR_CUDA;
+  return launched();
 }
 
 tpl_status tpl_trace_set(void* buffer, int64_t capacity) {

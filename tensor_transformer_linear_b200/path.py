@@ -19,7 +19,7 @@ from ._tpl import (Partition, TplError, tpl_argmax_merge, tpl_column_linear,
                    tpl_lmhead_workspace_size, tpl_partition_subparams, tpl_reduce_slots,
                    tpl_reduce_slots_allgather, tpl_reduce_slots_rmsnorm, tpl_rmsnorm,
                    tpl_row_linear_reduce,
-                   tpl_row_linear_scatter)
+                   tpl_row_linear_scatter, tpl_tp_mlp_fp32)
 
 
 def shard_views(y: torch.Tensor, p: Partition, M: int) -> List[torch.Tensor]:
@@ -55,7 +55,7 @@ class TPMLP:
     def __init__(self, w1: torch.Tensor, w2_full: torch.Tensor, tp: int, act: str,
                  scale: Optional[torch.Tensor] = None, centered: bool = False,
                  norm: bool = True, residual: bool = False, eps: float = 1e-6,
-                 fused_norm: bool = False):
+                 fused_norm: bool = False, fused_fp32: bool = True):
         self.inter, self.hidden = w1.shape
         self.part = tpl_partition_subparams([self.inter], tp, 1)
         self.k_w = [self.part.shard_width[r] for r in range(tp)]
@@ -68,6 +68,9 @@ class TPMLP:
             self.w1 = tpl_fold_norm_scale(self.w1, scale, centered)
         self._bufs = {}
         self._norm_ws = None
+        # fp32 blocks without a norm: the whole block in one launch
+        # (tpl_tp_mlp_fp32) when the kernel takes the shapes
+        self.fused_fp32 = bool(fused_fp32 and not norm and w1.dtype == torch.float32)
 
     def _buf(self, name, numel, like):
         b = self._bufs.get(name)
@@ -85,6 +88,18 @@ class TPMLP:
 
     def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
         M = x.numel() // self.hidden
+        if self.fused_fp32:
+            if out is None:
+                out = torch.empty((M, self.hidden), dtype=x.dtype, device=x.device)
+            try:
+                return tpl_tp_mlp_fp32(x.view(M, self.hidden), self.w1, self.w2,
+                                       self.part.tp_size, self.act,
+                                       residual=x.view(M, self.hidden) if self.residual else None,
+                                       y=out, stream=stream)
+            except TplError as e:
+                if e.name not in ("TPL_ERR_UNSUPPORTED", "TPL_ERR_INDIVISIBLE"):
+                    raise
+                self.fused_fp32 = False     # shapes outside the fused kernel: two launches
         if self.fused_norm:
             h = self._buf("h", M * self.inter, x)
             ws = self.norm_workspace(M, x.device)

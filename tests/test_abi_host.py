@@ -29,7 +29,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = T.lib()
     names = _declared()
-    assert len(names) == 25, names
+    assert len(names) == 26, names
     for n in names:
         assert hasattr(L, n), n
     assert sorted(names) == sorted(_tpl.EXPORTED)
@@ -273,3 +273,25 @@ def test_reduce_slots_rmsnorm_rejections():
     assert L.tpl_reduce_slots_rmsnorm(FAKE, 2, 4, 16392, None, None, FAKE, None, 0, 1e-6, FAKE,
                                       s) == 8
     assert L.tpl_reduce_slots_rmsnorm(None, 2, 0, 64, None, None, None, None, 0, 1e-6, None, s) == 0
+
+
+def test_tp_mlp_fp32_rejections():
+    L = T.lib()
+    s = None
+    ok = dict(M=32, H=256, I=1024, tp=4, act=2)
+
+    def call(x=FAKE, w1=FAKE, w2=FAKE, y=FAKE, **kw):
+        a = dict(ok, **kw)
+        return L.tpl_tp_mlp_fp32(x, a["M"], a["H"], w1, None, a["I"], a["tp"], a["act"], w2,
+                                 None, None, y, s)
+    assert call(act=3) == 4                     # unknown activation
+    assert call(M=-1) == 2 and call(H=0) == 2
+    assert call(tp=3) == 3                      # 1024 % 3
+    assert call(tp=3, I=960) == 8               # 16 % 3: slices would straddle shards
+    assert call(H=250) == 8                     # H % 16
+    assert call(I=1040) == 8                    # I % 64
+    assert call(H=512, I=2048) == 8             # shared memory above 227 KB
+    assert call(M=16 * 65536) == 2              # more token tiles than grid.y holds
+    assert call(M=0, x=None, w1=None, w2=None, y=None) == 0
+    assert call(x=None) == 1
+    assert call(y=FAKE_ODD) == 5

@@ -35,11 +35,27 @@ def _status_clean():
     assert T.tpl_get_device_status() == 0
 
 
-def test_tiny_tp_mlp_fp32_full():
+def test_tiny_tp_mlp_fp32_fused_full():
+    # the whole block in one launch (tpl_tp_mlp_fp32), h kept on chip
     w = C.TINY_MLP
     x = C.mlp_x(w)
     w1, w2 = C.mlp_w1(w), C.mlp_w2(w)
     blk = T.TPMLP(w1.to(DEV), w2.to(DEV), w.tp, w.act, norm=False)
+    n0 = T.tpl_launch_count()
+    y = blk(x.to(DEV))
+    torch.cuda.synchronize()
+    assert blk.fused_fp32 and T.tpl_launch_count() - n0 == 1
+    ref = O.tp_mlp(f64(x), f64(w1), f64(w2), w.tp, w.act)
+    assert rel(y, ref) <= TOL_FP32
+    bref, own, car = Bd.mlp(f64(x), f64(w1), f64(w2), w.tp, w.act, bf16=False)
+    Bd.check(f64(y), bref, own, car, u_out=Bd.U_FP32)
+
+
+def test_tiny_tp_mlp_fp32_full():
+    w = C.TINY_MLP
+    x = C.mlp_x(w)
+    w1, w2 = C.mlp_w1(w), C.mlp_w2(w)
+    blk = T.TPMLP(w1.to(DEV), w2.to(DEV), w.tp, w.act, norm=False, fused_fp32=False)
     y = blk(x.to(DEV))
     torch.cuda.synchronize()
     part = O.partition_subparams([w.inter], w.tp, 1)
