@@ -49,6 +49,7 @@ struct LmArgs {
   unsigned long long* keys;  // [tp][B], zero on entry and on exit
   unsigned int* counter;
   uint32_t trace_seq;  // launch number for the optional timing records (trace.cuh)
+  int32_t tn;          // 1: run lmhead_argmax_tn (batch as the M operand), lmhead_tn.cuh
 };
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).

@@ -1,0 +1,286 @@
+// lmhead_tn.cuh -- the decode LM head of lmhead.cuh with the operands the
+// other way round, for batches of up to 32 rows (Tenstorrent LMHead1D;
+// google-research unembed_manual computes the logits in fp32).
+//
+// In lmhead_argmax_tcgen05 a slab of W is the M = 128 operand and the batch
+// the N operand, so every tcgen05.mma covers 128 vocab rows x 16 K.  An MMA
+// costs about the same number of SM cycles whatever its N, so at B = 32 that
+// kernel needs about 260k SM cycles per launch: HBM-bound only while the SM
+// clock stays above about 1.6 GHz.  Here the batch is the M = 128 operand (its
+// rows past B are never read back) and a slab of slab_rows <= 256 vocab rows
+// is the N operand, so one MMA covers up to 256 vocab rows x 16 K: about half
+// the instructions for the same bytes of W, and the kernel stays HBM-bound
+// down to about 0.9 GHz.
+//
+// Stage s of the TMA ring holds the A operand [128][64] (16 KB: the batch
+// tile in rows 0..31, rows past B zero-filled by the copy, and rows 32..127
+// zeroed once at the start, so the MMA's unused rows multiply zeros and D
+// rows 32..127 stay zero), then the W tile [slab_rows][64].
+// D is [128 lanes][slab_rows] fp32 in TMEM, two buffers.  One epilogue warp
+// (TMEM lanes 0-31: lane b holds batch row b) walks each finished slab's
+// columns in ascending vocab id, keeps the best (logit, id) of the current
+// shard and folds it into the workspace with atomicMax when the shard changes
+// and at the slab's end.  The last CTA finalises as in lmhead.cuh.
+//
+// Warps: 0 epilogue, 1 TMA producer, 2 MMA issuer (and TMEM owner).
+#pragma once
+
+#include "common.cuh"
+#include "lmhead.cuh"
+#include "ptx.cuh"
+#include "trace.cuh"
+
+namespace tpl {
+
+constexpr int kLmTnThreads = 96;
+constexpr int kLmTnXBytes = 32 * kLmBK * 2;    // the batch tile a stage loads (4 KB)
+constexpr int kLmTnABytes = 128 * kLmBK * 2;   // the 128-row A operand of a stage (16 KB)
+constexpr int kLmTnAccCols = 256;              // TMEM columns per accumulator buffer
+
+__device__ __forceinline__ void lm_tn_flush(const LmArgs& a, int b, int shard, float v, int id) {
+  if (id >= 0) atomicMax(&a.keys[shard * a.B + b], make_key(v, id));
+}
+
+__global__ void __launch_bounds__(kLmTnThreads, 1)
+    lmhead_argmax_tn(const __grid_constant__ LmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.stages * a.stage_bytes);
+  uint64_t* empty = full + kLmMaxStages;
+  uint64_t* tfull = empty + kLmMaxStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int S = a.stages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&tfull[i], 1);
+      ptx::mbar_init(&tempty[i], 1);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::prefetch_tmap(&a.tmW);
+    ptx::prefetch_tmap(&a.tmX);
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(tmem_slot, a.tmem_cols);
+    ptx::tmem_relinquish();
+  }
+  // rows 32..127 of every stage's A operand: zero, never written again
+  for (int s = 0; s < S; ++s) {
+    uint4* z = reinterpret_cast<uint4*>(smem + s * a.stage_bytes + kLmTnXBytes);
+    for (int i = threadIdx.x; i < (kLmTnABytes - kLmTnXBytes) / 16; i += kLmTnThreads)
+      z[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // the prologue above overlaps the previous kernel's tail; global memory after
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const TraceStamp trace = trace_begin();
+
+  if (warp == 1) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = ptx::policy_evict_first();
+      const uint64_t pol_x = ptx::policy_evict_last();
+      const uint32_t bytes = static_cast<uint32_t>(kLmTnXBytes + a.slab_rows * kLmBK * 2);
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int slab = blockIdx.x; ok && slab < a.n_slabs; slab += gridDim.x) {
+        for (int kb = 0; kb < a.k_iters; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * a.stage_bytes;
+          ptx::mbar_arrive_expect_tx(&full[stage], bytes);
+          ptx::tma_load_2d(st, &a.tmX, &full[stage], kb * kLmBK, 0, pol_x);
+          ptx::tma_load_2d(st + kLmTnABytes, &a.tmW, &full[stage], kb * kLmBK,
+                           slab * a.slab_rows, pol_w);
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_timeout();
+        // wait (bounded) for the copies still in flight before the CTA exits
+        const int back = issued < S ? issued : S;
+        int s = stage;
+        uint32_t ph = phase;
+        volatile int no_abort = 0;
+        for (int i = 0; i < back; ++i) {
+          if (--s < 0) {
+            s = S - 1;
+            ph ^= 1u;
+          }
+          ptx::mbar_wait(&full[s], ph, &no_abort, 200000000ull);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_bf16(128, a.slab_rows);
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true, any_mma = false;
+      for (int slab = blockIdx.x; ok && slab < a.n_slabs; slab += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kLmTnAccCols;
+        for (int kb = 0; kb < a.k_iters; ++kb) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t st = ptx::smem_u32(smem + stage * a.stage_bytes);
+          const uint64_t adesc = ptx::sdesc_kmajor_sw128(st);                // batch rows
+          const uint64_t bdesc = ptx::sdesc_kmajor_sw128(st + kLmTnABytes);  // vocab rows
+#pragma unroll
+          for (int kk = 0; kk < kLmBK / 16; ++kk)
+            ptx::umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          ptx::umma_commit(&empty[stage]);
+          any_mma = true;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::umma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        record_timeout();
+        if (any_mma) {
+          volatile int no_abort = 0;
+          ptx::umma_commit(drain);
+          ptx::mbar_wait(drain, 0, &no_abort, 200000000ull);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // warp 0: TMEM lanes 0-31, lane b = batch row b
+    const int b = lane;
+    const bool row_ok = b < a.B;
+    int it = 0;
+    bool ok = true;
+    for (int slab = blockIdx.x; slab < a.n_slabs; slab += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      int w_ok = 1;
+      if (lane == 0) w_ok = ptx::mbar_wait(&tfull[acc], acc_phase, abort_flag);
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          record_timeout();
+        }
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      const int slab0 = slab * a.slab_rows;
+      const int row_end = min(slab0 + a.slab_rows, a.V);  // ids at or past it are not this slab's
+      int cur = slab0 / a.shard;                           // shard of the running best
+      int next = (cur + 1) * a.shard;                      // first id of the next shard
+      float best = 0.f;
+      int best_id = -1;
+      for (int c = 0; c < a.slab_rows; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem_base + static_cast<uint32_t>(acc * kLmTnAccCols + c), r);
+        ptx::tmem_ld_wait();
+        if (!row_ok) continue;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int v = slab0 + c + j;
+          if (v >= row_end) break;
+          const float f = __uint_as_float(r[j]);
+          if (a.logits != nullptr) a.logits[static_cast<int64_t>(b) * a.V + v] = f;
+          if (v >= next) {  // ascending ids: the previous shard is complete in this slab
+            lm_tn_flush(a, b, cur, best, best_id);
+            cur = v / a.shard;
+            next = (cur + 1) * a.shard;
+            best_id = -1;
+          }
+          if (best_id < 0 || f > best) {  // ties keep the lower id
+            best = f;
+            best_id = v;
+          }
+        }
+      }
+      if (row_ok) lm_tn_flush(a, b, cur, best, best_id);
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&tempty[acc]);
+    }
+
+    // ------------------------------------------------ completion: last CTA
+    __threadfence();
+    __syncwarp();
+    unsigned last = 0;
+    if (lane == 0) last = (atomicAdd(a.counter, 1u) == gridDim.x - 1) ? 1u : 0u;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last && ok && !*abort_flag) {
+      __threadfence();
+      for (int bb = lane; bb < a.B; bb += 32) {
+        unsigned long long best_key = 0ull;
+        for (int s = 0; s < a.tp; ++s) {
+          unsigned long long* kp = &a.keys[s * a.B + bb];
+          const unsigned long long k = __ldcg(kp);
+          if (k == 0ull) {
+            a.shard_max[s * a.B + bb] = -__int_as_float(0x7f800000);
+            a.shard_idx[s * a.B + bb] = -1;
+          } else {
+            a.shard_max[s * a.B + bb] = key_float(static_cast<uint32_t>(k >> 32));
+            a.shard_idx[s * a.B + bb] =
+                static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(k & 0xFFFFFFFFull));
+          }
+          best_key = k > best_key ? k : best_key;
+          *kp = 0ull;
+        }
+        a.ids[bb] = best_key == 0ull
+                        ? -1
+                        : static_cast<int32_t>(0xFFFFFFFFu -
+                                               static_cast<uint32_t>(best_key & 0xFFFFFFFFull));
+      }
+      if (lane == 0) *a.counter = 0u;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) trace_end(trace, kTraceLmHead, a.trace_seq);
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, a.tmem_cols);
+  }
+}
+
+}  // namespace tpl

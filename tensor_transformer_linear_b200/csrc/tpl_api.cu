@@ -20,6 +20,7 @@
 #include "gemm_bf16_pair.cuh"
 #include "gemm_fp32.cuh"
 #include "lmhead.cuh"
+#include "lmhead_tn.cuh"
 #include "mlp_fp32.cuh"
 #include "norm_fold.cuh"
 #include "rmsnorm.cuh"
@@ -72,6 +73,8 @@ tpl_status device_info(DeviceInfo** out) {
   }
   if (!d.lm_attr) {
     if (cudaFuncSetAttribute(tpl::lmhead_argmax_tcgen05,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(tpl::lmhead_argmax_tn,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return TPL_ERR_CUDA;
     d.lm_attr = true;
@@ -838,6 +841,13 @@ namespace {
 // Every check of an LM-head call and the kernel's arguments (tensor maps
 // included), with nothing enqueued; `scratch` is the keys + counter area of
 // `ws_bytes` bytes (the caller's workspace or the library's fixed array).
+// The transposed decode LM head (lmhead_tn.cuh) for batches of up to 32 rows;
+// TPL_LMHEAD_TN=0 keeps the swap-AB kernel for every batch.
+bool lmhead_tn_enabled() {
+  static const bool on = env_int("TPL_LMHEAD_TN", 0) != 0;
+  return on;
+}
+
 tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
                           int32_t tp, int32_t n_chunks, float* logits, float* shard_max,
                           int32_t* shard_idx, int32_t* ids, void* scratch, size_t ws_bytes,
@@ -905,12 +915,47 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
                                                static_cast<size_t>(tp) * B * 8);
   *smem = a->stages * a->stage_bytes + 1024 + 256 + tpl::kLmTbufBytes;
   *grid = std::min(a->n_slabs, dev->sm_count);
+  if (B <= 32 && lmhead_tn_enabled()) {
+    // The batch as the M operand, vocab slabs of 16..256 rows (a multiple of
+    // 16) as N (lmhead_tn.cuh).  Slab height: the one that gives the busiest
+    // CTA the fewest vocab rows, the taller on a tie (fewer MMAs).  For
+    // V = 128256 on 148 SMs: 176 rows, 729 slabs, 880 rows on the busiest CTA.
+    const int64_t sms = dev->sm_count;
+    int64_t best_rows = INT64_MAX, best_r = 16;
+    for (int64_t r = 256; r >= 16; r -= 16) {
+      const int64_t slabs = (V + r - 1) / r;
+      const int64_t busiest = (slabs + sms - 1) / sms * r;
+      if (busiest < best_rows) {
+        best_rows = busiest;
+        best_r = r;
+      }
+    }
+    a->tn = 1;
+    a->slab_rows = static_cast<int32_t>(best_r);
+    const uint64_t wd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(V)};
+    const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(B)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    if ((s = encode_bf16(&a->tmW, w, 2, wd, str, static_cast<uint32_t>(a->slab_rows))) != TPL_OK)
+      return s;
+    if ((s = encode_bf16(&a->tmX, x, 2, xd, str, 32u)) != TPL_OK) return s;
+    a->n_slabs = static_cast<int32_t>((V + a->slab_rows - 1) / a->slab_rows);
+    // the 128-row A operand (16 KB) and the W tile
+    a->stage_bytes = tpl::kLmTnABytes + (a->slab_rows * tpl::kLmBK * 2 + 1023) / 1024 * 1024;
+    a->stages = std::min(tpl::kLmMaxStages, (227 * 1024 - 1024 - 256) / a->stage_bytes);
+    if (a->stages < 2) return TPL_ERR_UNSUPPORTED;
+    a->tmem_cols = 2 * tpl::kLmTnAccCols;
+    *smem = a->stages * a->stage_bytes + 1024 + 256;
+    *grid = std::min(a->n_slabs, dev->sm_count);
+  }
   return TPL_OK;
 }
 
 tpl_status lmhead_launch(const tpl::LmArgs& args, int smem, int grid, cudaStream_t st) {
   tpl::LmArgs a = args;
   a.trace_seq = static_cast<uint32_t>(g_launch_count.load(std::memory_order_relaxed));
+  if (a.tn)
+    return launch_ex(tpl::lmhead_argmax_tn, dim3(grid), dim3(tpl::kLmTnThreads),
+                     static_cast<size_t>(smem), st, a);
   return launch_ex(tpl::lmhead_argmax_tcgen05, dim3(grid), dim3(tpl::kLmThreads),
                    static_cast<size_t>(smem), st, a);
 }
