@@ -47,6 +47,15 @@ from workloads import gen  # noqa: E402
 
 METRIC = "sharded-linear TFLOP/s (% bf16 peak); LM-head decode GB/s (% HBM) at 1 B200"
 DECODE_LAUNCHES = 50
+
+
+def lmhead_kernel(batch: int) -> str:
+    """The LM-head kernel the library runs for this batch (TPL_LMHEAD_TN, read
+    the way the library reads it: 2 by default)."""
+    mode = os.environ.get("TPL_LMHEAD_TN", "2").strip() or "2"
+    if batch <= 32 and mode in ("1", "2"):
+        return "lmhead_argmax_tn<64>" if mode == "2" else "lmhead_argmax_tn<128>"
+    return "lmhead_argmax_tcgen05"
 FUSED_NORM = True   # the block's RMSNorm runs inside its c_fc GEMM
 ALONE_LAUNCHES = 30
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -1389,17 +1398,19 @@ def main():
                 line["roofline"]["tensor_pipe_at_kernel_clock"] = tp_clk
         lb = wl.lmhead_bytes()
         if lb is not None:
+            lm_kernel = lmhead_kernel(C.LM_HEAD.batch)
             lm_ms = part_ms[wl.parts.index("lmhead_argmax")]
             gbs = lb / (lm_ms * 1e-3) / 1e9
             line["roofline_lmhead"] = {
-                "kernel": "lmhead_argmax_tcgen05", "bound": "hbm", "achieved": round(gbs, 1),
+                "kernel": lm_kernel, "bound": "hbm", "achieved": round(gbs, 1),
                 "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
                 "frac_of_8000": round(gbs / 8000.0, 4), "bytes_per_launch": lb,
                 "ms": round(lm_ms, 4),
                 "measured": "inside the block steps, right after the GEMMs, from CUDA events "
                             "around the launch",
-                "traffic": ncu_traffic("lmhead_argmax_tcgen05", "lmhead",
-                                       ["lmhead.cuh", "ptx.cuh", "common.cuh", "trace.cuh"])}
+                "traffic": ncu_traffic(lm_kernel, "lmhead",
+                                       ["lmhead.cuh", "lmhead_tn.cuh", "ptx.cuh", "common.cuh",
+                                        "trace.cuh"])}
             if lm_marginal_ms is not None and lm_marginal_ms > 0:
                 gm = lb / (lm_marginal_ms * 1e-3) / 1e9
                 line["roofline_lmhead"]["in_step_marginal"] = {
@@ -1412,7 +1423,7 @@ def main():
             if decode_ms is not None:
                 dg = lb / (decode_ms * 1e-3) / 1e9
                 line["roofline_lmhead_decode"] = {
-                    "kernel": "lmhead_argmax_tcgen05", "bound": "hbm", "achieved": round(dg, 1),
+                    "kernel": lm_kernel, "bound": "hbm", "achieved": round(dg, 1),
                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(dg / pk["hbm_gbs"], 4),
                     "frac_of_8000": round(dg / 8000.0, 4), "ms_per_launch": round(decode_ms, 4),
                     "measured": f"{DECODE_LAUNCHES} back-to-back launches (a decode loop), "

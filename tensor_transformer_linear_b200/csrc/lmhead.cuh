@@ -49,7 +49,7 @@ struct LmArgs {
   unsigned long long* keys;  // [tp][B], zero on entry and on exit
   unsigned int* counter;
   uint32_t trace_seq;  // launch number for the optional timing records (trace.cuh)
-  int32_t tn;          // 1: run lmhead_argmax_tn (batch as the M operand), lmhead_tn.cuh
+  int32_t tn;          // 128 or 64: run lmhead_argmax_tn<tn> (lmhead_tn.cuh); 0: this kernel
 };
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).

@@ -6,23 +6,26 @@
 // the N operand, so every tcgen05.mma covers 128 vocab rows x 16 K.  An MMA
 // costs about the same number of SM cycles whatever its N, so at B = 32 that
 // kernel needs about 260k SM cycles per launch: HBM-bound only while the SM
-// clock stays above about 1.6 GHz.  Here the batch is the M = 128 operand (its
-// rows past B are never read back) and a slab of slab_rows <= 256 vocab rows
-// is the N operand, so one MMA covers up to 256 vocab rows x 16 K: about half
-// the instructions for the same bytes of W, and the kernel stays HBM-bound
-// down to about 0.9 GHz.
+// clock stays above about 1.6 GHz.  Here the batch is the M operand and a
+// slab of slab_rows <= 256 vocab rows is the N operand, so one MMA covers up
+// to 256 vocab rows x 16 K: about half the instructions for the same bytes of
+// W, and the kernel stays HBM-bound down to about 1 GHz.
 //
-// Stage s of the TMA ring holds the A operand [128][64] (16 KB: the batch
-// tile in rows 0..31, rows past B zero-filled by the copy, and rows 32..127
-// zeroed once at the start, so the MMA's unused rows multiply zeros and D
-// rows 32..127 stay zero), then the W tile [slab_rows][64].
-// D is [128 lanes][slab_rows] fp32 in TMEM, two buffers.  One epilogue warp
-// (TMEM lanes 0-31: lane b holds batch row b) walks each finished slab's
-// columns in ascending vocab id, keeps the best (logit, id) of the current
-// shard and folds it into the workspace with atomicMax when the shard changes
-// and at the slab's end.  The last CTA finalises as in lmhead.cuh.
+// kM is the height of the A operand: 128, or 64 (half the A bytes the tensor
+// core reads from shared memory per MMA, and more stages in the same space).
+// Stage s of the TMA ring holds the A operand [kM][64] (the batch tile in rows
+// 0..31, rows past B zero-filled by the copy, rows 32..kM-1 zeroed once at the
+// start, so the MMA's unused rows multiply zeros), then the W tile
+// [slab_rows][64].  D is [kM rows][slab_rows] fp32 in TMEM, two buffers.  For
+// kM = 128, D row i is TMEM lane i; for kM = 64, rows 0-15 are lanes 0-15 and
+// rows 16-31 lanes 32-47 (16 lanes of each 32-lane quarter).  The epilogue
+// warps (warp q reads lane quarter q) walk each finished slab's columns in
+// ascending vocab id, keep the best (logit, id) of the current shard per batch
+// row and fold it into the workspace with atomicMax when the shard changes and
+// at the slab's end.  The last CTA finalises as in lmhead.cuh.
 //
-// Warps: 0 epilogue, 1 TMA producer, 2 MMA issuer (and TMEM owner).
+// Warps: 0 .. E-1 epilogue (E = 1 for kM = 128, 2 for kM = 64), E TMA
+// producer, E + 1 MMA issuer (and TMEM owner).
 #pragma once
 
 #include "common.cuh"
@@ -32,17 +35,25 @@
 
 namespace tpl {
 
-constexpr int kLmTnThreads = 96;
-constexpr int kLmTnXBytes = 32 * kLmBK * 2;    // the batch tile a stage loads (4 KB)
-constexpr int kLmTnABytes = 128 * kLmBK * 2;   // the 128-row A operand of a stage (16 KB)
-constexpr int kLmTnAccCols = 256;              // TMEM columns per accumulator buffer
+constexpr int kLmTnXBytes = 32 * kLmBK * 2;  // the batch tile a stage loads (4 KB)
+constexpr int kLmTnAccCols = 256;            // TMEM columns per accumulator buffer
+
+template <int kM>
+struct LmTn {
+  static constexpr int kEpi = kM == 128 ? 1 : 2;           // epilogue warps
+  static constexpr int kLaneRows = kM == 128 ? 32 : 16;    // batch rows per epilogue warp
+  static constexpr int kThreads = 32 * (kEpi + 2);
+  static constexpr int kABytes = kM * kLmBK * 2;           // A operand of a stage
+};
 
 __device__ __forceinline__ void lm_tn_flush(const LmArgs& a, int b, int shard, float v, int id) {
   if (id >= 0) atomicMax(&a.keys[shard * a.B + b], make_key(v, id));
 }
 
-__global__ void __launch_bounds__(kLmTnThreads, 1)
+template <int kM>
+__global__ void __launch_bounds__(LmTn<kM>::kThreads, 1)
     lmhead_argmax_tn(const __grid_constant__ LmArgs a) {
+  using C = LmTn<kM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -53,10 +64,12 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int S = a.stages;
+  constexpr int kProd = C::kEpi, kMma = C::kEpi + 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -65,22 +78,23 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&tfull[i], 1);
-      ptx::mbar_init(&tempty[i], 1);
+      ptx::mbar_init(&tempty[i], C::kEpi);
     }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
+    *last_flag = 0;
     ptx::fence_barrier_init();
     ptx::prefetch_tmap(&a.tmW);
     ptx::prefetch_tmap(&a.tmX);
   }
-  if (warp == 2) {
+  if (warp == kMma) {
     ptx::tmem_alloc(tmem_slot, a.tmem_cols);
     ptx::tmem_relinquish();
   }
-  // rows 32..127 of every stage's A operand: zero, never written again
+  // rows 32..kM-1 of every stage's A operand: zero, never written again
   for (int s = 0; s < S; ++s) {
     uint4* z = reinterpret_cast<uint4*>(smem + s * a.stage_bytes + kLmTnXBytes);
-    for (int i = threadIdx.x; i < (kLmTnABytes - kLmTnXBytes) / 16; i += kLmTnThreads)
+    for (int i = threadIdx.x; i < (C::kABytes - kLmTnXBytes) / 16; i += C::kThreads)
       z[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
@@ -93,7 +107,7 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
   ptx::griddep_launch_dependents();
   const TraceStamp trace = trace_begin();
 
-  if (warp == 1) {
+  if (warp == kProd) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_w = ptx::policy_evict_first();
@@ -111,7 +125,7 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
           uint8_t* st = smem + stage * a.stage_bytes;
           ptx::mbar_arrive_expect_tx(&full[stage], bytes);
           ptx::tma_load_2d(st, &a.tmX, &full[stage], kb * kLmBK, 0, pol_x);
-          ptx::tma_load_2d(st + kLmTnABytes, &a.tmW, &full[stage], kb * kLmBK,
+          ptx::tma_load_2d(st + C::kABytes, &a.tmW, &full[stage], kb * kLmBK,
                            slab * a.slab_rows, pol_w);
           ++issued;
           if (++stage == S) {
@@ -137,10 +151,10 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
         }
       }
     }
-  } else if (warp == 2) {
+  } else if (warp == kMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = ptx::idesc_bf16(128, a.slab_rows);
+      const uint32_t idesc = ptx::idesc_bf16(kM, a.slab_rows);
       int stage = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true, any_mma = false;
@@ -161,7 +175,7 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
           ptx::tc_fence_after();
           const uint32_t st = ptx::smem_u32(smem + stage * a.stage_bytes);
           const uint64_t adesc = ptx::sdesc_kmajor_sw128(st);                // batch rows
-          const uint64_t bdesc = ptx::sdesc_kmajor_sw128(st + kLmTnABytes);  // vocab rows
+          const uint64_t bdesc = ptx::sdesc_kmajor_sw128(st + C::kABytes);  // vocab rows
 #pragma unroll
           for (int kk = 0; kk < kLmBK / 16; ++kk)
             ptx::umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
@@ -187,9 +201,11 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // warp 0: TMEM lanes 0-31, lane b = batch row b
-    const int b = lane;
-    const bool row_ok = b < a.B;
+    // warp q reads TMEM lane quarter q; its lane l holds batch row
+    // q * kLaneRows + l for l < kLaneRows
+    const int b = warp * C::kLaneRows + lane;
+    const bool row_ok = lane < C::kLaneRows && b < a.B;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     int it = 0;
     bool ok = true;
     for (int slab = blockIdx.x; slab < a.n_slabs; slab += gridDim.x, ++it) {
@@ -214,7 +230,7 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
       int best_id = -1;
       for (int c = 0; c < a.slab_rows; c += 16) {
         uint32_t r[16];
-        tmem_ld16(tmem_base + static_cast<uint32_t>(acc * kLmTnAccCols + c), r);
+        tmem_ld16(tmem_base + lane_base + static_cast<uint32_t>(acc * kLmTnAccCols + c), r);
         ptx::tmem_ld_wait();
         if (!row_ok) continue;
 #pragma unroll
@@ -243,13 +259,12 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
 
     // ------------------------------------------------ completion: last CTA
     __threadfence();
-    __syncwarp();
-    unsigned last = 0;
-    if (lane == 0) last = (atomicAdd(a.counter, 1u) == gridDim.x - 1) ? 1u : 0u;
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last && ok && !*abort_flag) {
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * C::kEpi) : "memory");
+    if (threadIdx.x == 0) *last_flag = (atomicAdd(a.counter, 1u) == gridDim.x - 1) ? 1 : 0;
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * C::kEpi) : "memory");
+    if (*last_flag && ok && !*abort_flag) {
       __threadfence();
-      for (int bb = lane; bb < a.B; bb += 32) {
+      for (int bb = threadIdx.x; bb < a.B; bb += 32 * C::kEpi) {
         unsigned long long best_key = 0ull;
         for (int s = 0; s < a.tp; ++s) {
           unsigned long long* kp = &a.keys[s * a.B + bb];
@@ -270,14 +285,14 @@ __global__ void __launch_bounds__(kLmTnThreads, 1)
                         : static_cast<int32_t>(0xFFFFFFFFu -
                                                static_cast<uint32_t>(best_key & 0xFFFFFFFFull));
       }
-      if (lane == 0) *a.counter = 0u;
+      if (threadIdx.x == 0) *a.counter = 0u;
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) trace_end(trace, kTraceLmHead, a.trace_seq);
-  if (warp == 2) {
+  if (warp == kMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, a.tmem_cols);
   }

@@ -74,7 +74,9 @@ tpl_status device_info(DeviceInfo** out) {
   if (!d.lm_attr) {
     if (cudaFuncSetAttribute(tpl::lmhead_argmax_tcgen05,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(tpl::lmhead_argmax_tn,
+        cudaFuncSetAttribute(tpl::lmhead_argmax_tn<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(tpl::lmhead_argmax_tn<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return TPL_ERR_CUDA;
     d.lm_attr = true;
@@ -841,11 +843,14 @@ namespace {
 // Every check of an LM-head call and the kernel's arguments (tensor maps
 // included), with nothing enqueued; `scratch` is the keys + counter area of
 // `ws_bytes` bytes (the caller's workspace or the library's fixed array).
-// The transposed decode LM head (lmhead_tn.cuh) for batches of up to 32 rows;
-// TPL_LMHEAD_TN=0 keeps the swap-AB kernel for every batch.
-bool lmhead_tn_enabled() {
-  static const bool on = env_int("TPL_LMHEAD_TN", 0) != 0;
-  return on;
+// The transposed decode LM head (lmhead_tn.cuh) for batches of up to 32 rows,
+// with a 64-row A operand (TPL_LMHEAD_TN=2, the default) or a 128-row one (1);
+// TPL_LMHEAD_TN=0 keeps the swap-AB kernel for every batch.  Measured on one
+// B200 at B = 32: even with swap-AB at a 1.8 GHz SM clock (within 1-3 us of
+// 158 us), 18-29 us faster at 1.2-1.4 GHz.  Returns the A operand height, or 0.
+int lmhead_tn_rows() {
+  static const int v = env_int("TPL_LMHEAD_TN", 2);
+  return v == 1 ? 128 : (v == 2 ? 64 : 0);
 }
 
 tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, int64_t V,
@@ -915,7 +920,7 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
                                                static_cast<size_t>(tp) * B * 8);
   *smem = a->stages * a->stage_bytes + 1024 + 256 + tpl::kLmTbufBytes;
   *grid = std::min(a->n_slabs, dev->sm_count);
-  if (B <= 32 && lmhead_tn_enabled()) {
+  if (B <= 32 && lmhead_tn_rows() != 0) {
     // The batch as the M operand, vocab slabs of 16..256 rows (a multiple of
     // 16) as N (lmhead_tn.cuh).  Slab height: the one that gives the busiest
     // CTA the fewest vocab rows, the taller on a tie (fewer MMAs).  For
@@ -930,7 +935,7 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
         best_r = r;
       }
     }
-    a->tn = 1;
+    a->tn = lmhead_tn_rows();
     a->slab_rows = static_cast<int32_t>(best_r);
     const uint64_t wd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(V)};
     const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(B)};
@@ -939,8 +944,8 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
       return s;
     if ((s = encode_bf16(&a->tmX, x, 2, xd, str, 32u)) != TPL_OK) return s;
     a->n_slabs = static_cast<int32_t>((V + a->slab_rows - 1) / a->slab_rows);
-    // the 128-row A operand (16 KB) and the W tile
-    a->stage_bytes = tpl::kLmTnABytes + (a->slab_rows * tpl::kLmBK * 2 + 1023) / 1024 * 1024;
+    // the A operand (a->tn rows) and the W tile
+    a->stage_bytes = a->tn * tpl::kLmBK * 2 + (a->slab_rows * tpl::kLmBK * 2 + 1023) / 1024 * 1024;
     a->stages = std::min(tpl::kLmMaxStages, (227 * 1024 - 1024 - 256) / a->stage_bytes);
     if (a->stages < 2) return TPL_ERR_UNSUPPORTED;
     a->tmem_cols = 2 * tpl::kLmTnAccCols;
@@ -953,8 +958,11 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
 tpl_status lmhead_launch(const tpl::LmArgs& args, int smem, int grid, cudaStream_t st) {
   tpl::LmArgs a = args;
   a.trace_seq = static_cast<uint32_t>(g_launch_count.load(std::memory_order_relaxed));
-  if (a.tn)
-    return launch_ex(tpl::lmhead_argmax_tn, dim3(grid), dim3(tpl::kLmTnThreads),
+  if (a.tn == 64)
+    return launch_ex(tpl::lmhead_argmax_tn<64>, dim3(grid), dim3(tpl::LmTn<64>::kThreads),
+                     static_cast<size_t>(smem), st, a);
+  if (a.tn == 128)
+    return launch_ex(tpl::lmhead_argmax_tn<128>, dim3(grid), dim3(tpl::LmTn<128>::kThreads),
                      static_cast<size_t>(smem), st, a);
   return launch_ex(tpl::lmhead_argmax_tcgen05, dim3(grid), dim3(tpl::kLmThreads),
                    static_cast<size_t>(smem), st, a);

@@ -1,6 +1,8 @@
-"""The transposed decode LM head (lmhead_tn.cuh: the batch as the M operand,
-vocab slabs as N), which TPL_LMHEAD_TN=1 selects for batches of up to 32 rows.
-The variable is read once per process, so the LM-head parity tests (every case,
+"""The decode LM head's other kernels.  For batches of up to 32 rows the
+library runs the transposed kernel with a 64-row A operand (lmhead_tn.cuh,
+TPL_LMHEAD_TN=2, the default); TPL_LMHEAD_TN=1 selects its 128-row form and
+TPL_LMHEAD_TN=0 the swap-AB kernel (lmhead.cuh), which larger batches always
+use.  The variable is read once per process, so the LM-head parity tests (every case,
 the planted ids and cross-shard ties, the full-size decode workload, the merged
 ranks and the static-scratch entry point) run again in a child process with it
 set; they compare against the same fp64 oracle."""
@@ -14,8 +16,9 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def test_lmhead_parity_with_the_transposed_kernel():
-    env = dict(os.environ, TPL_LMHEAD_TN="1")
+@pytest.mark.parametrize("mode", ["0", "1"])
+def test_lmhead_parity_with_the_transposed_kernel(mode):
+    env = dict(os.environ, TPL_LMHEAD_TN=mode)
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
            "tests/test_gpu_kernels.py", "tests/test_gpu_workloads.py", "tests/test_gpu_ranks.py",
            "tests/test_zz_no_alloc.py", "-k", "lmhead or argmax or no_alloc or static"]
