@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kReduceThreads)
 constexpr int kRowThreads = 256;
 
 template <int VPT>
-__global__ void __launch_bounds__(kRowThreads, 4)
+__global__ void __launch_bounds__(kRowThreads, VPT <= 2 ? 4 : (VPT <= 4 ? 2 : 1))
     reduce_slots_rmsnorm_kernel(const __nv_bfloat16* __restrict__ recv, int tp, int64_t rows,
                                 int N, const __nv_bfloat16* __restrict__ bias,
                                 const __nv_bfloat16* residual, __nv_bfloat16* y,
