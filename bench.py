@@ -1149,6 +1149,36 @@ def measure_stack(args, dev, stream, pg, world, pk, pk_kind):
     return rec
 
 
+def host_link_ms(dev, bytes_in, bytes_out, reps=5):
+    """Time to move one step's upload and download bytes over the host link at
+    once (pinned buffers, one stream per direction, no compute): the floor of
+    the end-to-end step."""
+    try:
+        h_in = torch.empty(int(bytes_in), dtype=torch.uint8, pin_memory=True)
+        h_out = torch.empty(int(bytes_out), dtype=torch.uint8, pin_memory=True)
+        d_in = torch.empty(int(bytes_in), dtype=torch.uint8, device=dev)
+        d_out = torch.empty(int(bytes_out), dtype=torch.uint8, device=dev)
+    except RuntimeError:
+        return None
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ts = []
+    for _ in range(reps + 1):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(up)
+        down.wait_event(a)
+        with torch.cuda.stream(up):
+            d_in.copy_(h_in, non_blocking=True)
+        with torch.cuda.stream(down):
+            h_out.copy_(d_out, non_blocking=True)
+        up.wait_stream(down)
+        b.record(up)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    del h_in, h_out, d_in, d_out
+    return statistics.median(ts[1:])
+
+
 def measure_tiny(dev, stream, reps=200):
     """The tiny fp32 TP MLP (x[2,16,256], 256->1024->256, tp 4, GELU tanh): the
     latency of one block.  Median over ``reps`` blocks, each bracketed by CUDA
@@ -1329,6 +1359,7 @@ def main():
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
     e2e.close()
+    link_ms = host_link_ms(dev, b_in, b_out)
 
     if pg is not None:
         ms, e_ms = max_over_ranks([ms, e_ms], dev)
@@ -1387,6 +1418,15 @@ def main():
                               f"streams over {E2E_SETS} device buffer sets, so step k+1's "
                               "upload and step k-1's download overlap step k's compute"},
         }
+        if link_ms:
+            bound = replica_rate(copies, wl.flops, max(link_ms, step_ms))
+            line["e2e"]["host_link_bound"] = {
+                "value": round(bound, 2), "frac": round(e2e_val / bound, 4),
+                "copy_ms_per_step": round(link_ms, 4),
+                "measured": "one step's upload and download bytes copied at the same time "
+                            "between pinned host buffers and the device, no compute, median "
+                            "of 5; the bound is the step's FLOPs over the longer of that "
+                            "and the device step time"}
         if kclk:
             line["kernel_clocks"] = {
                 "parts": kclk,
