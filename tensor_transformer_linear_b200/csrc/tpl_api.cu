@@ -661,7 +661,7 @@ const char* tpl_status_string(tpl_status s) {
     case TPL_ERR_ALIGN: return "TPL_ERR_ALIGN: pointer or row stride breaks the 16-byte rule";
     case TPL_ERR_CUDA: return "TPL_ERR_CUDA: a CUDA call failed";
     case TPL_ERR_TIMEOUT: return "TPL_ERR_TIMEOUT: a kernel gave up waiting on its pipeline";
-    case TPL_ERR_UNSUPPORTED: return "TPL_ERR_UNSUPPORTED: outside what this build implements";
+    case TPL_ERR_UNSUPPORTED: return "TPL_ERR_UNSUPPORTED: outside what this library implements";
   }
   return "unknown tpl_status";
 }
