@@ -47,6 +47,7 @@ from workloads import gen  # noqa: E402
 
 METRIC = "sharded-linear TFLOP/s (% bf16 peak); LM-head decode GB/s (% HBM) at 1 B200"
 DECODE_LAUNCHES = 50
+PARTS_PAUSE_S = 0.3
 
 
 def lmhead_kernel(batch: int) -> str:
@@ -985,7 +986,11 @@ def timed_steps(wl, stream, steps, pg, dev):
             pg.barrier()
         if T.tpl_get_device_status(stream) != 0:
             raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
-        # per-launch times: a second pass with an event between every two launches
+        # per-launch times: a second pass with an event between every two
+        # launches, after an idle pause so that it starts from the power state
+        # the timed region started from (the power limit lowers the clock
+        # within tens of milliseconds of load)
+        time.sleep(PARTS_PAUSE_S)
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
                for _ in range(steps)]
         for k in range(steps):
