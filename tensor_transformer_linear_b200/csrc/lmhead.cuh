@@ -50,6 +50,13 @@ struct LmArgs {
   unsigned int* counter;
   uint32_t trace_seq;  // launch number for the optional timing records (trace.cuh)
   int32_t tn;          // 128 or 64: run lmhead_argmax_tn<tn> (lmhead_tn.cuh); 0: this kernel
+  // lmhead_argmax_tn only.  ranged = 0: slab g covers rows [g slab_rows, ...)
+  // and CTA c takes slabs c, c + grid, ...  ranged = 1: CTA c owns the
+  // contiguous rows [c range_base + min(c, range_rem), + range_base + (c <
+  // range_rem)), cut into slabs of slab_rows (= 256) and one shorter last slab,
+  // loaded through tmWt (box {64, tail_rows}) and multiplied with N = tail_n.
+  int32_t ranged, range_base, range_rem, tail_rows, tail_n;
+  CUtensorMap tmWt;
 };
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).

@@ -7,16 +7,21 @@
 // costs about the same number of SM cycles whatever its N, so at B = 32 that
 // kernel needs about 260k SM cycles per launch: HBM-bound only while the SM
 // clock stays above about 1.6 GHz.  Here the batch is the M operand and a
-// slab of slab_rows <= 256 vocab rows is the N operand, so one MMA covers up
-// to 256 vocab rows x 16 K: about half the instructions for the same bytes of
-// W, and the kernel stays HBM-bound down to about 1 GHz.
+// slab of up to 256 vocab rows is the N operand, so one MMA covers up to 256
+// vocab rows x 16 K.  By default each CTA owns one contiguous vocab range
+// (V / grid rows, +1 for the first V % grid CTAs) cut into 256-row slabs and
+// one shorter last slab: for V = 128256 on 148 SMs, 4 x 256 MMAs per CTA,
+// against 7 x 256 for swap-AB and 5 x 256 for uniform 176-row slabs dealt out
+// in turn (LmArgs::ranged = 0, which the kernel also runs).
 //
 // kM is the height of the A operand: 128, or 64 (half the A bytes the tensor
 // core reads from shared memory per MMA, and more stages in the same space).
 // Stage s of the TMA ring holds the A operand [kM][64] (the batch tile in rows
 // 0..31, rows past B zero-filled by the copy, rows 32..kM-1 zeroed once at the
 // start, so the MMA's unused rows multiply zeros), then the W tile
-// [slab_rows][64].  D is [kM rows][slab_rows] fp32 in TMEM, two buffers.  For
+// [slab_rows][64] (a short last slab fills its first rows; the MMA's columns
+// past the slab's rows are never read).  D is [kM rows][N] fp32 in TMEM, two
+// buffers of 256 columns.  For
 // kM = 128, D row i is TMEM lane i; for kM = 64, rows 0-15 are lanes 0-15 and
 // rows 16-31 lanes 32-47 (16 lanes of each 32-lane quarter).  The epilogue
 // warps (warp q reads lane quarter q) walk each finished slab's columns in
@@ -45,6 +50,31 @@ struct LmTn {
   static constexpr int kThreads = 32 * (kEpi + 2);
   static constexpr int kABytes = kM * kLmBK * 2;           // A operand of a stage
 };
+
+// Slab s of this CTA: its first vocab row and its rows; false past the last.
+// Uniform slabs (ranged = 0) are dealt out in turn; with ranged = 1 the CTA
+// walks its own contiguous range (LmArgs).
+__device__ __forceinline__ bool lm_tn_slab(const LmArgs& a, int s, int& row0, int& rows) {
+  if (!a.ranged) {
+    const int g = static_cast<int>(blockIdx.x) + s * static_cast<int>(gridDim.x);
+    if (g >= a.n_slabs) return false;
+    row0 = g * a.slab_rows;
+    rows = min(a.slab_rows, a.V - row0);
+    return true;
+  }
+  const int c = static_cast<int>(blockIdx.x);
+  const int r0 = c * a.range_base + min(c, a.range_rem);
+  const int r1 = r0 + a.range_base + (c < a.range_rem ? 1 : 0);
+  row0 = r0 + s * a.slab_rows;
+  if (row0 >= r1) return false;
+  rows = min(a.slab_rows, r1 - row0);
+  return true;
+}
+
+// A ranged CTA's short last slab goes through tmWt and an MMA of N = tail_n.
+__device__ __forceinline__ bool lm_tn_is_tail(const LmArgs& a, int rows) {
+  return a.ranged && rows < a.slab_rows;
+}
 
 __device__ __forceinline__ void lm_tn_flush(const LmArgs& a, int b, int shard, float v, int id) {
   if (id >= 0) atomicMax(&a.keys[shard * a.B + b], make_key(v, id));
@@ -112,11 +142,15 @@ __global__ void __launch_bounds__(LmTn<kM>::kThreads, 1)
     if (lane == 0) {
       const uint64_t pol_w = ptx::policy_evict_first();
       const uint64_t pol_x = ptx::policy_evict_last();
-      const uint32_t bytes = static_cast<uint32_t>(kLmTnXBytes + a.slab_rows * kLmBK * 2);
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int slab = blockIdx.x; ok && slab < a.n_slabs; slab += gridDim.x) {
+      int row0, rows;
+      for (int s = 0; ok && lm_tn_slab(a, s, row0, rows); ++s) {
+        const bool tail = lm_tn_is_tail(a, rows);
+        const CUtensorMap* mw = tail ? &a.tmWt : &a.tmW;
+        const uint32_t bytes = static_cast<uint32_t>(
+            kLmTnXBytes + (tail ? a.tail_rows : a.slab_rows) * kLmBK * 2);
         for (int kb = 0; kb < a.k_iters; ++kb) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -125,8 +159,7 @@ __global__ void __launch_bounds__(LmTn<kM>::kThreads, 1)
           uint8_t* st = smem + stage * a.stage_bytes;
           ptx::mbar_arrive_expect_tx(&full[stage], bytes);
           ptx::tma_load_2d(st, &a.tmX, &full[stage], kb * kLmBK, 0, pol_x);
-          ptx::tma_load_2d(st + C::kABytes, &a.tmW, &full[stage], kb * kLmBK,
-                           slab * a.slab_rows, pol_w);
+          ptx::tma_load_2d(st + C::kABytes, mw, &full[stage], kb * kLmBK, row0, pol_w);
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -154,11 +187,14 @@ __global__ void __launch_bounds__(LmTn<kM>::kThreads, 1)
   } else if (warp == kMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = ptx::idesc_bf16(kM, a.slab_rows);
+      const uint32_t idesc_slab = ptx::idesc_bf16(kM, a.slab_rows);
+      const uint32_t idesc_tail = ptx::idesc_bf16(kM, a.ranged ? a.tail_n : a.slab_rows);
       int stage = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true, any_mma = false;
-      for (int slab = blockIdx.x; ok && slab < a.n_slabs; slab += gridDim.x, ++it) {
+      int row0, rows;
+      for (int s = 0; ok && lm_tn_slab(a, s, row0, rows); ++s, ++it) {
+        const uint32_t idesc = lm_tn_is_tail(a, rows) ? idesc_tail : idesc_slab;
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!ptx::mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -208,7 +244,8 @@ __global__ void __launch_bounds__(LmTn<kM>::kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     int it = 0;
     bool ok = true;
-    for (int slab = blockIdx.x; slab < a.n_slabs; slab += gridDim.x, ++it) {
+    int row0, rows;
+    for (int s = 0; lm_tn_slab(a, s, row0, rows); ++s, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       int w_ok = 1;
@@ -222,13 +259,13 @@ __global__ void __launch_bounds__(LmTn<kM>::kThreads, 1)
         break;
       }
       ptx::tc_fence_after();
-      const int slab0 = slab * a.slab_rows;
-      const int row_end = min(slab0 + a.slab_rows, a.V);  // ids at or past it are not this slab's
-      int cur = slab0 / a.shard;                           // shard of the running best
-      int next = (cur + 1) * a.shard;                      // first id of the next shard
+      const int slab0 = row0;
+      const int row_end = row0 + rows;  // ids at or past it are not this slab's
+      int cur = slab0 / a.shard;        // shard of the running best
+      int next = (cur + 1) * a.shard;   // first id of the next shard
       float best = 0.f;
       int best_id = -1;
-      for (int c = 0; c < a.slab_rows; c += 16) {
+      for (int c = 0; c < rows; c += 16) {
         uint32_t r[16];
         tmem_ld16(tmem_base + lane_base + static_cast<uint32_t>(acc * kLmTnAccCols + c), r);
         ptx::tmem_ld_wait();

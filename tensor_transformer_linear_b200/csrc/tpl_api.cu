@@ -921,29 +921,50 @@ tpl_status lmhead_prepare(const void* x, int64_t B, int64_t K, const void* w, in
   *smem = a->stages * a->stage_bytes + 1024 + 256 + tpl::kLmTbufBytes;
   *grid = std::min(a->n_slabs, dev->sm_count);
   if (B <= 32 && lmhead_tn_rows() != 0) {
-    // The batch as the M operand, vocab slabs of 16..256 rows (a multiple of
-    // 16) as N (lmhead_tn.cuh).  Slab height: the one that gives the busiest
-    // CTA the fewest vocab rows, the taller on a tie (fewer MMAs).  For
-    // V = 128256 on 148 SMs: 176 rows, 729 slabs, 880 rows on the busiest CTA.
+    // The batch as the M operand, vocab slabs as N (lmhead_tn.cuh).  An MMA
+    // costs about the same whatever its N, so by default every CTA owns one
+    // contiguous vocab range cut into 256-row slabs and one shorter last slab:
+    // for V = 128256 on 148 SMs, 866-867 rows per CTA in 3 x 256 + 98/99, so
+    // 4 x 256 MMAs per CTA instead of 5 x 256 with uniform slabs.
+    // TPL_LMHEAD_RANGES=0: uniform slabs of 16..256 rows (a multiple of 16)
+    // dealt out in turn, the height that gives the busiest CTA the fewest rows
+    // (176 rows, 729 slabs, 880 rows on the busiest CTA).
     const int64_t sms = dev->sm_count;
-    int64_t best_rows = INT64_MAX, best_r = 16;
-    for (int64_t r = 256; r >= 16; r -= 16) {
-      const int64_t slabs = (V + r - 1) / r;
-      const int64_t busiest = (slabs + sms - 1) / sms * r;
-      if (busiest < best_rows) {
-        best_rows = busiest;
-        best_r = r;
-      }
-    }
     a->tn = lmhead_tn_rows();
-    a->slab_rows = static_cast<int32_t>(best_r);
     const uint64_t wd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(V)};
     const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(B)};
     const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+    a->ranged = env_int("TPL_LMHEAD_RANGES", 1) != 0 ? 1 : 0;
+    if (a->ranged) {
+      const int64_t g = std::min<int64_t>(V, sms);
+      a->range_base = static_cast<int32_t>(V / g);
+      a->range_rem = static_cast<int32_t>(V % g);
+      a->slab_rows = 256;
+      // the longest last slab of any CTA (ranges of range_base or range_base + 1 rows)
+      int64_t tail = a->range_base % 256;
+      if (a->range_rem > 0 && (a->range_base + 1) % 256 > tail) tail = (a->range_base + 1) % 256;
+      a->tail_rows = static_cast<int32_t>(tail > 0 ? tail : 256);
+      a->tail_n = (a->tail_rows + 15) / 16 * 16;
+      if ((s = encode_bf16(&a->tmWt, w, 2, wd, str, static_cast<uint32_t>(a->tail_rows))) !=
+          TPL_OK)
+        return s;
+      a->n_slabs = static_cast<int32_t>(g);  // ranges, one per CTA
+    } else {
+      int64_t best_rows = INT64_MAX, best_r = 16;
+      for (int64_t r = 256; r >= 16; r -= 16) {
+        const int64_t slabs = (V + r - 1) / r;
+        const int64_t busiest = (slabs + sms - 1) / sms * r;
+        if (busiest < best_rows) {
+          best_rows = busiest;
+          best_r = r;
+        }
+      }
+      a->slab_rows = static_cast<int32_t>(best_r);
+      a->n_slabs = static_cast<int32_t>((V + a->slab_rows - 1) / a->slab_rows);
+    }
     if ((s = encode_bf16(&a->tmW, w, 2, wd, str, static_cast<uint32_t>(a->slab_rows))) != TPL_OK)
       return s;
     if ((s = encode_bf16(&a->tmX, x, 2, xd, str, 32u)) != TPL_OK) return s;
-    a->n_slabs = static_cast<int32_t>((V + a->slab_rows - 1) / a->slab_rows);
     // the A operand (a->tn rows) and the W tile
     a->stage_bytes = a->tn * tpl::kLmBK * 2 + (a->slab_rows * tpl::kLmBK * 2 + 1023) / 1024 * 1024;
     a->stages = std::min(tpl::kLmMaxStages, (227 * 1024 - 1024 - 256) / a->stage_bytes);
