@@ -295,6 +295,11 @@ LM_CASES = [
     (128, 256, 5000, 4, 2, True),       # one full 128-row batch tile
     (129, 128, 3000, 2, 3, True),       # two batch tiles, the second with one row
     (256, 192, 40000, 8, 4, True),      # two full batch tiles of 160 columns: one TMEM buffer
+    # vocab ranges of the transposed kernel on 148 SMs: 255-row ranges that are
+    # one short last slab next to 256-row ones that are one whole slab, and
+    # 512-row ranges with no short slab at all
+    (8, 64, 148 * 255 + 50, 4, 2, True),
+    (5, 128, 148 * 512, 8, 1, False),
 ]
 
 
