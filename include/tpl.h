@@ -43,6 +43,17 @@
  *     module-level variables per device, loaded with the library: the status
  *     word, the fixed scratch of tpl_lmhead_argmax_static and the pointer to
  *     an optional trace buffer (tpl_trace_set).  The calls are thread-safe.
+ *   - Environment variables (for measurements; results are the same under
+ *     every setting): TPL_PDL=0 launches without programmatic dependent
+ *     launch; TPL_GEMM_CTA_PAIRS=0 keeps every GEMM on single CTAs;
+ *     TPL_GEMM_GROUP_M and TPL_GEMM_KSERP set the CTA-pair GEMM's tile raster
+ *     (m-blocks per group, K order reversed on alternate tiles); TPL_LMHEAD_TN
+ *     picks the decode LM-head kernel for batches of up to 32 rows (2, the
+ *     default: the batch as a 64-row MMA operand; 1: a 128-row one; 0: the
+ *     swap-AB kernel that larger batches use) and TPL_LMHEAD_RANGES=0 gives
+ *     the transposed kernel uniform vocab slabs instead of one contiguous
+ *     range per CTA.  TPL_PDL and TPL_LMHEAD_TN are read once per process,
+ *     the others per call.
  */
 #ifndef TPL_H
 #define TPL_H
