@@ -404,15 +404,13 @@ class Block:
 
 
 class Stack:
-    """The 4-layer residual TP stack."""
+    """The 4-layer residual TP stack (or another MLPWorkload of residual layers)."""
 
-    name = C.STACK4.name
-
-    def __init__(self, dev):
+    def __init__(self, dev, w=C.STACK4):
         import tensor_transformer_linear_b200 as T
         self.T = T
-        w = C.STACK4
         self.w = w
+        self.name = w.name
         self.x0 = C.mlp_x(w, dev)
         self.x = self.x0.clone()
         self.io_in, self.io_out = ["x"], ["x"]   # the residual stream is updated in place
@@ -765,9 +763,8 @@ def oracle_job_block(parts=("qkv", "mlp", "lmhead"), rows_qkv=256, rows_mlp=96,
     return run, flops, ", ".join(desc)
 
 
-def oracle_job_stack(rows=8):
+def oracle_job_stack(rows=8, w=C.STACK4):
     import oracle as O
-    w = C.STACK4
     xs = _f64(gen.rows((w.M, w.hidden), _sample_rows(w.M, rows), 1.0, tensor_id=gen.TID_X))
     layers = [(C.mlp_w1(w, i).to(torch.float32).numpy(),
                C.mlp_w2(w, i).to(torch.float32).numpy()) for i in range(w.layers)]
@@ -810,6 +807,7 @@ def oracle_job_next(kind, rows=64):
 
 
 ORACLE_JOBS = {"block": oracle_job_block, "stack": oracle_job_stack,
+               "stack_layer": lambda: oracle_job_stack(w=C.STACK_LAYER),
                "qkv": lambda: oracle_job_block(("qkv",)),
                "mlp": lambda: oracle_job_block(("mlp",)),
                "lmhead": lambda: oracle_job_block(("lmhead",)),
@@ -821,7 +819,8 @@ ORACLE_JOBS = {"block": oracle_job_block, "stack": oracle_job_stack,
 # Workload names for the reference arm's line, without building the workload.
 WORKLOAD_NAMES = {
     "block": "tp-block: " + " + ".join((C.GQA_QKV.name, C.TP_MLP.name, C.LM_HEAD.name)),
-    "stack": C.STACK4.name, "qkv": C.GQA_QKV.name, "mlp": C.TP_MLP.name,
+    "stack": C.STACK4.name, "stack_layer": C.STACK_LAYER.name,
+    "qkv": C.GQA_QKV.name, "mlp": C.TP_MLP.name,
     "lmhead": C.LM_HEAD.name,
     "swiglu": "fused-swiglu-column x[8,1024,4096] bf16 4096->2x14336 tp8",
     "embed": "vocab-sharded-embedding ids[8,1024] W[128256,4096] bf16 tp8",
@@ -853,6 +852,7 @@ def workload_config(kind, world):
 
 
 WORKLOADS = {"block": Block, "stack": Stack,
+             "stack_layer": lambda dev: Stack(dev, C.STACK_LAYER),
              "qkv": lambda dev: Block(dev, ("qkv",)),
              "mlp": lambda dev: Block(dev, ("mlp",)),
              "lmhead": lambda dev: Block(dev, ("lmhead",)),

@@ -115,6 +115,14 @@ STACK4 = MLPWorkload("4-layer-tp-stack x[4,4096,8192] bf16 8192->28672->8192 tp8
                      w_sigma=0.01, dtype=torch.bfloat16, norm=True, norm_scale=False,
                      residual=True, layers=4)
 
+# One layer of the stack on a quarter of its tokens: the same two GEMM shapes in
+# K and N with about 1.3 GB on the device, small enough for a multi-pass
+# profiler capture.
+STACK_LAYER = MLPWorkload("1-layer-of-tp-stack x[1,4096,8192] bf16 8192->28672->8192 tp8 "
+                          "gelu-erf", batch=1, seq=4096, hidden=8192, inter=28672, tp=8,
+                          act="gelu_erf", w_sigma=0.01, dtype=torch.bfloat16, norm=True,
+                          norm_scale=False, residual=True, layers=1)
+
 ALL = (TINY_MLP, GQA_QKV, TP_MLP, LM_HEAD, STACK4)
 
 
