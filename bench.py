@@ -14,9 +14,11 @@ One step is one pass of the whole hot path over one batch of synthetic input
 
 ``value`` is the sharded-linear FLOP rate of the step (algorithmic FLOPs of
 the three contractions / step time).  ``--workload stack`` runs the 4-layer
-residual stack x[4,4096,8192], 8192->28672->8192 instead; the other workloads
-(``qkv``, ``mlp``, ``lmhead``, ``swiglu``, ``seqpar``, ``embed``, ``tp_ranks``)
-time one part or a next-step variant of the path.
+residual stack x[4,4096,8192], 8192->28672->8192 instead (``stack_layer``: one
+of its layers on x[1,4096,8192], the same GEMM shapes in K and N, small enough
+for a multi-pass profiler capture); the other workloads (``qkv``, ``mlp``,
+``lmhead``, ``swiglu``, ``seqpar``, ``embed``, ``tp_ranks``) time one part or a
+next-step variant of the path.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
 workload, on the host cores, without loading the CUDA library.  Under torchrun
