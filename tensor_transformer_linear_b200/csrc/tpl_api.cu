@@ -195,8 +195,19 @@ tpl_status launch_gemm(tpl::GemmArgs& a, int64_t M, DeviceInfo* dev, cudaStream_
   // bytes, 696 -> 686 us); row mode (K = 14336, a wave's operand blocks about
   // fill L2) with 8 m-blocks and the K order reversed on every other tile,
   // so consecutive waves meet in L2 (1.09 -> 0.96 GB read).
+  // Column mode on CTA pairs: the largest group (at most 16) whose A slabs fit
+  // in 32 MB, so they stay in L2 while the group sweeps its n-tiles: 16 at
+  // K = 4096, 8 at K = 8192 (the 4-layer stack, whose c_fc has K = 8192, ran at
+  // 1172 TFLOP/s with 8 and 1131 with 16).
   const bool row = a.mode == tpl::kModeRow;
-  a.group_m = env_int("TPL_GEMM_GROUP_M", (pairs && row) ? 8 : 16);
+  int group = 16;
+  if (pairs && row) {
+    group = 8;
+  } else if (pairs) {
+    const int64_t slab = static_cast<int64_t>(tpl::kPairBM) * a.k_iters * tpl::kBK * 2;
+    while (group > 1 && group * slab > (int64_t{32} << 20)) group /= 2;
+  }
+  a.group_m = env_int("TPL_GEMM_GROUP_M", group);
   a.k_serp = pairs ? env_int("TPL_GEMM_KSERP", row ? 1 : 0) : 0;
   const int64_t tiles = static_cast<int64_t>(a.m_blocks) * a.n_tiles;
   if (tiles > INT32_MAX) return TPL_ERR_SHAPE;
