@@ -147,6 +147,29 @@ def test_column_linear_many_pieces_two_launches():
         Bd.check(f64(g), r, e)
 
 
+def test_column_linear_raster_leaves_results_bitwise_equal(monkeypatch):
+    # The CTA-pair GEMM's raster (m-blocks per group, TPL_GEMM_GROUP_M, read per
+    # call) only reorders whole tiles; each tile's K sum runs in the same order,
+    # so every setting gives the same bits.  K = 8192 is where the library's own
+    # choice drops from 16 to 8 blocks per group.
+    subs, tp, M, K = [2048], 2, 1300, 8192
+    x = _t((M, K), 1.0, 0, seed=7).to(DEV)
+    w = _t((sum(subs), K), 0.01, 1, seed=7).to(DEV)
+    p = T.tpl_partition_subparams(subs, tp, 1)
+    outs = []
+    for g in ("", "1", "3", "16"):
+        monkeypatch.setenv("TPL_GEMM_GROUP_M", g)
+        outs.append(T.tpl_column_linear(p, x, w, None, "gelu_erf"))
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    part = O.partition_subparams(subs, tp, 1)
+    rows = [0, 1, 511, 512, 1299]
+    ref, own, _ = Bd.column(f64(x.cpu()[rows]), f64(w.cpu()), None, part, "gelu_erf")
+    for g, r, e in zip(T.shard_views(outs[0], p, M), ref, own):
+        Bd.check(f64(g[rows]), r, e)
+
+
 def test_column_linear_empty_rows():
     p = T.tpl_partition_subparams([256], 2, 1)
     x = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
